@@ -1,0 +1,400 @@
+"""Benchmark of the fused MoE layer forward (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config decode|prefill|fp8|skew|tiny]
+                    [--impl ours|reference] [--no-cpu-baseline]
+
+A step is one moe_forward over one batch of the workload's T tokens (router
+logits, top-k, permute, [FP8 activation quantisation], gate-up GEMM, down GEMM,
+combine), inputs resident in HBM.  K steps are timed on the device with CUDA
+events (barrier + synchronize on both sides), max over ranks.  Every rank
+runs its own replica on its own batch (tokens are independent given the
+weights, so the layer shards over tokens with no collective): "scaling" is
+"weak" and `value` = all ranks' tokens / the slowest rank's time.
+
+Extra keys: `roofline` (dominant kernel, from the events the library records
+at the stage boundaries inside the timed region), `cpu_baseline` (the FP64
+oracle on a bounded token sample, rank 0, N=1), `e2e` (the same metric through
+moe_forward_host: host->device copy of x, the layer, device->host copy of y,
+every step), `clocks` (nvidia-smi samples taken during the timed region),
+`gpu_launches` (kernels of this library launched in the timed region).
+
+`--impl reference` times the oracle (the plain FP64 CPU implementation) on
+the host cores instead, as the reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from expert_layer_dual_b200.configs import CONFIGS, MoEConfig  # noqa: E402
+from expert_layer_dual_b200.inputs import make_layer  # noqa: E402
+
+METRIC = "fused MoE layer tokens/s"
+UNIT = "tokens/s"
+# oracle token sample per step of the CPU baseline / reference arm
+CPU_SAMPLE = {"tiny": 16, "decode": 16, "prefill": 8, "fp8": 4, "skew": 8}
+
+
+def describe(cfg: MoEConfig) -> str:
+    s = f"{cfg.name}: T={cfg.T} d={cfg.d} E={cfg.E} top-{cfg.k}"
+    s += f" + shared I={cfg.I}" if cfg.Is else f" I={cfg.I}"
+    s += ", FP8 e4m3 128x128 block-scaled weights" if cfg.wdtype else ", BF16 weights"
+    if cfg.zipf_bias:
+        s += ", Zipf(1.2)-biased routing"
+    return s
+
+
+# ------------------------------------------------------------------ ranks
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world: int, backend: str):
+    if world > 1 and not torch.distributed.is_initialized():
+        import datetime
+        torch.distributed.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+
+
+def max_over_ranks(value: float, device) -> float:
+    """Largest value over all ranks (identity without a process group)."""
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier():
+    if torch.distributed.is_available() and torch.distributed.is_initialized():
+        torch.distributed.barrier()
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.gpu), "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        return parse_clock_samples(open(self.path).read().splitlines())
+
+
+def parse_clock_samples(lines):
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    sm, smax, reasons, power = [], [], set(), []
+    for ln in lines:
+        parts = [p.strip() for p in ln.split(",")]
+        if len(parts) < 9:
+            continue
+        try:
+            sm.append(float(parts[1]))
+            smax.append(float(parts[2]))
+            power.append(float(parts[3]))
+        except ValueError:
+            continue
+        for n, v in zip(names, parts[5:9]):
+            if v.lower() == "active":
+                reasons.add(n)
+    if not sm:
+        return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+    loaded = [s for s, p in zip(sm, power) if p > 0.3 * max(power)] or sm
+    return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(smax),
+            "power_w_max": max(power), "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------------ roofline
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p.get("hbm_gbs", 6650.0), p.get("bf16_tflops_sustained", 1397.0), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+def gateup_algorithmic(cfg: MoEConfig, T: int, n_active: int):
+    """Algorithmic work of one gate-up launch: FLOPs, and bytes = the weights
+    of every expert that received tokens (+ shared) read once, x read once,
+    h written once."""
+    R = T * cfg.k + (T if cfg.Is else 0)
+    wbytes = 1 if cfg.wdtype else 2
+    groups = n_active + (1 if cfg.Is else 0)
+    flops = 2.0 * R * cfg.d * 2 * cfg.I
+    byts = groups * 2 * cfg.I * cfg.d * wbytes + T * cfg.d * wbytes + R * cfg.I * wbytes
+    return flops, byts
+
+
+def down_algorithmic(cfg: MoEConfig, T: int, n_active: int):
+    R = T * cfg.k + (T if cfg.Is else 0)
+    wbytes = 1 if cfg.wdtype else 2
+    groups = n_active + (1 if cfg.Is else 0)
+    flops = 2.0 * R * cfg.I * cfg.d
+    byts = groups * cfg.d * cfg.I * wbytes + R * cfg.I * wbytes + R * cfg.d * 2
+    return flops, byts
+
+
+# ------------------------------------------------------------------ CPU oracle
+def _bits(t):
+    return t.detach().contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
+
+
+def oracle_sample_time(cfg: MoEConfig, inp: dict, n_tokens: int, repeats: int = 1):
+    """Seconds the oracle takes for the whole layer on n_tokens of the
+    workload (host copies made first, outside the timing)."""
+    import oracle
+    oracle.build()
+    n = min(n_tokens, cfg.T)
+    xs = _bits(inp["x"][:n])
+    rw = inp["router_w"].detach().cpu().numpy()
+    bias = None if inp.get("router_bias") is None else inp["router_bias"].cpu().numpy()
+    hi, lo = oracle.router_split(rw)
+    lg = oracle.router_logits(xs, hi, lo, bias)
+    need = np.unique(oracle.route_topk(lg.astype(np.float32), cfg.k)[0])
+    w_gu = np.empty((cfg.E, 2 * cfg.I, cfg.d), np.uint16)
+    w_d = np.empty((cfg.E, cfg.d, cfg.I), np.uint16)
+    for e in need:
+        w_gu[e] = _bits(inp["w_gu"][int(e)])
+        w_d[e] = _bits(inp["w_d"][int(e)])
+    L = oracle.Layer(T=n, d=cfg.d, E=cfg.E, k=cfg.k, I=cfg.I, Is=cfg.Is, w_gu=w_gu, w_d=w_d,
+                     ws_gu=None if inp.get("ws_gu") is None else _bits(inp["ws_gu"]),
+                     ws_d=None if inp.get("ws_d") is None else _bits(inp["ws_d"]),
+                     router_w=rw, router_bias=bias, wdtype=cfg.wdtype, renorm=cfg.renorm)
+    times = []
+    for _ in range(repeats):
+        t0 = time.perf_counter()
+        oracle.forward(L, xs)
+        times.append(time.perf_counter() - t0)
+    return times, n, oracle.num_threads()
+
+
+def run_reference(args, cfg: MoEConfig):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    inp = make_layer(cfg, device="cuda" if torch.cuda.is_available() else "cpu")
+    # size the per-step sample so the whole run stays within a few minutes
+    t1, _, _ = oracle_sample_time(cfg, inp, 1, repeats=1)
+    budget = 150.0 / (args.warmup + args.steps)
+    n = int(max(1, min(CPU_SAMPLE.get(cfg.name, 8), budget / max(t1[0], 1e-3))))
+    times, n, cores = oracle_sample_time(cfg, inp, n, repeats=args.warmup + args.steps)
+    timed = times[args.warmup:]
+    tps = n * len(timed) / sum(timed)
+    sample = f"{n} tokens of the {cfg.name} workload per step (whole layer, FP64)"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": tps, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sum(timed) / len(timed),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": describe(cfg)},
+        "cpu_baseline": {"value": tps, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": tps, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args, cfg: MoEConfig):
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    init_dist(world, "nccl")
+    dev = torch.device("cuda", local)
+    import expert_layer_dual_b200.moe as M
+
+    inp = make_layer(cfg, device=dev)
+    # each rank's own batch: same weights, a different draw of x
+    if rank > 0:
+        g = torch.Generator(device=dev).manual_seed(cfg.seed * 1000 + 500 + rank)
+        inp["x"] = torch.randn(inp["x"].shape, generator=g, device=dev).to(torch.bfloat16)
+    layer = M.MoELayer(cfg, inp, device=dev)
+    x = inp["x"]
+    y = torch.empty_like(x)
+    shape = layer.shape(cfg.T)
+    stream = torch.cuda.current_stream()
+
+    # routing statistics of this batch (outside the timed region)
+    logits = torch.empty((cfg.T, cfg.E), dtype=torch.float32, device=dev)
+    M.router_logits(x.view(torch.uint16), layer.router_hi, layer.router_lo, layer.router_bias, logits)
+    ids = torch.empty((cfg.T, cfg.k), dtype=torch.int32, device=dev)
+    wts = torch.empty((cfg.T, cfg.k), dtype=torch.float32, device=dev)
+    M.route_topk(logits, cfg.k, int(cfg.renorm), ids, wts)
+    counts = torch.bincount(ids.view(-1).long(), minlength=cfg.E)
+    n_active = int((counts > 0).sum().item())
+
+    nev = M.PROFILE_EVENTS
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(args.steps)]
+    for row in events:
+        for e in row:
+            e.record(stream)  # creates the event handles
+    warm = [torch.cuda.Event(enable_timing=True) for _ in range(nev)]
+    for e in warm:
+        e.record(stream)
+    for _ in range(args.warmup):
+        M.forward_profiled(shape, layer.weights, x.view(torch.uint16), y.view(torch.uint16), layer.ws, warm)
+    torch.cuda.synchronize()
+    if layer.device_status() != M.OK:
+        raise RuntimeError("device status after warm-up: " + M.status_string(layer.device_status()))
+
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        barrier()
+        torch.cuda.synchronize()
+        t_start.record(stream)
+        for i in range(args.steps):
+            M.forward_profiled(shape, layer.weights, x.view(torch.uint16), y.view(torch.uint16),
+                               layer.ws, events[i])
+        t_end.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    ms_total = t_start.elapsed_time(t_end)
+    ms_total = max_over_ranks(ms_total, dev)
+    ms_step = ms_total / args.steps
+    value = world * cfg.T * args.steps / (ms_total / 1e3)
+
+    stage_ms = {name: 0.0 for name in M.STAGES}
+    for row in events:
+        for j, name in enumerate(M.STAGES):
+            stage_ms[name] += row[j].elapsed_time(row[j + 1]) / args.steps
+    if layer.device_status() != M.OK:
+        raise RuntimeError("device status after timing: " + M.status_string(layer.device_status()))
+
+    # roofline of the dominant kernel (the gate-up GEMM)
+    hbm_peak, tflops_peak, peak_kind = load_peaks()
+    gu_ms = stage_ms["gemm_gateup"]
+    gu_flops, gu_bytes = gateup_algorithmic(cfg, cfg.T, n_active)
+    dn_flops, dn_bytes = down_algorithmic(cfg, cfg.T, n_active)
+    ai = gu_flops / gu_bytes
+    ridge = tflops_peak * 1e12 / (hbm_peak * 1e9) * (2 if cfg.wdtype else 1)
+    if ai < ridge:
+        roof = {"bound": "hbm", "achieved": gu_bytes / (gu_ms / 1e3) / 1e9, "peak": hbm_peak,
+                "unit": "GB/s"}
+    else:
+        peak = tflops_peak * (2 if cfg.wdtype else 1)
+        roof = {"bound": "tensor", "achieved": gu_flops / (gu_ms / 1e3) / 1e12, "peak": peak,
+                "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["kernel"] = "k_gateup_" + ("fp8" if cfg.wdtype else "bf16")
+    roof["peak_source"] = (f"{peak_kind} MEASURED_PEAKS.json "
+                           + ("hbm_gbs" if roof["bound"] == "hbm" else "bf16_tflops_sustained"
+                              + (" x2 (e4m3 nominal ratio)" if cfg.wdtype else "")))
+    roof["traffic"] = None
+    roof["algorithmic_bytes"] = gu_bytes
+    roof["algorithmic_flops"] = gu_flops
+    roof["launch_ms"] = gu_ms
+
+    # end to end through host buffers: copy x in, forward, copy y out, every step
+    xh = x.cpu().pin_memory()
+    yh = torch.empty_like(xh).pin_memory()
+    for _ in range(max(1, args.warmup)):
+        layer.forward_host(xh, yh)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.steps):
+        layer.forward_host(xh, yh)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
+    e2e = {"value": world * cfg.T * args.steps / (e2e_ms / 1e3), "unit": UNIT,
+           "h2d_bytes_per_step": xh.numel() * xh.element_size(),
+           "d2h_bytes_per_step": yh.numel() * yh.element_size()}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n = CPU_SAMPLE.get(cfg.name, 8)
+        times, n, cores = oracle_sample_time(cfg, inp, n, repeats=1)
+        cpu = {"value": n / times[0], "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": f"first {n} tokens of the {cfg.name} batch, whole layer in FP64 "
+                         f"({times[0]:.1f} s)"}
+
+    kernels_per_step = 8 + (1 if cfg.wdtype else 0)
+    if rank == 0:
+        out = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f8e4m3" if cfg.wdtype else "bf16",
+            "data": "synthetic",
+            "config": {"workload": describe(cfg), "tokens_per_gpu": cfg.T,
+                       "active_experts": n_active,
+                       "l2": "no flush: the expert weights read each step "
+                             f"({(gu_bytes + dn_bytes) / 1e9:.1f} GB) exceed the 126 MB L2",
+                       "parallelism": f"{world} independent replicas (tokens sharded, no collective)"},
+            "roofline": roof,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": kernels_per_step * args.steps,
+            "clocks": clocks.summary(),
+            "stages_ms": stage_ms,
+            "tflops": cfg.flops() / (ms_step / 1e3) / 1e12 * world,
+            "layer_weight_gbs": (gu_bytes + dn_bytes) / (ms_step / 1e3) / 1e9,
+        }
+        print(json.dumps(out), flush=True)
+    if torch.distributed.is_initialized():
+        torch.distributed.destroy_process_group()
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="decode", choices=sorted(CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    args.warmup = max(args.warmup, 3)  # at least 3 untimed warm-up steps, whatever is asked
+    cfg = CONFIGS[args.config]
+    if args.impl == "reference":
+        run_reference(args, cfg)
+    else:
+        run_ours(args, cfg)
+
+
+if __name__ == "__main__":
+    main()

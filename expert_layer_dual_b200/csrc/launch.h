@@ -1,0 +1,72 @@
+// launch.h -- host-side launchers of the MoE kernels (internal to the
+// library; the public ABI is include/moe.h).  Every launcher enqueues on
+// `stream` and returns the launch error, if any.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace moe {
+
+struct DevInfo {
+    int device;
+    int num_sms;
+    int cc_major, cc_minor;
+};
+
+// Cached per-device properties of the current device.
+const DevInfo& current_device_info();
+
+// ---- routing.cu
+cudaError_t launch_router_split(const float* W, uint16_t* hi, uint16_t* lo, int64_t n,
+                                cudaStream_t s);
+cudaError_t launch_route_topk(const float* logits, int T, int E, int k, int renorm, int32_t* ids,
+                              float* w, cudaStream_t s);
+// Scratch: seg_hist [nseg][E] int32, nseg = permute_segments(T*k).
+int permute_segments(int64_t n_assign);
+cudaError_t launch_permute(const int32_t* ids, int T, int E, int k, int32_t* counts,
+                           int32_t* offsets, int32_t* perm, int32_t* inv, int32_t* seg_hist,
+                           int32_t* status, cudaStream_t s);
+cudaError_t launch_combine(const uint16_t* o, const int32_t* inv, const float* w, uint16_t* y,
+                           int T, int d, int k, int has_shared, cudaStream_t s);
+cudaError_t launch_quant_act_fp8(const uint16_t* x, int64_t rows, int cols, uint8_t* q,
+                                 float* scale, cudaStream_t s);
+cudaError_t launch_quant_weights_fp8(const uint16_t* W, int64_t batch, int rows, int cols,
+                                     uint8_t* q, float* scale, cudaStream_t s);
+cudaError_t launch_selftest_timeout(int32_t* status, uint64_t limit_ns, cudaStream_t s);
+
+// ---- router.cu (tcgen05 dual-BF16 GEMM)
+cudaError_t launch_router_logits(const uint16_t* x, const uint16_t* hi, const uint16_t* lo,
+                                 const float* bias, float* logits, int T, int d, int E,
+                                 int32_t* status, cudaStream_t s);
+
+// ---- gemm_bf16.cu (tcgen05 grouped GEMMs)
+struct GroupedGemmArgs {
+    int T, d, E, k, I, has_shared;
+    const int32_t* offsets;  // [E+1]
+    const int32_t* perm;     // [T*k]
+    int32_t* status;
+    uint64_t timeout_ns;
+};
+cudaError_t launch_gateup_bf16(const GroupedGemmArgs& a, const uint16_t* x, const uint16_t* w_gu,
+                               const uint16_t* ws_gu, uint16_t* h, cudaStream_t s);
+cudaError_t launch_down_bf16(const GroupedGemmArgs& a, const uint16_t* h, const uint16_t* w_d,
+                             const uint16_t* ws_d, uint16_t* o, cudaStream_t s);
+
+// ---- gemm_fp8.cu (tcgen05 grouped GEMMs, e4m3 with 128x128 block scales)
+cudaError_t launch_gateup_fp8(const GroupedGemmArgs& a, const uint8_t* xq, const float* xs,
+                              const uint8_t* w_gu, const float* w_gu_s, const uint8_t* ws_gu,
+                              const float* ws_gu_s, uint8_t* hq, float* hs, cudaStream_t s);
+cudaError_t launch_down_fp8(const GroupedGemmArgs& a, const uint8_t* hq, const float* hs,
+                            const uint8_t* w_d, const float* w_d_s, const uint8_t* ws_d,
+                            const float* ws_d_s, uint16_t* o, cudaStream_t s);
+
+// ---- tensor maps (api.cu)
+// 2-D row-major tensor [rows][cols] of `elem_bytes`-sized elements, box
+// [box_rows][box_cols], 128-byte swizzle, zero fill out of bounds.
+bool make_tmap_2d(CUtensorMap* map, const void* base, int elem_bytes, uint64_t rows,
+                  uint64_t cols, uint32_t box_rows, uint32_t box_cols);
+
+}  // namespace moe

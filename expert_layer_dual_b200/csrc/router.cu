@@ -1,0 +1,176 @@
+// router.cu -- dual-BF16 router GEMM on the sm_100a tensor cores.
+//
+// "HPC-Ops - 騰訊混元開源的工業級高性能大模型推理算子庫", section HPC-Ops的技術原理,
+// paragraph "Router GEMM 雙 BF16 模擬 FP32": the FP32 router weight is split
+// offline into hi (BF16) and lo (BF16 residual, scale 1/256); at inference two
+// BF16 tensor-core GEMMs run in ONE kernel, the BF16 activations are moved
+// once, two accumulators hold the partial results and the epilogue applies a
+// single FMA (acc_hi + acc_lo / 256) before writing.
+//
+// B200 form: one CTA per 128-token x 64-expert tile.  A TMA warp streams the
+// x tile and the hi and lo tiles of each 64-wide k-block into a 4-stage
+// shared-memory ring (128-byte swizzle); one thread issues two tcgen05.mma per
+// 16-wide k-step, sharing the A descriptor, into two TMEM accumulators
+// (columns 0-63 hi, 64-127 lo); four epilogue warps read both accumulators
+// with tcgen05.ld and write FP32 logits.  Every wait is bounded.
+#include "common.cuh"
+#include "launch.h"
+
+namespace moe {
+namespace {
+
+constexpr int BM = 128, BN = 64, BK = 64, STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;
+constexpr int B_BYTES = BN * BK * 2;
+constexpr int STAGE_BYTES = A_BYTES + 2 * B_BYTES;
+constexpr int THREADS = 192;  // warps 0-3 epilogue, 4 MMA + TMEM owner, 5 TMA
+constexpr uint32_t TMEM_COLS = 128;
+constexpr size_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
+
+__global__ void __launch_bounds__(THREADS, 1)
+    k_router_dual(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_hi,
+                  const __grid_constant__ CUtensorMap tm_lo, const float* __restrict__ bias,
+                  float* __restrict__ logits, int T, int d, int E, int32_t* status,
+                  uint64_t timeout_ns) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+    uint64_t* empty = full + STAGES;
+    uint64_t* done = empty + STAGES;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int m0 = blockIdx.x * BM, e0 = blockIdx.y * BN;
+    const int nk = d / BK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(done, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 4) tmem_alloc(tmem_slot, TMEM_COLS);
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 5 && lane == 0) {
+        // ---------------- TMA producer
+        tma_prefetch_desc(&tm_x);
+        tma_prefetch_desc(&tm_hi);
+        tma_prefetch_desc(&tm_lo);
+        int issued = 0;
+        for (int kb = 0; kb < nk; ++kb) {
+            const int s = kb % STAGES;
+            const uint32_t ph = (kb / STAGES) & 1;
+            if (!mbar_wait(&empty[s], ph ^ 1, timeout_ns, abort_flag)) {
+                report_status(status, MOE_ERR_DEVICE_TIMEOUT);
+                *abort_flag = 1;
+                break;
+            }
+            uint8_t* st = smem + s * STAGE_BYTES;
+            mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
+            tma_load_2d(st, &tm_x, &full[s], kb * BK, m0);
+            tma_load_2d(st + A_BYTES, &tm_hi, &full[s], kb * BK, e0);
+            tma_load_2d(st + A_BYTES + B_BYTES, &tm_lo, &full[s], kb * BK, e0);
+            ++issued;
+        }
+        if (*abort_flag) {  // let the copies still in flight land before the block exits
+            for (int it = (issued > STAGES ? issued - STAGES : 0); it < issued; ++it)
+                mbar_wait(&full[it % STAGES], (it / STAGES) & 1, timeout_ns, nullptr);
+        }
+    } else if (warp == 4 && lane == 0) {
+        // ---------------- MMA issuer
+        constexpr uint32_t idesc = idesc_bf16(BM, BN);
+        for (int kb = 0; kb < nk; ++kb) {
+            const int s = kb % STAGES;
+            const uint32_t ph = (kb / STAGES) & 1;
+            if (!mbar_wait(&full[s], ph, timeout_ns, abort_flag)) {
+                report_status(status, MOE_ERR_DEVICE_TIMEOUT);
+                *abort_flag = 1;
+                break;
+            }
+            tc_fence_after_sync();
+            const uint32_t a = smem_u32(smem + s * STAGE_BYTES);
+            const uint32_t bh = a + A_BYTES, bl = a + A_BYTES + B_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk) {
+                const uint64_t ad = sdesc_k_sw128(a + kk * 32);
+                const uint32_t acc = (kb | kk) != 0;
+                umma_bf16(tmem, ad, sdesc_k_sw128(bh + kk * 32), idesc, acc);
+                umma_bf16(tmem + BN, ad, sdesc_k_sw128(bl + kk * 32), idesc, acc);
+            }
+            umma_commit(&empty[s]);
+        }
+        umma_commit(done);  // also on abort: arrives once the issued MMAs are done
+    } else if (warp < 4) {
+        // ---------------- epilogue: logit = fma(acc_lo, 1/256, acc_hi) + bias
+        const bool ok = mbar_wait(done, 0, timeout_ns, abort_flag);
+        if (!ok) {
+            report_status(status, MOE_ERR_DEVICE_TIMEOUT);
+            *abort_flag = 1;
+        }
+        tc_fence_after_sync();
+        if (ok && !*abort_flag) {
+            const int row = warp * 32 + lane;
+            const int t = m0 + row;
+            const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+#pragma unroll 1
+            for (int c = 0; c < BN / 32; ++c) {
+                float h[32], l[32];
+                tmem_load32x2(lane_base + c * 32, lane_base + BN + c * 32, h, l);
+                if (t < T) {
+                    float* dst = logits + (int64_t)t * E;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const int e = e0 + c * 32 + i;
+                        if (e < E) {
+                            float v = fmaf(l[i], 0.00390625f, h[i]);
+                            if (bias != nullptr) v += bias[e];
+                            dst[e] = v;
+                        }
+                    }
+                }
+            }
+        }
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 4) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_router_logits(const uint16_t* x, const uint16_t* hi, const uint16_t* lo,
+                                 const float* bias, float* logits, int T, int d, int E,
+                                 int32_t* status, cudaStream_t s) {
+    if (T == 0) return cudaSuccess;
+    CUtensorMap tx, th, tl;
+    if (!make_tmap_2d(&tx, x, 2, (uint64_t)T, (uint64_t)d, BM, BK) ||
+        !make_tmap_2d(&th, hi, 2, (uint64_t)E, (uint64_t)d, BN, BK) ||
+        !make_tmap_2d(&tl, lo, 2, (uint64_t)E, (uint64_t)d, BN, BK))
+        return cudaErrorInvalidValue;
+    static bool attr_set[64] = {false};
+    const int dev = current_device_info().device;
+    if (dev < 64 && !attr_set[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(k_router_dual, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        attr_set[dev] = true;
+    }
+    dim3 grid((T + BM - 1) / BM, (E + BN - 1) / BN);
+    k_router_dual<<<grid, THREADS, SMEM_BYTES, s>>>(tx, th, tl, bias, logits, T, d, E, status,
+                                                    kDefaultTimeoutNs);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,426 @@
+// routing.cu -- the non-GEMM stages of the MoE layer on sm_100a:
+// router weight split, top-k routing, per-expert count / scan / permute,
+// top-k weighted combine, FP8 quantisation of activations and weights.
+// All of them are HBM- or latency-bound; they use coalesced 16-byte or
+// warp-contiguous accesses and warp-level primitives, no tensor cores.
+//
+// Sources (page title -- section):
+//  "HPC-Ops - 騰訊混元開源的工業級高性能大模型推理算子庫":
+//    HPC-Ops的技術原理, "Router GEMM 雙 BF16 模擬 FP32" (the offline split);
+//    HPC-Ops的技術原理, "FusedMoE 流水線重構" (shared-memory blocked per-expert
+//      counting with one contiguous output interval per expert);
+//    HPC-Ops的主要功能, "FusedMoE" (activation quantisation, Top-K weighted
+//      aggregation) and "GroupGEMM FP8" (block-wise FP8).
+//  "PR #54160 完整报告", 功能与动机 (top-8 of 256 experts + 1 shared expert);
+//    实现拆解 item 4 (FP8 block-wise 128x128 scales).
+#include "common.cuh"
+#include "launch.h"
+
+namespace moe {
+
+// ---------------------------------------------------------------------------
+// Router weight split: hi = RNE_bf16(W); lo = RNE_bf16((W - hi) * 256).
+// W - hi is exact in FP32 and the scaling by 256 is exact, so both steps are
+// a single rounding.
+// ---------------------------------------------------------------------------
+__global__ void k_router_split(const float* __restrict__ W, uint16_t* __restrict__ hi,
+                               uint16_t* __restrict__ lo, int64_t n) {
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const float w = W[i];
+        const __nv_bfloat16 h = __float2bfloat16_rn(w);
+        const float r = w - __bfloat162float(h);
+        const __nv_bfloat16 l = __float2bfloat16_rn(r * 256.0f);
+        hi[i] = __bfloat16_as_ushort(h);
+        lo[i] = __bfloat16_as_ushort(l);
+    }
+}
+
+cudaError_t launch_router_split(const float* W, uint16_t* hi, uint16_t* lo, int64_t n,
+                                cudaStream_t s) {
+    if (n == 0) return cudaSuccess;
+    const int threads = 256;
+    int64_t blocks = (n + threads - 1) / threads;
+    const int cap = current_device_info().num_sms * 8;
+    if (blocks > cap) blocks = cap;
+    k_router_split<<<(unsigned)blocks, threads, 0, s>>>(W, hi, lo, n);
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Top-k routing: one warp per token; lane l holds logits l, l+32, ... (E <=
+// 256).  k rounds of a warp arg-max over (value desc, id asc) -- a total
+// order, so every lane converges to the same winner -- select the experts in
+// descending order with ties to the lower id.  Weights: softmax over the
+// selected logits (or over all E when renorm == 0), in FP32.
+// ---------------------------------------------------------------------------
+constexpr int kTopkWarps = 8;
+
+__global__ void __launch_bounds__(kTopkWarps * 32)
+    k_route_topk(const float* __restrict__ logits, int T, int E, int k, int renorm,
+                 int32_t* __restrict__ ids, float* __restrict__ w) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t = blockIdx.x * kTopkWarps + warp;
+    if (t >= T) return;
+    const float* l = logits + (int64_t)t * E;
+    float v[8];
+    uint32_t taken = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int e = lane + 32 * i;
+        v[i] = (e < E) ? l[e] : 0.0f;
+        if (e >= E) taken |= 1u << i;
+    }
+    float my_v = 0.0f;
+    int my_e = 0;
+    for (int j = 0; j < k; ++j) {
+        float bv = -INFINITY;
+        int be = 0x7fffffff;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            if (!((taken >> i) & 1u)) {
+                const int e = lane + 32 * i;
+                if (be == 0x7fffffff || v[i] > bv) {  // ids ascend with i: first max wins ties
+                    bv = v[i];
+                    be = e;
+                }
+            }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+            const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+            const bool other_better = (oe != 0x7fffffff) &&
+                                      (be == 0x7fffffff || ov > bv || (ov == bv && oe < be));
+            if (other_better) {
+                bv = ov;
+                be = oe;
+            }
+        }
+        if ((be & 31) == lane) taken |= 1u << (be >> 5);
+        if (lane == j) {
+            my_v = bv;
+            my_e = be;
+        }
+    }
+    const float lmax = __shfl_sync(0xffffffffu, my_v, 0);
+    float part = 0.0f;
+    if (renorm) {
+        if (lane < k) part = expf(my_v - lmax);
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            if (lane + 32 * i < E) part += expf(v[i] - lmax);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+    if (lane < k) {
+        ids[(int64_t)t * k + lane] = my_e;
+        w[(int64_t)t * k + lane] = expf(my_v - lmax) / part;
+    }
+}
+
+cudaError_t launch_route_topk(const float* logits, int T, int E, int k, int renorm, int32_t* ids,
+                              float* w, cudaStream_t s) {
+    if (T == 0) return cudaSuccess;
+    k_route_topk<<<(T + kTopkWarps - 1) / kTopkWarps, kTopkWarps * 32, 0, s>>>(logits, T, E, k,
+                                                                              renorm, ids, w);
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Count / scan / permute.  The flat assignment list a = t*k + j is cut into
+// segments of kSeg; (1) each block counts its segment's experts in a
+// shared-memory histogram; (2) one block turns the per-segment counts into
+// per-expert totals, the exclusive scan over experts (offsets) and, per
+// segment, the first output row of each expert; (3) each segment is placed
+// in order by one warp: __match_any_sync groups equal experts inside 32
+// consecutive assignments, the rank inside the group keeps the order stable.
+// No step depends on atomic ordering, so perm / inv are deterministic.
+// ---------------------------------------------------------------------------
+constexpr int kSeg = 1024;
+
+int permute_segments(int64_t n) { return (int)((n + kSeg - 1) / kSeg); }
+
+__global__ void __launch_bounds__(256)
+    k_perm_count(const int32_t* __restrict__ ids, int64_t n, int E, int32_t* __restrict__ seg_hist,
+                 int32_t* status) {
+    __shared__ int32_t hist[256];
+    for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+    __syncthreads();
+    const int64_t a0 = (int64_t)blockIdx.x * kSeg;
+    const int64_t a1 = (a0 + kSeg < n) ? a0 + kSeg : n;
+    for (int64_t a = a0 + threadIdx.x; a < a1; a += blockDim.x) {
+        const int e = ids[a];
+        if ((unsigned)e < (unsigned)E)
+            atomicAdd(&hist[e], 1);
+        else
+            report_status(status, MOE_ERR_DEVICE_BAD_INDEX);
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x)
+        seg_hist[(int64_t)blockIdx.x * E + e] = hist[e];
+}
+
+__global__ void __launch_bounds__(256)
+    k_perm_scan(int32_t* __restrict__ seg_hist, int nseg, int E, int32_t* __restrict__ counts,
+                int32_t* __restrict__ offsets) {
+    __shared__ int32_t buf[2][256];
+    const int e = threadIdx.x;
+    int32_t run = 0;
+    if (e < E) {
+        for (int s = 0; s < nseg; ++s) {
+            const int32_t c = seg_hist[(int64_t)s * E + e];
+            seg_hist[(int64_t)s * E + e] = run;
+            run += c;
+        }
+        counts[e] = run;
+    }
+    // inclusive Hillis-Steele scan of the totals over the 256 lanes
+    int cur = 0;
+    buf[0][e] = (e < E) ? run : 0;
+    __syncthreads();
+    for (int off = 1; off < 256; off <<= 1) {
+        const int32_t x = buf[cur][e] + (e >= off ? buf[cur][e - off] : 0);
+        buf[cur ^ 1][e] = x;
+        cur ^= 1;
+        __syncthreads();
+    }
+    const int32_t excl = buf[cur][e] - ((e < E) ? run : 0);
+    if (e < E) {
+        offsets[e] = excl;
+        if (e == E - 1) offsets[E] = excl + run;
+        for (int s = 0; s < nseg; ++s) seg_hist[(int64_t)s * E + e] += excl;
+    }
+}
+
+__global__ void __launch_bounds__(32)
+    k_perm_scatter(const int32_t* __restrict__ ids, int64_t n, int E,
+                   const int32_t* __restrict__ seg_base, int32_t* __restrict__ perm,
+                   int32_t* __restrict__ inv) {
+    __shared__ int32_t cur[256];
+    const int lane = threadIdx.x;
+    for (int e = lane; e < E; e += 32) cur[e] = seg_base[(int64_t)blockIdx.x * E + e];
+    __syncwarp();
+    const int64_t a0 = (int64_t)blockIdx.x * kSeg;
+    const int64_t a1 = (a0 + kSeg < n) ? a0 + kSeg : n;
+    for (int64_t base = a0; base < a1; base += 32) {
+        const int64_t a = base + lane;
+        const int e = (a < a1) ? ids[a] : -1;
+        const bool ok = (unsigned)e < (unsigned)E;
+        const unsigned peers = __match_any_sync(0xffffffffu, ok ? e : -1 - lane);
+        int32_t start = 0;
+        if (ok) {
+            start = cur[e];
+            const int32_t pos = start + __popc(peers & ((1u << lane) - 1u));
+            perm[pos] = (int32_t)a;
+            inv[a] = pos;
+        }
+        __syncwarp();
+        if (ok && lane == __ffs(peers) - 1) cur[e] = start + __popc(peers);
+        __syncwarp();
+    }
+}
+
+cudaError_t launch_permute(const int32_t* ids, int T, int E, int k, int32_t* counts,
+                           int32_t* offsets, int32_t* perm, int32_t* inv, int32_t* seg_hist,
+                           int32_t* status, cudaStream_t s) {
+    const int64_t n = (int64_t)T * k;
+    const int nseg = permute_segments(n);
+    if (nseg > 0) {
+        k_perm_count<<<nseg, 256, 0, s>>>(ids, n, E, seg_hist, status);
+    }
+    k_perm_scan<<<1, 256, 0, s>>>(seg_hist, nseg, E, counts, offsets);
+    if (nseg > 0) {
+        k_perm_scatter<<<nseg, 32, 0, s>>>(ids, n, E, seg_hist, perm, inv);
+    }
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Combine: y[t] = sum_j w[t][j] * o[inv[t*k+j]] + o[T*k+t], FP32 sum in the
+// order j = 0..k-1 then the shared row, one bf16 rounding.  One block per
+// token, 16-byte loads along d.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float* f) {
+    const uint32_t r[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(r[i] << 16);
+        f[2 * i + 1] = __uint_as_float(r[i] & 0xffff0000u);
+    }
+}
+
+__global__ void __launch_bounds__(128)
+    k_combine(const uint16_t* __restrict__ o, const int32_t* __restrict__ inv,
+              const float* __restrict__ w, uint16_t* __restrict__ y, int T, int d, int k,
+              int has_shared) {
+    __shared__ int32_t rows[8];
+    __shared__ float wts[8];
+    const int t = blockIdx.x;
+    if (threadIdx.x < k) {
+        rows[threadIdx.x] = inv[(int64_t)t * k + threadIdx.x];
+        wts[threadIdx.x] = w[(int64_t)t * k + threadIdx.x];
+    }
+    __syncthreads();
+    const int64_t shared_row = (int64_t)T * k + t;
+    for (int c = threadIdx.x * 8; c < d; c += blockDim.x * 8) {
+        float acc[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+        for (int j = 0; j < k; ++j) {
+            const uint4 u = __ldg(reinterpret_cast<const uint4*>(o + (int64_t)rows[j] * d + c));
+            float f[8];
+            bf16x8_to_f32(u, f);
+            const float wj = wts[j];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[i] = fmaf(wj, f[i], acc[i]);
+        }
+        if (has_shared) {
+            const uint4 u = __ldg(reinterpret_cast<const uint4*>(o + shared_row * d + c));
+            float f[8];
+            bf16x8_to_f32(u, f);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[i] += f[i];
+        }
+        uint4 out;
+        out.x = pack_bf16x2(acc[0], acc[1]);
+        out.y = pack_bf16x2(acc[2], acc[3]);
+        out.z = pack_bf16x2(acc[4], acc[5]);
+        out.w = pack_bf16x2(acc[6], acc[7]);
+        *reinterpret_cast<uint4*>(y + (int64_t)t * d + c) = out;
+    }
+}
+
+cudaError_t launch_combine(const uint16_t* o, const int32_t* inv, const float* w, uint16_t* y,
+                           int T, int d, int k, int has_shared, cudaStream_t s) {
+    if (T == 0) return cudaSuccess;
+    k_combine<<<T, 128, 0, s>>>(o, inv, w, y, T, d, k, has_shared);
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// FP8 e4m3 quantisation.  One group (1x128 of an activation row, or a 128x128
+// weight block): s = fp32(amax) / 448 (amax == 0 -> 1); q = e4m3 of
+// fp32(v / s), round to nearest even, saturating to +-448.  The divisions are
+// IEEE round-to-nearest (__fdiv_rn), the conversion is the hardware
+// cvt.rn.satfinite: the same decision the oracle takes in FP32.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t quant4_e4m3(float a, float b, float c, float d, float s) {
+    const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(
+        make_float2(__fdiv_rn(a, s), __fdiv_rn(b, s)), __NV_SATFINITE, __NV_E4M3);
+    const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(
+        make_float2(__fdiv_rn(c, s), __fdiv_rn(d, s)), __NV_SATFINITE, __NV_E4M3);
+    return (uint32_t)lo | ((uint32_t)hi << 16);
+}
+
+__device__ __forceinline__ float group_scale(float amax) {
+    return amax == 0.0f ? 1.0f : __fdiv_rn(amax, 448.0f);
+}
+
+// one warp per (row, 128-column group); lane holds 4 consecutive values
+__global__ void __launch_bounds__(256)
+    k_quant_act(const uint16_t* __restrict__ x, int64_t rows, int cols, uint8_t* __restrict__ q,
+                float* __restrict__ scale) {
+    const int64_t gw = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    const int groups = cols / 128;
+    if (gw >= rows * groups) return;
+    const int64_t r = gw / groups;
+    const int g = (int)(gw % groups);
+    const int64_t off = r * cols + g * 128 + lane * 4;
+    const uint2 raw = *reinterpret_cast<const uint2*>(x + off);
+    const float v0 = __uint_as_float(raw.x << 16), v1 = __uint_as_float(raw.x & 0xffff0000u);
+    const float v2 = __uint_as_float(raw.y << 16), v3 = __uint_as_float(raw.y & 0xffff0000u);
+    float amax = fmaxf(fmaxf(fabsf(v0), fabsf(v1)), fmaxf(fabsf(v2), fabsf(v3)));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const float s = group_scale(amax);
+    *reinterpret_cast<uint32_t*>(q + off) = quant4_e4m3(v0, v1, v2, v3, s);
+    if (lane == 0) scale[r * groups + g] = s;
+}
+
+cudaError_t launch_quant_act_fp8(const uint16_t* x, int64_t rows, int cols, uint8_t* q,
+                                 float* scale, cudaStream_t s) {
+    const int64_t warps = rows * (cols / 128);
+    if (warps == 0) return cudaSuccess;
+    const int64_t blocks = (warps + 7) / 8;
+    k_quant_act<<<(unsigned)blocks, 256, 0, s>>>(x, rows, cols, q, scale);
+    return cudaGetLastError();
+}
+
+// one block of 256 threads per 128x128 block; thread = half a row (64 values)
+__global__ void __launch_bounds__(256)
+    k_quant_w(const uint16_t* __restrict__ W, int rows, int cols, uint8_t* __restrict__ q,
+              float* __restrict__ scale) {
+    __shared__ float red[8];
+    const int rb = rows / 128, cb = cols / 128;
+    const int64_t blk = blockIdx.x;
+    const int64_t b = blk / ((int64_t)rb * cb);
+    const int r0 = (int)((blk / cb) % rb) * 128, c0 = (int)(blk % cb) * 128;
+    const int rr = threadIdx.x >> 1, half = threadIdx.x & 1;
+    const int64_t off = (b * rows + r0 + rr) * (int64_t)cols + c0 + half * 64;
+    uint4 u[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) u[i] = *reinterpret_cast<const uint4*>(W + off + i * 8);
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        float f[8];
+        bf16x8_to_f32(u[i], f);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(f[j]));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+    __syncthreads();
+    amax = red[0];
+#pragma unroll
+    for (int i = 1; i < 8; ++i) amax = fmaxf(amax, red[i]);
+    const float s = group_scale(amax);
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+        float f[16];
+        bf16x8_to_f32(u[i], f);
+        bf16x8_to_f32(u[i + 1], f + 8);
+        uint4 o;
+        o.x = quant4_e4m3(f[0], f[1], f[2], f[3], s);
+        o.y = quant4_e4m3(f[4], f[5], f[6], f[7], s);
+        o.z = quant4_e4m3(f[8], f[9], f[10], f[11], s);
+        o.w = quant4_e4m3(f[12], f[13], f[14], f[15], s);
+        *reinterpret_cast<uint4*>(q + off + i * 8) = o;
+    }
+    if (threadIdx.x == 0) scale[blk] = s;
+}
+
+cudaError_t launch_quant_weights_fp8(const uint16_t* W, int64_t batch, int rows, int cols,
+                                     uint8_t* q, float* scale, cudaStream_t s) {
+    const int64_t blocks = batch * (rows / 128) * (cols / 128);
+    if (blocks == 0) return cudaSuccess;
+    k_quant_w<<<(unsigned)blocks, 256, 0, s>>>(W, rows, cols, q, scale);
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Failure-path check: one thread waits on a barrier that nothing arrives at,
+// gives up after limit_ns and records the timeout.
+// ---------------------------------------------------------------------------
+__global__ void k_selftest_timeout(int32_t* status, uint64_t limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        if (!mbar_wait(&bar, 0, limit_ns, nullptr)) report_status(status, MOE_ERR_DEVICE_TIMEOUT);
+    }
+}
+
+cudaError_t launch_selftest_timeout(int32_t* status, uint64_t limit_ns, cudaStream_t s) {
+    k_selftest_timeout<<<1, 32, 0, s>>>(status, limit_ns);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,270 @@
+"""ctypes binding of libmoe_b200.so (the C ABI in include/moe.h).
+
+Argument marshalling only: every function here hands device pointers, sizes
+and the current CUDA stream to the entry point of the same name and raises
+``MoEError`` on a non-zero status.  All arithmetic runs in the library's
+CUDA kernels; there is no CPU path.  PyTorch supplies device memory and
+streams.
+
+Loading fails loudly: importing this module raises ``ImportError`` when the
+shared library has not been built (``python -m expert_layer_dual_b200.build``).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+from .configs import MoEConfig
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m expert_layer_dual_b200.build`")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+OK, INVALID_ARG, UNSUPPORTED, CUDA_ERROR, WORKSPACE_TOO_SMALL, DEVICE_TIMEOUT, DEVICE_BAD_INDEX = range(7)
+WDTYPE_BF16, WDTYPE_FP8_BLOCK128 = 0, 1
+
+EXPORTS = ["moe_status_string", "moe_workspace_bytes", "moe_permute_workspace_bytes",
+           "moe_router_split", "moe_quantize_weights_fp8", "moe_quantize_act_fp8",
+           "moe_router_logits", "moe_route_topk", "moe_permute", "moe_gemm_gateup",
+           "moe_gemm_down", "moe_combine", "moe_forward", "moe_forward_profiled", "moe_forward_host",
+           "moe_read_device_status", "moe_selftest_timeout"]
+
+
+class moe_shape(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int32), ("d", ctypes.c_int32), ("E", ctypes.c_int32),
+                ("k", ctypes.c_int32), ("I", ctypes.c_int32), ("I_shared", ctypes.c_int32),
+                ("wdtype", ctypes.c_int32), ("renormalize", ctypes.c_int32)]
+
+
+class moe_weights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("w_gu", "w_d", "w_gu_scale", "w_d_scale", "ws_gu", "ws_d", "ws_gu_scale",
+                 "ws_d_scale", "router_hi", "router_lo", "router_bias")]
+
+
+_vp, _i32, _i64, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+_S, _W = ctypes.POINTER(moe_shape), ctypes.POINTER(moe_weights)
+_sig = {
+    "moe_status_string": (ctypes.c_char_p, [_i32]),
+    "moe_workspace_bytes": (_sz, [_S]),
+    "moe_permute_workspace_bytes": (_sz, [_i32, _i32, _i32]),
+    "moe_router_split": (_i32, [_vp, _vp, _vp, _i64, _vp]),
+    "moe_quantize_weights_fp8": (_i32, [_vp, _i64, _i32, _i32, _vp, _vp, _vp]),
+    "moe_quantize_act_fp8": (_i32, [_vp, _i64, _i32, _vp, _vp, _vp]),
+    "moe_router_logits": (_i32, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _vp]),
+    "moe_route_topk": (_i32, [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
+    "moe_permute": (_i32, [_vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "moe_gemm_gateup": (_i32, [_S, _W, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "moe_gemm_down": (_i32, [_S, _W, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "moe_combine": (_i32, [_S, _vp, _vp, _vp, _vp, _vp]),
+    "moe_forward": (_i32, [_S, _W, _vp, _vp, _vp, _sz, _vp]),
+    "moe_forward_profiled": (_i32, [_S, _W, _vp, _vp, _vp, _sz, _vp, ctypes.POINTER(_vp), _i32]),
+    "moe_forward_host": (_i32, [_S, _W, _vp, _vp, _vp, _sz, _vp]),
+    "moe_read_device_status": (_i32, [_vp, _vp]),
+    "moe_selftest_timeout": (_i32, [_vp, _i32, _vp]),
+}
+for _name, (_res, _args) in _sig.items():
+    _f = getattr(_lib, _name)
+    _f.restype, _f.argtypes = _res, _args
+
+
+class MoEError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {status_string(code)} (status {code})")
+
+
+def status_string(code: int) -> str:
+    return _lib.moe_status_string(code).decode()
+
+
+def _check(code: int, where: str) -> None:
+    if code != OK:
+        raise MoEError(code, where)
+
+
+def _p(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if t.numel() and not t.is_contiguous():
+        raise ValueError("tensors passed to the MoE library must be contiguous")
+    return ctypes.c_void_p(t.data_ptr()) if t.numel() else None
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def shape_of(cfg: MoEConfig, T: Optional[int] = None) -> moe_shape:
+    return moe_shape(cfg.T if T is None else T, cfg.d, cfg.E, cfg.k, cfg.I, cfg.Is, cfg.wdtype,
+                     int(cfg.renorm))
+
+
+# ------------------------------------------------------------------ entry points
+def workspace_bytes(shape: moe_shape) -> int:
+    return int(_lib.moe_workspace_bytes(ctypes.byref(shape)))
+
+
+def permute_workspace_bytes(T: int, E: int, k: int) -> int:
+    return int(_lib.moe_permute_workspace_bytes(T, E, k))
+
+
+def router_split(W, hi, lo, stream=None):
+    _check(_lib.moe_router_split(_p(W), _p(hi), _p(lo), W.numel(), _stream(stream)), "moe_router_split")
+
+
+def quantize_weights_fp8(W, q, scale, stream=None):
+    rows, cols = W.shape[-2:]
+    batch = W.numel() // (rows * cols) if W.numel() else 0
+    _check(_lib.moe_quantize_weights_fp8(_p(W), batch, rows, cols, _p(q), _p(scale), _stream(stream)),
+           "moe_quantize_weights_fp8")
+
+
+def quantize_act_fp8(x, q, scale, stream=None):
+    rows, cols = x.shape
+    _check(_lib.moe_quantize_act_fp8(_p(x), rows, cols, _p(q), _p(scale), _stream(stream)),
+           "moe_quantize_act_fp8")
+
+
+def router_logits(x, hi, lo, bias, logits, stream=None):
+    T, d = x.shape
+    _check(_lib.moe_router_logits(_p(x), _p(hi), _p(lo), _p(bias), _p(logits), T, d, hi.shape[0],
+                                  _stream(stream)), "moe_router_logits")
+
+
+def route_topk(logits, k, renormalize, ids, w, stream=None):
+    T, E = logits.shape
+    _check(_lib.moe_route_topk(_p(logits), T, E, k, int(renormalize), _p(ids), _p(w), _stream(stream)),
+           "moe_route_topk")
+
+
+def permute(ids, E, counts, offsets, perm, inv, ws, stream=None):
+    T, k = ids.shape
+    _check(_lib.moe_permute(_p(ids), T, E, k, _p(counts), _p(offsets), _p(perm), _p(inv), _p(ws),
+                            ws.numel() * ws.element_size(), _stream(stream)), "moe_permute")
+
+
+def gemm_gateup(shape, weights, x, x_scale, perm, offsets, h, h_scale, ws, stream=None):
+    _check(_lib.moe_gemm_gateup(ctypes.byref(shape), ctypes.byref(weights), _p(x), _p(x_scale),
+                                _p(perm), _p(offsets), _p(h), _p(h_scale), _p(ws),
+                                ws.numel() * ws.element_size(), _stream(stream)), "moe_gemm_gateup")
+
+
+def gemm_down(shape, weights, h, h_scale, offsets, o, ws, stream=None):
+    _check(_lib.moe_gemm_down(ctypes.byref(shape), ctypes.byref(weights), _p(h), _p(h_scale),
+                              _p(offsets), _p(o), _p(ws), ws.numel() * ws.element_size(),
+                              _stream(stream)), "moe_gemm_down")
+
+
+def combine(shape, o, inv, w, y, stream=None):
+    _check(_lib.moe_combine(ctypes.byref(shape), _p(o), _p(inv), _p(w), _p(y), _stream(stream)),
+           "moe_combine")
+
+
+def forward(shape, weights, x, y, ws, stream=None):
+    _check(_lib.moe_forward(ctypes.byref(shape), ctypes.byref(weights), _p(x), _p(y), _p(ws),
+                            ws.numel() * ws.element_size(), _stream(stream)), "moe_forward")
+
+
+PROFILE_EVENTS = 8
+STAGES = ["router_logits", "route_topk", "permute", "quant_act", "gemm_gateup", "gemm_down", "combine"]
+
+
+def forward_profiled(shape, weights, x, y, ws, events, stream=None):
+    """moe_forward recording `events` (8 torch.cuda.Event(enable_timing=True),
+    already recorded once so their handles exist) at the stage boundaries."""
+    arr = (_vp * PROFILE_EVENTS)(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    _check(_lib.moe_forward_profiled(ctypes.byref(shape), ctypes.byref(weights), _p(x), _p(y), _p(ws),
+                                     ws.numel() * ws.element_size(), _stream(stream), arr,
+                                     PROFILE_EVENTS), "moe_forward_profiled")
+
+
+def forward_host(shape, weights, x_host, y_host, ws, stream=None):
+    _check(_lib.moe_forward_host(ctypes.byref(shape), ctypes.byref(weights), _p(x_host), _p(y_host),
+                                 _p(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "moe_forward_host")
+
+
+def read_device_status(ws, stream=None) -> int:
+    return int(_lib.moe_read_device_status(_p(ws), _stream(stream)))
+
+
+def selftest_timeout(ws, limit_us: int, stream=None):
+    _check(_lib.moe_selftest_timeout(_p(ws), int(limit_us), _stream(stream)), "moe_selftest_timeout")
+
+
+# ------------------------------------------------------------------ layer object
+class MoELayer:
+    """One MoE layer resident on the GPU: weights in the library's layout,
+    a workspace, and `forward(x) -> y` through moe_forward.
+
+    `inputs` holds the BF16 expert weights and the FP32 router weight (as
+    drawn by expert_layer_dual_b200.inputs.make_layer).  Preparation runs the
+    library's offline kernels: the dual-BF16 router split and, for FP8
+    layers, the 128x128 block quantisation of every expert matrix."""
+
+    def __init__(self, cfg: MoEConfig, inputs: dict, device="cuda", max_tokens: Optional[int] = None):
+        self.cfg = cfg
+        dev = torch.device(device)
+        self.max_tokens = cfg.T if max_tokens is None else max_tokens
+        E, d = cfg.E, cfg.d
+        rw = inputs["router_w"].to(dev, torch.float32).contiguous()
+        self.router_hi = torch.empty((E, d), dtype=torch.uint16, device=dev)
+        self.router_lo = torch.empty((E, d), dtype=torch.uint16, device=dev)
+        router_split(rw, self.router_hi, self.router_lo)
+        self.router_bias = None if inputs.get("router_bias") is None else \
+            inputs["router_bias"].to(dev, torch.float32).contiguous()
+        self.scales = {}
+        self.mats = {}
+        for name in ("w_gu", "w_d", "ws_gu", "ws_d"):
+            t = inputs.get(name)
+            if t is None:
+                self.mats[name] = None
+                self.scales[name] = None
+                continue
+            t = t.to(dev, torch.bfloat16).contiguous()
+            if cfg.wdtype == WDTYPE_FP8_BLOCK128:
+                q = torch.empty(t.shape, dtype=torch.uint8, device=dev)
+                s = torch.empty(t.shape[:-2] + (t.shape[-2] // 128, t.shape[-1] // 128),
+                                dtype=torch.float32, device=dev)
+                quantize_weights_fp8(t.view(torch.uint16), q, s)
+                self.mats[name], self.scales[name] = q, s
+            else:
+                self.mats[name], self.scales[name] = t.view(torch.uint16), None
+        self.weights = moe_weights(*[_p(v) for v in (
+            self.mats["w_gu"], self.mats["w_d"], self.scales["w_gu"], self.scales["w_d"],
+            self.mats["ws_gu"], self.mats["ws_d"], self.scales["ws_gu"], self.scales["ws_d"],
+            self.router_hi, self.router_lo, self.router_bias)])
+        nbytes = workspace_bytes(shape_of(cfg, self.max_tokens))
+        if nbytes == 0:
+            raise MoEError(UNSUPPORTED, "moe_workspace_bytes")
+        self.ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+
+    def shape(self, T: int) -> moe_shape:
+        if T > self.max_tokens:
+            raise ValueError(f"T={T} exceeds the layer's max_tokens={self.max_tokens}")
+        return shape_of(self.cfg, T)
+
+    def forward(self, x: torch.Tensor, y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        if y is None:
+            y = torch.empty_like(x)
+        forward(self.shape(x.shape[0]), self.weights, x.view(torch.uint16), y.view(torch.uint16),
+                self.ws, stream)
+        return y
+
+    def forward_host(self, x_host: torch.Tensor, y_host: torch.Tensor, stream=None) -> torch.Tensor:
+        forward_host(self.shape(x_host.shape[0]), self.weights, x_host.view(torch.uint16),
+                     y_host.view(torch.uint16), self.ws, stream)
+        return y_host
+
+    def device_status(self, stream=None) -> int:
+        return read_device_status(self.ws, stream)

@@ -1,0 +1,223 @@
+/* moe.h -- C ABI of the B200 (sm_100a) fused Mixture-of-Experts layer forward.
+ *
+ *   y = sum_{j<k} w[t][j] * E_{ids[t][j]}(x[t]) + S(x[t])
+ *   E_e(x) = (silu(x Wg_e^T) * (x Wu_e^T)) Wd_e^T,  silu(z) = z / (1 + e^-z)
+ *
+ * Sources (page title -- section):
+ *  [RG] "HPC-Ops - 騰訊混元開源的工業級高性能大模型推理算子庫", HPC-Ops的技術原理,
+ *       "Router GEMM 雙 BF16 模擬 FP32": the FP32 router weight is split
+ *       offline into a BF16 high part and a BF16 low residual with scale 1/256;
+ *       inference runs both BF16 GEMMs in one kernel, the activations stay
+ *       BF16 and are moved once, two accumulators, one FMA in the epilogue.
+ *  [FM] same page, HPC-Ops的主要功能, "FusedMoE": routing index -> Gate-Up
+ *       GEMM -> activation quantisation -> Down GEMM -> Top-K weighted
+ *       aggregation.
+ *  [FP] same page, HPC-Ops的技術原理, "FusedMoE 流水線重構": shared-memory
+ *       blocked per-expert counting, one contiguous output interval per
+ *       expert; Gate-Up reads the original input through the routing index.
+ *  [G8] same page, HPC-Ops的主要功能, "GroupGEMM FP8": grouped expert GEMM with
+ *       block-wise FP8 quantisation.
+ *  [HY] "PR #54160 完整报告" ([Hy4] support Hy4-preview model), 功能与动机:
+ *       256 routed experts, top-8, one shared expert; 实现拆解 item 4: FP8
+ *       block-wise 128x128 weight scales.
+ *
+ * Conventions shared by every entry point
+ *  - Pointers are DEVICE memory owned by the caller unless a comment says
+ *    HOST.  The library never allocates, frees or synchronises, except where
+ *    an entry point says so (moe_forward_host, moe_read_device_status).
+ *  - Layouts are row-major and contiguous.  BF16 travels as uint16_t bits,
+ *    FP8 e4m3 as uint8_t codes, scales as float.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Work is enqueued asynchronously in stream order; nothing
+ *    reads back counts, so a forward can be captured in a CUDA graph.
+ *  - Arguments are validated on the host before any launch.  A failed check
+ *    returns MOE_ERR_INVALID_ARG (null pointer, negative size, bad
+ *    workspace alignment) or MOE_ERR_UNSUPPORTED (a shape outside the
+ *    limits below, or no sm_100 device); nothing is launched then.  There is
+ *    no fallback path.  T == 0 is a valid no-op.
+ *  - Shape limits: d % 128 == 0, I % 128 == 0, I_shared in {0, I},
+ *    1 <= E <= 256, 1 <= k <= min(E, 8), T*k + T < 2^31.
+ *  - A launch failure returns MOE_ERR_CUDA.  Errors found on the device (an
+ *    expert id out of range, a bounded wait that ran out) are written into a
+ *    status word at the start of the workspace; moe_read_device_status()
+ *    returns it.  Each entry point that takes a workspace clears that word
+ *    first, so it reports the most recent such call.
+ *  - Inputs must be finite; NaN logits give an unspecified but in-range
+ *    routing.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int32_t moe_status;
+#define MOE_OK 0
+#define MOE_ERR_INVALID_ARG 1
+#define MOE_ERR_UNSUPPORTED 2
+#define MOE_ERR_CUDA 3
+#define MOE_ERR_WORKSPACE_TOO_SMALL 4
+#define MOE_ERR_DEVICE_TIMEOUT 5
+#define MOE_ERR_DEVICE_BAD_INDEX 6
+
+#define MOE_WDTYPE_BF16 0           /* expert weights bf16                         */
+#define MOE_WDTYPE_FP8_BLOCK128 1   /* expert weights e4m3 + f32 scale per 128x128
+                                       block; activations quantised per 1x128     */
+
+/* Layer shape.  T tokens of hidden size d; E routed experts of intermediate
+ * size I, top-k routing; I_shared = 0 (no shared expert) or I. */
+typedef struct moe_shape {
+    int32_t T, d, E, k, I, I_shared;
+    int32_t wdtype;       /* MOE_WDTYPE_*                                     */
+    int32_t renormalize;  /* 1: softmax over the selected k; 0: over all E    */
+} moe_shape;
+
+/* Layer weights (device).  Gate rows come first in every gate-up matrix.
+ *   w_gu  [E][2I][d]   bf16 (wdtype 0) or e4m3 (wdtype 1)
+ *   w_d   [E][d][I]
+ *   w_gu_scale [E][2I/128][d/128], w_d_scale [E][d/128][I/128]  (wdtype 1)
+ *   ws_gu [2I][d], ws_d [d][I], ws_*_scale likewise  (when I_shared > 0)
+ *   router_hi, router_lo [E][d] bf16 from moe_router_split; router_bias [E]
+ *   or NULL (added to the logits, so it steers both selection and weights). */
+typedef struct moe_weights {
+    const void* w_gu;
+    const void* w_d;
+    const float* w_gu_scale;
+    const float* w_d_scale;
+    const void* ws_gu;
+    const void* ws_d;
+    const float* ws_gu_scale;
+    const float* ws_d_scale;
+    const uint16_t* router_hi;
+    const uint16_t* router_lo;
+    const float* router_bias;
+} moe_weights;
+
+/* Human-readable name of a status code (static storage). */
+const char* moe_status_string(moe_status s);
+
+/* Workspace bytes that moe_forward / moe_forward_host / moe_gemm_gateup /
+ * moe_gemm_down need for `shape` (0 on an invalid shape).  The workspace is
+ * device memory, 256-byte aligned, owned by the caller, and may be reused
+ * across calls that are ordered on one stream. */
+size_t moe_workspace_bytes(const moe_shape* shape);
+
+/* Workspace bytes moe_permute needs for T tokens, E experts, top-k. */
+size_t moe_permute_workspace_bytes(int32_t T, int32_t E, int32_t k);
+
+/* [RG] Offline split of n FP32 router weights: hi = RNE_bf16(W),
+ * lo = RNE_bf16((W - hi) * 256); W ~= hi + lo / 256 within 2^-16 |W|. */
+moe_status moe_router_split(const float* W, uint16_t* hi, uint16_t* lo, int64_t n,
+                            void* stream);
+
+/* [G8][HY] Offline FP8 quantisation of `batch` bf16 matrices [rows][cols]
+ * (rows, cols multiples of 128): per 128x128 block s = fp32(amax)/448
+ * (amax == 0 -> 1), q = e4m3_rne_satfinite(fp32(W / s)).
+ * q [batch][rows][cols], scale [batch][rows/128][cols/128]. */
+moe_status moe_quantize_weights_fp8(const uint16_t* W, int64_t batch, int32_t rows,
+                                    int32_t cols, uint8_t* q, float* scale, void* stream);
+
+/* [FM] Activation quantisation of a bf16 [rows][cols] matrix (cols % 128 ==
+ * 0), per row per 1x128 group, same rule: q [rows][cols], scale
+ * [rows][cols/128]. */
+moe_status moe_quantize_act_fp8(const uint16_t* x, int64_t rows, int32_t cols,
+                                uint8_t* q, float* scale, void* stream);
+
+/* [RG] Router logits on tensor cores:
+ *   logits[t][e] = acc_hi + acc_lo / 256 (+ bias[e]),
+ *   acc_* = sum_i x[t][i] * {hi,lo}[e][i] accumulated in FP32.
+ * x [T][d] bf16, hi/lo [E][d] bf16, bias [E] or NULL, logits [T][E] f32. */
+moe_status moe_router_logits(const uint16_t* x, const uint16_t* hi, const uint16_t* lo,
+                             const float* bias, float* logits, int32_t T, int32_t d,
+                             int32_t E, void* stream);
+
+/* [FM][HY] Top-k routing of FP32 logits [T][E]: ids [T][k] in descending
+ * logit order, ties to the lower expert id; w [T][k] = exp(l - l_max) /
+ * sum over the selected k (renormalize = 1) or over all E (= 0). */
+moe_status moe_route_topk(const float* logits, int32_t T, int32_t E, int32_t k,
+                          int32_t renormalize, int32_t* ids, float* w, void* stream);
+
+/* [FP] Per-expert counts [E], offsets [E+1] (exclusive scan, offsets[E] =
+ * T*k), and the stable permutation of the flat assignments a = t*k + j:
+ * rows of expert e are offsets[e] .. offsets[e+1]-1 in ascending a;
+ * perm [T*k] maps row -> a, inv [T*k] maps a -> row.  Deterministic: the
+ * result does not depend on scheduling.  An id outside [0, E) sets
+ * MOE_ERR_DEVICE_BAD_INDEX in the workspace status word and is not placed.
+ * ws: moe_permute_workspace_bytes(T, E, k) bytes. */
+moe_status moe_permute(const int32_t* ids, int32_t T, int32_t E, int32_t k,
+                       int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv,
+                       void* ws, size_t ws_bytes, void* stream);
+
+/* [FM][FP][G8] Grouped Gate-Up GEMM with SiLU*mul epilogue.  Row p < T*k of
+ * expert e (offsets[e] <= p < offsets[e+1]) reads token perm[p] / k straight
+ * from x (no separate gather); rows T*k .. T*k+T-1 (when I_shared > 0) are
+ * the shared expert on token p - T*k.
+ *   h[p][n] = silu(x_t . Wg[e][n]) * (x_t . Wu[e][n]),  FP32 accumulation.
+ * wdtype 0: x [T][d] bf16, x_scale NULL; h [R][I] bf16, h_scale NULL.
+ * wdtype 1: x [T][d] e4m3 with x_scale [T][d/128] (moe_quantize_act_fp8);
+ *           h [R][I] e4m3 with h_scale [R][I/128] (1x128 quantisation of the
+ *           FP32 h in the epilogue).
+ * R = T*k + (I_shared ? T : 0).  ws: moe_workspace_bytes(shape). */
+moe_status moe_gemm_gateup(const moe_shape* shape, const moe_weights* weights,
+                           const void* x, const float* x_scale, const int32_t* perm,
+                           const int32_t* offsets, void* h, float* h_scale,
+                           void* ws, size_t ws_bytes, void* stream);
+
+/* [FM][G8] Grouped Down GEMM: o[p] = h[p] . Wd[e]^T (FP32 accumulation,
+ * one bf16 rounding), same row grouping as moe_gemm_gateup.
+ * o [R][d] bf16.  ws: moe_workspace_bytes(shape). */
+moe_status moe_gemm_down(const moe_shape* shape, const moe_weights* weights,
+                         const void* h, const float* h_scale, const int32_t* offsets,
+                         uint16_t* o, void* ws, size_t ws_bytes, void* stream);
+
+/* [FM] Top-K weighted aggregation plus the shared expert:
+ *   y[t] = sum_j w[t][j] * o[inv[t*k+j]] + o[T*k+t]   (FP32 sum, one bf16
+ * rounding; the shared term only when I_shared > 0).  y [T][d] bf16. */
+moe_status moe_combine(const moe_shape* shape, const uint16_t* o, const int32_t* inv,
+                       const float* w, uint16_t* y, void* stream);
+
+/* The whole layer in one call: router logits -> top-k -> permute ->
+ * (FP8: quantise x) -> gate-up -> down -> combine, all on `stream`.
+ * x [T][d] bf16, y [T][d] bf16.  ws: moe_workspace_bytes(shape). */
+moe_status moe_forward(const moe_shape* shape, const moe_weights* weights,
+                       const uint16_t* x, uint16_t* y, void* ws, size_t ws_bytes,
+                       void* stream);
+
+/* moe_forward that also records the caller's CUDA events (cudaEvent_t as
+ * void*, created by the caller) on `stream` at the stage boundaries, so the
+ * caller can time each kernel on the stream it runs on:
+ *   events[0] start, [1] after router logits, [2] top-k, [3] permute,
+ *   [4] activation quantisation (FP8; same point as [3] for BF16),
+ *   [5] gate-up GEMM, [6] down GEMM, [7] combine.
+ * n_events must be MOE_PROFILE_EVENTS. */
+#define MOE_PROFILE_EVENTS 8
+moe_status moe_forward_profiled(const moe_shape* shape, const moe_weights* weights,
+                                const uint16_t* x, uint16_t* y, void* ws, size_t ws_bytes,
+                                void* stream, void* const* events, int32_t n_events);
+
+/* moe_forward on HOST buffers: copies x_host [T][d] in, runs the layer,
+ * copies y_host [T][d] out and synchronises `stream` before returning.
+ * Pinned host memory gives asynchronous copies.  Staging lives in the
+ * workspace: ws_bytes >= moe_workspace_bytes(shape). */
+moe_status moe_forward_host(const moe_shape* shape, const moe_weights* weights,
+                            const uint16_t* x_host, uint16_t* y_host, void* ws,
+                            size_t ws_bytes, void* stream);
+
+/* Synchronises `stream` and returns the device status word of `ws`
+ * (MOE_OK, MOE_ERR_DEVICE_TIMEOUT or MOE_ERR_DEVICE_BAD_INDEX). */
+moe_status moe_read_device_status(const void* ws, void* stream);
+
+/* Failure-path check of the bounded device waits: launches one block that
+ * waits on a barrier nothing completes, gives up after `limit_us`
+ * microseconds, records MOE_ERR_DEVICE_TIMEOUT in the status word of ws
+ * (>= 256 bytes) and returns; read it with moe_read_device_status. */
+moe_status moe_selftest_timeout(void* ws, int32_t limit_us, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_B200_H */

@@ -1,0 +1,65 @@
+"""CPU checks of the C ABI: the shared library builds, loads and exports every
+entry point include/moe.h declares; host-only calls (sizes, status strings,
+argument validation) behave as documented.  No kernel is launched here."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe.h")
+
+
+def _declared():
+    src = open(HEADER, encoding="utf-8").read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z0-9_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from expert_layer_dual_b200 import build
+    build.build()
+    return ctypes.CDLL(build.LIB)
+
+
+def test_every_declared_entry_point_is_exported(lib):
+    names = _declared()
+    assert len(names) >= 16
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in moe.h but not exported"
+    from expert_layer_dual_b200 import moe
+    assert sorted(moe.EXPORTS) == names
+
+
+def test_status_strings_and_sizes(lib):
+    from expert_layer_dual_b200 import moe as M
+    assert M.status_string(M.OK) == "ok"
+    assert "workspace" in M.status_string(M.WORKSPACE_TOO_SMALL)
+    s = M.moe_shape(64, 4096, 256, 8, 1536, 1536, 0, 1)
+    n = M.workspace_bytes(s)
+    R = 64 * 8 + 64
+    assert n >= R * 4096 * 2 + R * 1536 * 2 and n % 256 == 0
+    s8 = M.moe_shape(4096, 6144, 256, 8, 2048, 2048, 1, 1)
+    assert M.workspace_bytes(s8) > 0
+    assert M.workspace_bytes(M.moe_shape(64, 4000, 256, 8, 1536, 1536, 0, 1)) == 0   # d % 128
+    assert M.workspace_bytes(M.moe_shape(64, 4096, 300, 8, 1536, 1536, 0, 1)) == 0   # E > 256
+    assert M.workspace_bytes(M.moe_shape(64, 4096, 256, 9, 1536, 1536, 0, 1)) == 0   # k > 8
+    assert M.workspace_bytes(M.moe_shape(64, 4096, 256, 8, 1536, 512, 0, 1)) == 0    # Is not in {0, I}
+    assert M.permute_workspace_bytes(16384, 256, 8) >= 256 + 128 * 256 * 4
+
+
+def test_validation_happens_before_any_launch(lib):
+    from expert_layer_dual_b200 import moe as M
+    s = M.moe_shape(16, 256, 8, 2, 128, 0, 0, 1)
+    w = M.moe_weights()
+    # null weights -> invalid argument, decided on the host
+    assert lib.moe_forward(ctypes.byref(s), ctypes.byref(w), None, None, None, 0, None) == M.INVALID_ARG
+    bad = M.moe_shape(16, 250, 8, 2, 128, 0, 0, 1)
+    assert lib.moe_forward(ctypes.byref(bad), ctypes.byref(w), None, None, None, 0, None) == M.UNSUPPORTED
+    zero = M.moe_shape(0, 256, 8, 2, 128, 0, 0, 1)
+    w2 = M.moe_weights(*([ctypes.c_void_p(256)] * 10 + [None]))
+    assert lib.moe_forward(ctypes.byref(zero), ctypes.byref(w2), None, None, None, 0, None) == M.OK
+    assert lib.moe_route_topk(None, 4, 300, 2, 1, None, None, None) == M.UNSUPPORTED
+    assert lib.moe_router_split(None, None, None, ctypes.c_int64(-1), None) == M.INVALID_ARG

@@ -1,0 +1,202 @@
+"""GPU parity of each stage entry point of the C ABI against the oracle, on
+seeded synthetic inputs at sizes the oracle finishes in seconds (several
+tiles, ragged tails).
+
+Tolerances (derived from the arithmetic):
+  - router split, top-k ids, counts / offsets / perm / inv, FP8 codes: exact;
+  - router logits: |g - o| <= 1e-5 * max(|o|, rms(row)) (FP32 accumulation of
+    exact bf16 products against the FP64 sum);
+  - top-k weights: 2e-6 absolute (FP32 exp and division of values <= 1);
+  - bf16 outputs of one FP32-accumulated GEMM or sum: one bf16 rounding
+    (relative 2^-9) plus FP32 noise: rtol 2^-8, atol 1e-3 * rms(ref).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from expert_layer_dual_b200.configs import MoEConfig
+from expert_layer_dual_b200.inputs import (make_layer, random_bf16, random_ids, random_logits,
+                                           random_weights)
+from gpu_util import assert_close_rel, bf16_to_f64, bits, oracle_layer, rms
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import expert_layer_dual_b200.moe as M
+
+DEV = "cuda"
+
+SMALL = [
+    MoEConfig("tiny", T=16, d=256, E=8, k=2, I=128, Is=0, seed=0),
+    MoEConfig("ragged", T=300, d=512, E=16, k=4, I=256, Is=256, seed=21),
+    MoEConfig("odd", T=203, d=384, E=40, k=8, I=128, Is=128, seed=22),
+    MoEConfig("wide", T=130, d=256, E=256, k=8, I=128, Is=128, seed=23),
+]
+IDS = [c.name for c in SMALL]
+
+
+def _u16(t):
+    return t.view(torch.uint16)
+
+
+@pytest.mark.parametrize("n", [1, 1000, 256 * 4096 + 3])
+def test_router_split_bit_exact(n):
+    g = torch.Generator().manual_seed(n)
+    W = torch.randn(n, generator=g) * torch.exp2(torch.randint(-20, 20, (n,), generator=g).float())
+    hi = torch.empty(n, dtype=torch.uint16, device=DEV)
+    lo = torch.empty(n, dtype=torch.uint16, device=DEV)
+    M.router_split(W.to(DEV), hi, lo)
+    ohi, olo = oracle.router_split(W.numpy())
+    assert np.array_equal(bits(hi), ohi) and np.array_equal(bits(lo), olo)
+
+
+@pytest.mark.parametrize("cfg", SMALL + [MoEConfig("d4096", T=257, d=4096, E=256, k=8, I=128, seed=24)],
+                         ids=IDS + ["d4096"])
+def test_router_logits(cfg):
+    inp = make_layer(cfg)
+    W = inp["router_w"]
+    hi = torch.empty(W.shape, dtype=torch.uint16, device=DEV)
+    lo = torch.empty_like(hi)
+    M.router_split(W.to(DEV), hi, lo)
+    bias = torch.randn(cfg.E, generator=torch.Generator().manual_seed(5)) if cfg.T % 2 else None
+    x = inp["x"].to(DEV)
+    logits = torch.empty((cfg.T, cfg.E), dtype=torch.float32, device=DEV)
+    M.router_logits(_u16(x), hi, lo, None if bias is None else bias.to(DEV), logits)
+    ref = oracle.router_logits(bits(inp["x"]), bits(hi), bits(lo), None if bias is None else bias.numpy())
+    got = logits.cpu().double().numpy()
+    scale = np.maximum(np.abs(ref), np.sqrt(np.mean(ref ** 2, axis=1, keepdims=True)))
+    rel = np.abs(got - ref) / scale
+    assert rel.max() <= 1e-5, f"max relative logit error {rel.max():.3g}"
+
+
+@pytest.mark.parametrize("T,E,k,renorm", [(16, 8, 2, 1), (999, 256, 8, 1), (77, 40, 8, 1),
+                                          (64, 256, 8, 0), (5, 3, 3, 1), (33, 256, 1, 1)])
+def test_route_topk(T, E, k, renorm):
+    l = random_logits(T, E, seed=T * 7 + E)
+    ids = torch.empty((T, k), dtype=torch.int32, device=DEV)
+    w = torch.empty((T, k), dtype=torch.float32, device=DEV)
+    M.route_topk(l.to(DEV), k, renorm, ids, w)
+    oids, ow = oracle.route_topk(l.numpy(), k, renorm=bool(renorm))
+    assert np.array_equal(ids.cpu().numpy(), oids)
+    assert np.max(np.abs(w.cpu().double().numpy() - ow)) <= 2e-6
+
+
+def test_route_topk_all_equal_logits():
+    T, E, k = 40, 256, 8
+    ids = torch.empty((T, k), dtype=torch.int32, device=DEV)
+    w = torch.empty((T, k), dtype=torch.float32, device=DEV)
+    M.route_topk(torch.zeros((T, E), device=DEV), k, 1, ids, w)
+    assert np.array_equal(ids.cpu().numpy(), np.tile(np.arange(k), (T, 1)))
+    assert torch.all(w == 1.0 / k)
+
+
+@pytest.mark.parametrize("T,E,k", [(16, 8, 2), (4097, 256, 8), (300, 16, 4), (1, 1, 1), (16384, 256, 8)])
+def test_permute_bit_exact(T, E, k):
+    ids = random_ids(T, E, k, seed=T + E)
+    counts = torch.empty(E, dtype=torch.int32, device=DEV)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=DEV)
+    perm = torch.empty(T * k, dtype=torch.int32, device=DEV)
+    inv = torch.empty(T * k, dtype=torch.int32, device=DEV)
+    ws = torch.empty(M.permute_workspace_bytes(T, E, k), dtype=torch.uint8, device=DEV)
+    M.permute(ids.to(DEV), E, counts, offsets, perm, inv, ws)
+    oc, oo, op, oi = oracle.permute(ids.numpy(), E)
+    for g, o in ((counts, oc), (offsets, oo), (perm, op), (inv, oi)):
+        assert np.array_equal(g.cpu().numpy(), o)
+    assert M.read_device_status(ws) == M.OK
+
+
+def test_permute_skewed_and_empty_experts():
+    T, E, k = 2000, 256, 8
+    g = torch.Generator().manual_seed(3)
+    hot = torch.randperm(E, generator=g)[:12]          # only 12 experts receive tokens
+    ids = torch.stack([hot[torch.randperm(12, generator=g)[:k]] for _ in range(T)]).to(torch.int32)
+    counts = torch.empty(E, dtype=torch.int32, device=DEV)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=DEV)
+    perm = torch.empty(T * k, dtype=torch.int32, device=DEV)
+    inv = torch.empty(T * k, dtype=torch.int32, device=DEV)
+    ws = torch.empty(M.permute_workspace_bytes(T, E, k), dtype=torch.uint8, device=DEV)
+    M.permute(ids.to(DEV), E, counts, offsets, perm, inv, ws)
+    oc, oo, op, oi = oracle.permute(ids.numpy(), E)
+    assert np.array_equal(perm.cpu().numpy(), op) and np.array_equal(offsets.cpu().numpy(), oo)
+    assert (oc == 0).sum() == E - 12
+
+
+def _gpu_permute(ids_dev, E):
+    T, k = ids_dev.shape
+    counts = torch.empty(E, dtype=torch.int32, device=DEV)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=DEV)
+    perm = torch.empty(T * k, dtype=torch.int32, device=DEV)
+    inv = torch.empty(T * k, dtype=torch.int32, device=DEV)
+    ws = torch.empty(M.permute_workspace_bytes(T, E, k), dtype=torch.uint8, device=DEV)
+    M.permute(ids_dev, E, counts, offsets, perm, inv, ws)
+    return counts, offsets, perm, inv
+
+
+@pytest.mark.parametrize("cfg", SMALL, ids=IDS)
+def test_gemm_gateup_bf16(cfg):
+    inp = make_layer(cfg)
+    layer = M.MoELayer(cfg, inp)
+    ids = random_ids(cfg.T, cfg.E, cfg.k, seed=cfg.seed + 100)
+    _, offsets, perm, _ = _gpu_permute(ids.to(DEV), cfg.E)
+    R = cfg.rows()
+    h = torch.empty((R, cfg.I), dtype=torch.bfloat16, device=DEV)
+    M.gemm_gateup(layer.shape(cfg.T), layer.weights, _u16(inp["x"].to(DEV)), None, perm, offsets,
+                  _u16(h), None, layer.ws)
+    assert M.read_device_status(layer.ws) == M.OK
+    _, ooff, operm, _ = oracle.permute(ids.numpy(), cfg.E)
+    ref = oracle.gateup(oracle_layer(cfg, inp), bits(inp["x"]), operm, ooff)
+    assert_close_rel(bf16_to_f64(h), ref, rtol=2.0 ** -8, atol=1e-3 * rms(ref), what="h")
+
+
+@pytest.mark.parametrize("cfg", SMALL, ids=IDS)
+def test_gemm_down_bf16(cfg):
+    inp = make_layer(cfg)
+    layer = M.MoELayer(cfg, inp)
+    ids = random_ids(cfg.T, cfg.E, cfg.k, seed=cfg.seed + 200)
+    _, offsets, _, _ = _gpu_permute(ids.to(DEV), cfg.E)
+    R = cfg.rows()
+    hin = random_bf16((R, cfg.I), seed=cfg.seed, idx=1, std=0.5)
+    o = torch.empty((R, cfg.d), dtype=torch.bfloat16, device=DEV)
+    M.gemm_down(layer.shape(cfg.T), layer.weights, _u16(hin.to(DEV)), None, offsets, _u16(o), layer.ws)
+    assert M.read_device_status(layer.ws) == M.OK
+    _, ooff, _, _ = oracle.permute(ids.numpy(), cfg.E)
+    ref = oracle.down(oracle_layer(cfg, inp), bf16_to_f64(hin), ooff, cfg.T)
+    assert_close_rel(bf16_to_f64(o), ref, rtol=2.0 ** -8, atol=1e-3 * rms(ref), what="o")
+
+
+@pytest.mark.parametrize("cfg", SMALL, ids=IDS)
+def test_combine(cfg):
+    ids = random_ids(cfg.T, cfg.E, cfg.k, seed=cfg.seed + 300)
+    _, _, _, inv = _gpu_permute(ids.to(DEV), cfg.E)
+    R = cfg.rows()
+    o = random_bf16((R, cfg.d), seed=cfg.seed, idx=2)
+    w = random_weights(cfg.T, cfg.k, seed=cfg.seed)
+    y = torch.empty((cfg.T, cfg.d), dtype=torch.bfloat16, device=DEV)
+    M.combine(M.shape_of(cfg), _u16(o.to(DEV)), inv, w.to(DEV), _u16(y))
+    _, _, _, oinv = oracle.permute(ids.numpy(), cfg.E)
+    L = oracle_layer(cfg, {"router_w": torch.zeros(1), "w_gu": torch.zeros(1, dtype=torch.bfloat16),
+                           "w_d": torch.zeros(1, dtype=torch.bfloat16)})
+    ref = oracle.combine(L, bf16_to_f64(o), oinv, w.double().numpy(), cfg.T)
+    assert_close_rel(bf16_to_f64(y), ref, rtol=2.0 ** -8, atol=1e-5 * rms(ref), what="y")
+
+
+@pytest.mark.parametrize("rows,cols", [(1, 128), (300, 512), (4096, 6144)])
+def test_quantize_act_fp8_bit_exact(rows, cols):
+    x = random_bf16((rows, cols), seed=rows, idx=3, std=3.0)
+    x[0, :128] = 0                                             # an all-zero group
+    q = torch.empty((rows, cols), dtype=torch.uint8, device=DEV)
+    s = torch.empty((rows, cols // 128), dtype=torch.float32, device=DEV)
+    M.quantize_act_fp8(_u16(x.to(DEV)), q, s)
+    oq, os_ = oracle.quant_fp8_rows(x.float().numpy())
+    assert np.array_equal(q.cpu().numpy(), oq) and np.array_equal(s.cpu().numpy(), os_)
+
+
+@pytest.mark.parametrize("batch,rows,cols", [(1, 128, 128), (3, 256, 384), (2, 4096, 1024)])
+def test_quantize_weights_fp8_bit_exact(batch, rows, cols):
+    W = random_bf16((batch, rows, cols), seed=rows + cols, idx=4, std=0.02)
+    q = torch.empty(W.shape, dtype=torch.uint8, device=DEV)
+    s = torch.empty((batch, rows // 128, cols // 128), dtype=torch.float32, device=DEV)
+    M.quantize_weights_fp8(_u16(W.to(DEV)), q, s)
+    oq, os_ = oracle.quant_fp8_blocks(bits(W))
+    assert np.array_equal(q.cpu().numpy(), oq) and np.array_equal(s.cpu().numpy(), os_)
