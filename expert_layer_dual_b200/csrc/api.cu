@@ -105,7 +105,7 @@ WsLayout ws_layout(const moe_shape& s) {
         L.xq = L.xs = L.hs = 0;
         L.h = take(R * I * 2);
     }
-    L.o = take(R * d * 2);
+    L.o = take(R * d * 4);                                // FP32 rows of the down GEMM
     L.xin = take(T * d * 2);
     L.yout = take(T * d * 2);
     L.total = off;
@@ -197,7 +197,7 @@ moe_status run_gateup(const moe_shape* s, const moe_weights* w, const void* x, c
 }
 
 moe_status run_down(const moe_shape* s, const moe_weights* w, const void* h, const float* hs,
-                    const int32_t* offsets, uint16_t* o, int32_t* status, cudaStream_t st) {
+                    const int32_t* offsets, float* o, int32_t* status, cudaStream_t st) {
     const GroupedGemmArgs a = gemm_args(s, offsets, nullptr, status);
     if (s->wdtype == MOE_WDTYPE_BF16)
         return cuda_status(launch_down_bf16(a, static_cast<const uint16_t*>(h),
@@ -255,7 +255,7 @@ moe_status forward_device(const moe_shape* s, const moe_weights* w, const uint16
     if (!mark(4)) return MOE_ERR_CUDA;
     void* h = at<uint8_t>(ws, L.h);
     float* hs = fp8 ? at<float>(ws, L.hs) : nullptr;
-    uint16_t* o = at<uint16_t>(ws, L.o);
+    float* o = at<float>(ws, L.o);
     if ((r = run_gateup(s, w, a_in, a_scale, perm, offsets, h, hs, status, st)) != MOE_OK) return r;
     if (!mark(5)) return MOE_ERR_CUDA;
     if ((r = run_down(s, w, h, hs, offsets, o, status, st)) != MOE_OK) return r;
@@ -380,7 +380,7 @@ moe_status moe_gemm_gateup(const moe_shape* shape, const moe_weights* weights, c
 }
 
 moe_status moe_gemm_down(const moe_shape* shape, const moe_weights* weights, const void* h,
-                         const float* h_scale, const int32_t* offsets, uint16_t* o, void* ws,
+                         const float* h_scale, const int32_t* offsets, float* o, void* ws,
                          size_t ws_bytes, void* stream) {
     moe_status r = check_shape(shape);
     if (r != MOE_OK) return r;
@@ -397,7 +397,7 @@ moe_status moe_gemm_down(const moe_shape* shape, const moe_weights* weights, con
     return run_down(shape, weights, h, h_scale, offsets, o, status, st);
 }
 
-moe_status moe_combine(const moe_shape* shape, const uint16_t* o, const int32_t* inv,
+moe_status moe_combine(const moe_shape* shape, const float* o, const int32_t* inv,
                        const float* w, uint16_t* y, void* stream) {
     moe_status r = check_shape(shape);
     if (r != MOE_OK) return r;

@@ -16,12 +16,15 @@
 //  - gate-up: the 256 B columns are 128 gate rows and the matching 128 up
 //    rows of W_gu, so one N=256 MMA yields both halves of h's 128 columns;
 //    the A rows are gathered from x by the routing permutation with
-//    cp.async (4 warps, one row each), the weights arrive by TMA;
+//    cp.async (4 warps, 8 lanes per 128-byte row slice), the weights arrive
+//    by TMA;
 //  - down: A (contiguous permuted rows of h) and B by TMA;
 //  - one thread issues tcgen05.mma into one of two 256-column TMEM
 //    accumulators, so the epilogue of a tile overlaps the next tile's MMAs;
 //  - 4 epilogue warps read TMEM (tcgen05.ld), apply SiLU*mul (gate-up) and
-//    store bf16 rows.
+//    store rows (h in bf16, the MMA operand of the down GEMM; o in FP32);
+//  - the TMA warp also prefetches the weight tiles kPrefetch k-blocks ahead
+//    into L2, so the loads into the ring mostly hit L2.
 // Every wait is bounded; a timeout sets the device status word and all roles
 // stop, drain their copies in flight and free TMEM.
 #include "common.cuh"
@@ -32,6 +35,7 @@ namespace moe {
 namespace {
 
 constexpr int BM = 128, BK = 64, BN = 256, STAGES = 4;
+constexpr int kPrefetch = 8;  // k-blocks of weights prefetched into L2 ahead of the ring
 constexpr int A_BYTES = BM * BK * 2;      // 16 KB
 constexpr int B_HALF = 128 * BK * 2;      // 16 KB
 constexpr int B_BYTES = 2 * B_HALF;       // 32 KB
@@ -171,13 +175,33 @@ __global__ void __launch_bounds__(GATEUP_THREADS, 1)
             tma_prefetch_desc(&tm_ws);
             uint32_t it = 0, issued = 0;
             bool ok = true;
+            // weight rows of a tile: 128 gate rows and the matching 128 up rows
+            auto rows_of = [&](const Tile& t, const CUtensorMap*& map, int& rg, int& ru) {
+                const bool shared = t.g >= a.E;
+                map = shared ? &tm_ws : &tm_w;
+                const int rbase = shared ? 0 : t.g * 2 * a.I;
+                rg = rbase + t.n * 128;
+                ru = rbase + a.I + t.n * 128;
+            };
             for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
                 const Tile t = decode_tile(sm.tt, G, n_tiles, tile, BM);
-                const bool shared = t.g >= a.E;
-                const CUtensorMap* map = shared ? &tm_ws : &tm_w;
-                const int rbase = shared ? 0 : t.g * 2 * a.I;
-                const int rg = rbase + t.n * 128, ru = rbase + a.I + t.n * 128;
+                const CUtensorMap* map;
+                int rg, ru;
+                rows_of(t, map, rg, ru);
+                const int next = tile + (int)gridDim.x;
+                const CUtensorMap* nmap = map;
+                int nrg = rg, nru = ru;
+                if (next < total) rows_of(decode_tile(sm.tt, G, n_tiles, next, BM), nmap, nrg, nru);
                 for (int kb = 0; kb < nk; ++kb, ++it) {
+                    // keep the L2 kPrefetch k-blocks ahead of the shared-memory ring
+                    const int pk = kb + kPrefetch;
+                    if (pk < nk) {
+                        tma_prefetch_l2_2d(map, pk * BK, rg);
+                        tma_prefetch_l2_2d(map, pk * BK, ru);
+                    } else if (next < total) {
+                        tma_prefetch_l2_2d(nmap, (pk - nk) * BK, nrg);
+                        tma_prefetch_l2_2d(nmap, (pk - nk) * BK, nru);
+                    }
                     const int s = it % STAGES;
                     const uint32_t ph = (it / STAGES) & 1;
                     if (!mbar_wait(&b->empty[s], ph ^ 1, a.timeout_ns, ab)) {
@@ -198,22 +222,34 @@ __global__ void __launch_bounds__(GATEUP_THREADS, 1)
             }
         }
     } else if (warp >= GATHER_WARP0) {
-        // ---------------- A rows gathered from x through the permutation
-        const int r = threadIdx.x - GATHER_WARP0 * 32;  // tile row of this thread
+        // ---------------- A rows gathered from x through the permutation.
+        // Eight consecutive lanes copy the eight 16-byte chunks of one row's
+        // 128-byte k-slice, so each warp instruction reads four whole lines;
+        // thread j owns chunk j % 8 of rows j / 8 + 16 i, i = 0..7.  A stage
+        // is published (proxy fence + arrive) once its copies have landed,
+        // two stages behind the newest, so three stages are in flight.
+        const int j = threadIdx.x - GATHER_WARP0 * 32;
+        const uint32_t chunk = static_cast<uint32_t>(j & 7);
+        const int rr = j >> 3;
+        const uint32_t swz_off = ((chunk ^ static_cast<uint32_t>(rr & 7)) << 4);
         uint32_t it = 0;
-        int prev = -1;
+        int pend0 = -1, pend1 = -1;  // stages issued but not yet published, oldest first
         bool ok = true;
         for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
             const Tile t = decode_tile(sm.tt, G, n_tiles, tile, BM);
-            const bool valid = r < t.nrows;
-            int64_t tok = 0;
-            if (valid) {
-                const int p = t.row0 + r;
-                tok = (t.g < a.E) ? (int64_t)(a.perm[p] / a.k) : (int64_t)(p - Tk);
+            const uint16_t* src[8];
+            uint32_t valid = 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int r = rr + 16 * i;
+                int64_t tok = 0;
+                if (r < t.nrows) {
+                    const int p = t.row0 + r;
+                    tok = (t.g < a.E) ? (int64_t)(a.perm[p] / a.k) : (int64_t)(p - Tk);
+                    valid |= 1u << i;
+                }
+                src[i] = x + tok * a.d + chunk * 8;
             }
-            const uint16_t* src = x + tok * a.d;
-            const uint32_t nbytes = valid ? 16u : 0u;
-            const uint32_t swz = static_cast<uint32_t>(r & 7);
             for (int kb = 0; kb < nk; ++kb, ++it) {
                 const int s = it % STAGES;
                 const uint32_t ph = (it / STAGES) & 1;
@@ -222,24 +258,24 @@ __global__ void __launch_bounds__(GATEUP_THREADS, 1)
                     ok = false;
                     break;
                 }
-                const uint32_t dst = smem_u32(sm.stages + s * STAGE_BYTES) + r * 128;
-                const uint16_t* srck = src + kb * BK;
+                const uint32_t dst = smem_u32(sm.stages + s * STAGE_BYTES) + rr * 128 + swz_off;
 #pragma unroll
-                for (uint32_t c = 0; c < 8; ++c) cp_async_16(dst + ((c ^ swz) << 4), srck + c * 8, nbytes);
+                for (int i = 0; i < 8; ++i)
+                    cp_async_16(dst + i * 16 * 128, src[i] + kb * BK, ((valid >> i) & 1u) ? 16u : 0u);
                 cp_async_commit();
-                if (prev >= 0) {  // the previous stage's copies are done: publish them
-                    cp_async_wait<1>();
+                if (pend0 >= 0) {
+                    cp_async_wait<2>();  // the oldest of the three groups in flight is done
                     fence_proxy_async_smem();
-                    mbar_arrive(&b->full_a[prev]);
+                    mbar_arrive(&b->full_a[pend0]);
                 }
-                prev = s;
+                pend0 = pend1;
+                pend1 = s;
             }
         }
         cp_async_wait<0>();
-        if (prev >= 0) {
-            fence_proxy_async_smem();
-            mbar_arrive(&b->full_a[prev]);
-        }
+        fence_proxy_async_smem();
+        if (pend0 >= 0) mbar_arrive(&b->full_a[pend0]);
+        if (pend1 >= 0) mbar_arrive(&b->full_a[pend1]);
     } else if (warp == MMA_WARP) {
         if (lane == 0) mma_role(sm, a, tmem, G, n_tiles, true);
     } else {
@@ -279,10 +315,11 @@ __global__ void __launch_bounds__(GATEUP_THREADS, 1)
 // ---------------------------------------------------------------------------
 // Down: o[p][n0 + j] = h[p] . Wd[n0 + j]
 // ---------------------------------------------------------------------------
+// o stays FP32 [R][d]: rounding it to bf16 before the weighted combine would
+// add a second rounding of every term to the layer output's own.
 __global__ void __launch_bounds__(DOWN_THREADS, 1)
     k_down_bf16(const __grid_constant__ CUtensorMap tm_h, const __grid_constant__ CUtensorMap tm_w,
-                const __grid_constant__ CUtensorMap tm_ws, GroupedGemmArgs a,
-                uint16_t* __restrict__ o) {
+                const __grid_constant__ CUtensorMap tm_ws, GroupedGemmArgs a, float* __restrict__ o) {
     extern __shared__ uint8_t smem_raw[];
     Smem sm = carve_smem(smem_raw);
     Bars* b = sm.bars;
@@ -308,6 +345,12 @@ __global__ void __launch_bounds__(DOWN_THREADS, 1)
                 const int r0 = (shared ? 0 : t.g * a.d) + t.n * BN;
                 const bool two = t.n * BN + 128 < a.d;  // second 128-row half inside this matrix
                 for (int kb = 0; kb < nk; ++kb, ++it) {
+                    const int pk = kb + kPrefetch;
+                    if (pk < nk) {
+                        tma_prefetch_l2_2d(&tm_h, pk * BK, t.row0);
+                        tma_prefetch_l2_2d(map, pk * BK, r0);
+                        if (two) tma_prefetch_l2_2d(map, pk * BK, r0 + 128);
+                    }
                     const int s = it % STAGES;
                     const uint32_t ph = (it / STAGES) & 1;
                     if (!mbar_wait(&b->empty[s], ph ^ 1, a.timeout_ns, ab)) {
@@ -340,20 +383,18 @@ __global__ void __launch_bounds__(DOWN_THREADS, 1)
             tc_fence_after_sync();
             const uint32_t taddr = tmem + (static_cast<uint32_t>(warp * 32) << 16) + buf * BN;
             const int ncols = min(BN, a.d - t.n * BN);
-            uint16_t* dst = o + (int64_t)(t.row0 + row) * a.d + t.n * BN;
+            float* dst = o + (int64_t)(t.row0 + row) * a.d + t.n * BN;
 #pragma unroll 1
             for (int c = 0; c < BN / 32; ++c) {
                 if (c * 32 >= ncols) break;  // uniform across the warp
                 float v[32];
                 tmem_load32(taddr + c * 32, v);
                 if (row < t.nrows) {
-                    uint32_t pk[16];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        st_global_v4(dst + c * 32 + q * 8, pk[4 * q], pk[4 * q + 1], pk[4 * q + 2],
-                                     pk[4 * q + 3]);
+                    for (int q = 0; q < 8; ++q)
+                        st_global_v4(dst + c * 32 + q * 4, __float_as_uint(v[4 * q]),
+                                     __float_as_uint(v[4 * q + 1]), __float_as_uint(v[4 * q + 2]),
+                                     __float_as_uint(v[4 * q + 3]));
                 }
             }
             tc_fence_before_sync();
@@ -391,7 +432,7 @@ cudaError_t launch_gateup_bf16(const GroupedGemmArgs& a, const uint16_t* x, cons
 }
 
 cudaError_t launch_down_bf16(const GroupedGemmArgs& a, const uint16_t* h, const uint16_t* w_d,
-                             const uint16_t* ws_d, uint16_t* o, cudaStream_t s) {
+                             const uint16_t* ws_d, float* o, cudaStream_t s) {
     if (a.T == 0) return cudaSuccess;
     const uint64_t R = (uint64_t)a.T * a.k + (a.has_shared ? a.T : 0);
     CUtensorMap th, tw, tws;

@@ -12,7 +12,7 @@ cudaError_t launch_gateup_fp8(const GroupedGemmArgs&, const uint8_t*, const floa
 }
 
 cudaError_t launch_down_fp8(const GroupedGemmArgs&, const uint8_t*, const float*, const uint8_t*,
-                            const float*, const uint8_t*, const float*, uint16_t*, cudaStream_t) {
+                            const float*, const uint8_t*, const float*, float*, cudaStream_t) {
     return cudaErrorNotSupported;
 }
 

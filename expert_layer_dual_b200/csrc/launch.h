@@ -29,8 +29,9 @@ int permute_segments(int64_t n_assign);
 cudaError_t launch_permute(const int32_t* ids, int T, int E, int k, int32_t* counts,
                            int32_t* offsets, int32_t* perm, int32_t* inv, int32_t* seg_hist,
                            int32_t* status, cudaStream_t s);
-cudaError_t launch_combine(const uint16_t* o, const int32_t* inv, const float* w, uint16_t* y,
-                           int T, int d, int k, int has_shared, cudaStream_t s);
+// o [R][d] f32: routed rows then (has_shared) the shared expert's rows
+cudaError_t launch_combine(const float* o, const int32_t* inv, const float* w, uint16_t* y, int T,
+                           int d, int k, int has_shared, cudaStream_t s);
 cudaError_t launch_quant_act_fp8(const uint16_t* x, int64_t rows, int cols, uint8_t* q,
                                  float* scale, cudaStream_t s);
 cudaError_t launch_quant_weights_fp8(const uint16_t* W, int64_t batch, int rows, int cols,
@@ -53,7 +54,7 @@ struct GroupedGemmArgs {
 cudaError_t launch_gateup_bf16(const GroupedGemmArgs& a, const uint16_t* x, const uint16_t* w_gu,
                                const uint16_t* ws_gu, uint16_t* h, cudaStream_t s);
 cudaError_t launch_down_bf16(const GroupedGemmArgs& a, const uint16_t* h, const uint16_t* w_d,
-                             const uint16_t* ws_d, uint16_t* o, cudaStream_t s);
+                             const uint16_t* ws_d, float* o, cudaStream_t s);
 
 // ---- gemm_fp8.cu (tcgen05 grouped GEMMs, e4m3 with 128x128 block scales)
 cudaError_t launch_gateup_fp8(const GroupedGemmArgs& a, const uint8_t* xq, const float* xs,
@@ -61,7 +62,7 @@ cudaError_t launch_gateup_fp8(const GroupedGemmArgs& a, const uint8_t* xq, const
                               const float* ws_gu_s, uint8_t* hq, float* hs, cudaStream_t s);
 cudaError_t launch_down_fp8(const GroupedGemmArgs& a, const uint8_t* hq, const float* hs,
                             const uint8_t* w_d, const float* w_d_s, const uint8_t* ws_d,
-                            const float* ws_d_s, uint16_t* o, cudaStream_t s);
+                            const float* ws_d_s, float* o, cudaStream_t s);
 
 // ---- tensor maps (api.cu)
 // 2-D row-major tensor [rows][cols] of `elem_bytes`-sized elements, box

@@ -10,9 +10,17 @@
 // B200 form: one CTA per 128-token x 64-expert tile.  A TMA warp streams the
 // x tile and the hi and lo tiles of each 64-wide k-block into a 4-stage
 // shared-memory ring (128-byte swizzle); one thread issues two tcgen05.mma per
-// 16-wide k-step, sharing the A descriptor, into two TMEM accumulators
-// (columns 0-63 hi, 64-127 lo); four epilogue warps read both accumulators
-// with tcgen05.ld and write FP32 logits.  Every wait is bounded.
+// 16-wide k-step, sharing the A descriptor, into TMEM accumulators; four
+// epilogue warps read them with tcgen05.ld and write FP32 logits.  Every wait
+// is bounded.
+//
+// Accuracy: the tensor core's FP32 accumulation loses a little at every MMA
+// step, in proportion to the running sum, and over d = 4096 (256 steps) that
+// alone reaches ~1e-5 of a logit.  The hi product therefore accumulates in
+// C = min(4, k-blocks) separate TMEM accumulators, one per contiguous quarter
+// of the k-blocks, summed pairwise in FP32 by the epilogue before the single
+// correcting FMA; lo (already scaled down by 256) keeps one accumulator.
+// TMEM columns: hi chunk c at c*64 .. c*64+63, lo at C*64 .. C*64+63.
 #include "common.cuh"
 #include "launch.h"
 
@@ -24,7 +32,8 @@ constexpr int A_BYTES = BM * BK * 2;
 constexpr int B_BYTES = BN * BK * 2;
 constexpr int STAGE_BYTES = A_BYTES + 2 * B_BYTES;
 constexpr int THREADS = 192;  // warps 0-3 epilogue, 4 MMA + TMEM owner, 5 TMA
-constexpr uint32_t TMEM_COLS = 128;
+constexpr int MAX_CHUNKS = 4;
+constexpr uint32_t TMEM_COLS = 512;  // (MAX_CHUNKS + 1) * BN = 320 used
 constexpr size_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
 
 __global__ void __launch_bounds__(THREADS, 1)
@@ -44,6 +53,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int m0 = blockIdx.x * BM, e0 = blockIdx.y * BN;
     const int nk = d / BK;
+    const int nchunks = nk < MAX_CHUNKS ? nk : MAX_CHUNKS;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -99,12 +109,14 @@ __global__ void __launch_bounds__(THREADS, 1)
             tc_fence_after_sync();
             const uint32_t a = smem_u32(smem + s * STAGE_BYTES);
             const uint32_t bh = a + A_BYTES, bl = a + A_BYTES + B_BYTES;
+            const int chunk = kb * nchunks / nk;
+            const bool chunk_start = kb * nchunks % nk < nchunks;  // first k-block of its chunk
+            const uint32_t d_hi = tmem + chunk * BN, d_lo = tmem + nchunks * BN;
 #pragma unroll
             for (int kk = 0; kk < BK / 16; ++kk) {
                 const uint64_t ad = sdesc_k_sw128(a + kk * 32);
-                const uint32_t acc = (kb | kk) != 0;
-                umma_bf16(tmem, ad, sdesc_k_sw128(bh + kk * 32), idesc, acc);
-                umma_bf16(tmem + BN, ad, sdesc_k_sw128(bl + kk * 32), idesc, acc);
+                umma_bf16(d_hi, ad, sdesc_k_sw128(bh + kk * 32), idesc, !(chunk_start && kk == 0));
+                umma_bf16(d_lo, ad, sdesc_k_sw128(bl + kk * 32), idesc, (kb | kk) != 0);
             }
             umma_commit(&empty[s]);
         }
@@ -123,8 +135,19 @@ __global__ void __launch_bounds__(THREADS, 1)
             const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
 #pragma unroll 1
             for (int c = 0; c < BN / 32; ++c) {
-                float h[32], l[32];
-                tmem_load32x2(lane_base + c * 32, lane_base + BN + c * 32, h, l);
+                float h[32], l[32], h2[32], h3[32];
+                tmem_load32x2(lane_base + c * 32, lane_base + nchunks * BN + c * 32, h, l);
+                if (nchunks >= 2) {
+                    tmem_load32(lane_base + BN + c * 32, h2);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) h[i] += h2[i];
+                }
+                if (nchunks >= 3) {
+                    tmem_load32(lane_base + 2 * BN + c * 32, h2);
+                    if (nchunks == 4) tmem_load32(lane_base + 3 * BN + c * 32, h3);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) h[i] += (nchunks == 4) ? (h2[i] + h3[i]) : h2[i];
+                }
                 if (t < T) {
                     float* dst = logits + (int64_t)t * E;
 #pragma unroll

@@ -100,8 +100,8 @@ typedef struct moe_weights {
 /* Human-readable name of a status code (static storage). */
 const char* moe_status_string(moe_status s);
 
-/* Workspace bytes that moe_forward / moe_forward_host / moe_gemm_gateup /
- * moe_gemm_down need for `shape` (0 on an invalid shape).  The workspace is
+/* Workspace bytes that moe_forward / moe_forward_profiled / moe_forward_host
+ * need for `shape` (0 on an invalid shape).  The workspace is
  * device memory, 256-byte aligned, owned by the caller, and may be reused
  * across calls that are ordered on one stream. */
 size_t moe_workspace_bytes(const moe_shape* shape);
@@ -161,23 +161,25 @@ moe_status moe_permute(const int32_t* ids, int32_t T, int32_t E, int32_t k,
  * wdtype 1: x [T][d] e4m3 with x_scale [T][d/128] (moe_quantize_act_fp8);
  *           h [R][I] e4m3 with h_scale [R][I/128] (1x128 quantisation of the
  *           FP32 h in the epilogue).
- * R = T*k + (I_shared ? T : 0).  ws: moe_workspace_bytes(shape). */
+ * R = T*k + (I_shared ? T : 0).  ws: at least 256 bytes (the status word). */
 moe_status moe_gemm_gateup(const moe_shape* shape, const moe_weights* weights,
                            const void* x, const float* x_scale, const int32_t* perm,
                            const int32_t* offsets, void* h, float* h_scale,
                            void* ws, size_t ws_bytes, void* stream);
 
-/* [FM][G8] Grouped Down GEMM: o[p] = h[p] . Wd[e]^T (FP32 accumulation,
- * one bf16 rounding), same row grouping as moe_gemm_gateup.
- * o [R][d] bf16.  ws: moe_workspace_bytes(shape). */
+/* [FM][G8] Grouped Down GEMM: o[p] = h[p] . Wd[e]^T with FP32 accumulation,
+ * same row grouping as moe_gemm_gateup, stored FP32: o [R][d] f32.  (The
+ * rows stay FP32 until the weighted combine so the layer output is rounded
+ * to bf16 once.)  ws: at least 256 bytes (the status word). */
 moe_status moe_gemm_down(const moe_shape* shape, const moe_weights* weights,
                          const void* h, const float* h_scale, const int32_t* offsets,
-                         uint16_t* o, void* ws, size_t ws_bytes, void* stream);
+                         float* o, void* ws, size_t ws_bytes, void* stream);
 
 /* [FM] Top-K weighted aggregation plus the shared expert:
- *   y[t] = sum_j w[t][j] * o[inv[t*k+j]] + o[T*k+t]   (FP32 sum, one bf16
- * rounding; the shared term only when I_shared > 0).  y [T][d] bf16. */
-moe_status moe_combine(const moe_shape* shape, const uint16_t* o, const int32_t* inv,
+ *   y[t] = sum_j w[t][j] * o[inv[t*k+j]] + o[T*k+t]
+ * FP32 sum in the order j = 0..k-1 then the shared term (only when
+ * I_shared > 0), one bf16 rounding.  o [R][d] f32, y [T][d] bf16. */
+moe_status moe_combine(const moe_shape* shape, const float* o, const int32_t* inv,
                        const float* w, uint16_t* y, void* stream);
 
 /* The whole layer in one call: router logits -> top-k -> permute ->

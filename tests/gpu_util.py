@@ -55,12 +55,25 @@ def assert_close_rel(got, ref, rtol, atol, what=""):
                              f"got {got[i]!r} ref {ref[i]!r} (atol {atol:.3g}, rtol {rtol:.3g})")
 
 
+def row_scale(logits64: np.ndarray) -> np.ndarray:
+    """Per-row logit scale: rms over the entries that can be selected (a
+    masking bias of -1e4 on some experts would otherwise dominate it)."""
+    med = np.median(np.abs(logits64), axis=1, keepdims=True)
+    live = np.abs(logits64) <= 100.0 * np.maximum(med, 1e-30)
+    sq = np.where(live, logits64 ** 2, 0.0)
+    return np.sqrt(sq.sum(axis=1, keepdims=True) / np.maximum(live.sum(axis=1, keepdims=True), 1))
+
+
+def logit_rel_error(got: np.ndarray, ref: np.ndarray) -> np.ndarray:
+    """|g - o| / max(|o|, row scale): the router-logit error measure."""
+    return np.abs(got - ref) / np.maximum(np.abs(ref), row_scale(ref))
+
+
 def ambiguous_tokens(logits64: np.ndarray, k: int, rel: float = 1e-4) -> np.ndarray:
     """Tokens whose top-(k+1) oracle logits contain two values closer than
-    rel * rms of the row: there the FP32 kernel and the FP64 oracle may
+    rel * the row scale: there the FP32 kernel and the FP64 oracle may
     legitimately order or select differently (both are correct within the
     logits tolerance), so only validity is checked for them."""
     s = -np.sort(-logits64, axis=1)[:, : min(k + 1, logits64.shape[1])]
     gaps = -np.diff(s, axis=1)
-    scale = np.sqrt(np.mean(logits64 ** 2, axis=1, keepdims=True))
-    return np.any(gaps < rel * np.maximum(scale, 1e-30), axis=1)
+    return np.any(gaps < rel * np.maximum(row_scale(logits64), 1e-30), axis=1)

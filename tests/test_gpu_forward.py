@@ -15,7 +15,7 @@ import torch
 import oracle
 from expert_layer_dual_b200.configs import CONFIGS, MoEConfig
 from expert_layer_dual_b200.inputs import make_layer
-from gpu_util import ambiguous_tokens, bf16_to_f64, bits, oracle_layer, rms
+from gpu_util import ambiguous_tokens, bf16_to_f64, bits, logit_rel_error, oracle_layer, row_scale, rms
 
 pytestmark = pytest.mark.gpu
 
@@ -82,11 +82,12 @@ def _compare_tokens(cfg, y_gpu, st, ref, tol):
     ok = ~amb
     assert np.array_equal(gids[ok], ref["ids"][ok]), "expert ids differ on unambiguous tokens"
     # ambiguous tokens: every chosen expert's logit is within the tie band of the k-th best
+    scales = row_scale(ref["logits"])
     for t in np.where(amb)[0]:
         row = ref["logits"][t]
         kth = -np.sort(-row)[cfg.k - 1]
-        band = 1e-4 * np.sqrt(np.mean(row ** 2))
-        assert np.all(row[gids[t]] >= kth - 2 * band)
+        assert np.all(row[gids[t]] >= kth - 2e-4 * scales[t, 0])
+    assert ok.sum() >= 0.9 * len(ok), f"{int(amb.sum())} of {len(ok)} tokens ambiguous"
     err = np.abs(y_gpu[ok] - ref["y"][ok])
     scale = rms(ref["y"])
     assert err.max() <= tol * scale, f"max |dy| = {err.max() / scale:.3g} * rms(y)"
@@ -106,8 +107,7 @@ def test_forward_small(cfg):
     ref = oracle.forward(oracle_layer(cfg, inp), bits(inp["x"]))
     rel, namb = _compare_tokens(cfg, bf16_to_f64(y), st_np, ref, 2e-2)
     # the logits feeding the routing are FP32-accurate
-    scale = np.maximum(np.abs(ref["logits"]), np.sqrt(np.mean(ref["logits"] ** 2, axis=1, keepdims=True)))
-    assert np.max(np.abs(st_np["logits"] - ref["logits"]) / scale) <= 1e-5
+    assert logit_rel_error(st_np["logits"], ref["logits"]).max() <= 1e-5
     # y computed twice is identical (no atomics anywhere on the path)
     y2 = layer.forward(x)
     assert torch.equal(y, y2)
@@ -180,8 +180,6 @@ def _full_size_case(name, n_sample):
     assert layer.device_status() == M.OK
     st = _stage_outputs(layer, cfg, x)
     _check_routing_validity(st, cfg, cfg.T)
-    # the one-call forward and the stage sequence are the same computation
-    h_needed = None
     g = torch.Generator().manual_seed(99)
     sample = torch.sort(torch.randperm(cfg.T, generator=g)[:n_sample]).values.numpy()
     xs = bits(x[torch.as_tensor(sample, device=DEV)])
@@ -204,8 +202,7 @@ def _full_size_case(name, n_sample):
     st_np = {k: v.cpu().numpy()[sample] for k, v in st.items() if k in ("logits", "ids", "w")}
     tol = 6e-2 if cfg.wdtype else 2e-2
     rel, namb = _compare_tokens(cfg, bf16_to_f64(y)[sample], st_np, ref, tol)
-    scale = np.maximum(np.abs(ref["logits"]), np.sqrt(np.mean(ref["logits"] ** 2, axis=1, keepdims=True)))
-    assert np.max(np.abs(st_np["logits"] - ref["logits"]) / scale) <= 1e-5
+    assert logit_rel_error(st_np["logits"], ref["logits"]).max() <= 1e-5
     return cfg, st
 
 

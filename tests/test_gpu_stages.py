@@ -18,7 +18,7 @@ import oracle
 from expert_layer_dual_b200.configs import MoEConfig
 from expert_layer_dual_b200.inputs import (make_layer, random_bf16, random_ids, random_logits,
                                            random_weights)
-from gpu_util import assert_close_rel, bf16_to_f64, bits, oracle_layer, rms
+from gpu_util import assert_close_rel, bf16_to_f64, bits, logit_rel_error, oracle_layer, rms
 
 pytestmark = pytest.mark.gpu
 
@@ -64,9 +64,7 @@ def test_router_logits(cfg):
     logits = torch.empty((cfg.T, cfg.E), dtype=torch.float32, device=DEV)
     M.router_logits(_u16(x), hi, lo, None if bias is None else bias.to(DEV), logits)
     ref = oracle.router_logits(bits(inp["x"]), bits(hi), bits(lo), None if bias is None else bias.numpy())
-    got = logits.cpu().double().numpy()
-    scale = np.maximum(np.abs(ref), np.sqrt(np.mean(ref ** 2, axis=1, keepdims=True)))
-    rel = np.abs(got - ref) / scale
+    rel = logit_rel_error(logits.cpu().double().numpy(), ref)
     assert rel.max() <= 1e-5, f"max relative logit error {rel.max():.3g}"
 
 
@@ -157,12 +155,13 @@ def test_gemm_down_bf16(cfg):
     _, offsets, _, _ = _gpu_permute(ids.to(DEV), cfg.E)
     R = cfg.rows()
     hin = random_bf16((R, cfg.I), seed=cfg.seed, idx=1, std=0.5)
-    o = torch.empty((R, cfg.d), dtype=torch.bfloat16, device=DEV)
-    M.gemm_down(layer.shape(cfg.T), layer.weights, _u16(hin.to(DEV)), None, offsets, _u16(o), layer.ws)
+    o = torch.empty((R, cfg.d), dtype=torch.float32, device=DEV)
+    M.gemm_down(layer.shape(cfg.T), layer.weights, _u16(hin.to(DEV)), None, offsets, o, layer.ws)
     assert M.read_device_status(layer.ws) == M.OK
     _, ooff, _, _ = oracle.permute(ids.numpy(), cfg.E)
     ref = oracle.down(oracle_layer(cfg, inp), bf16_to_f64(hin), ooff, cfg.T)
-    assert_close_rel(bf16_to_f64(o), ref, rtol=2.0 ** -8, atol=1e-3 * rms(ref), what="o")
+    # FP32 rows: only the tensor core's FP32 accumulation over I terms
+    assert_close_rel(o.cpu().double().numpy(), ref, rtol=1e-4, atol=1e-4 * rms(ref), what="o")
 
 
 @pytest.mark.parametrize("cfg", SMALL, ids=IDS)
@@ -170,14 +169,14 @@ def test_combine(cfg):
     ids = random_ids(cfg.T, cfg.E, cfg.k, seed=cfg.seed + 300)
     _, _, _, inv = _gpu_permute(ids.to(DEV), cfg.E)
     R = cfg.rows()
-    o = random_bf16((R, cfg.d), seed=cfg.seed, idx=2)
+    o = torch.randn((R, cfg.d), generator=torch.Generator().manual_seed(cfg.seed))
     w = random_weights(cfg.T, cfg.k, seed=cfg.seed)
     y = torch.empty((cfg.T, cfg.d), dtype=torch.bfloat16, device=DEV)
-    M.combine(M.shape_of(cfg), _u16(o.to(DEV)), inv, w.to(DEV), _u16(y))
+    M.combine(M.shape_of(cfg), o.to(DEV), inv, w.to(DEV), _u16(y))
     _, _, _, oinv = oracle.permute(ids.numpy(), cfg.E)
     L = oracle_layer(cfg, {"router_w": torch.zeros(1), "w_gu": torch.zeros(1, dtype=torch.bfloat16),
                            "w_d": torch.zeros(1, dtype=torch.bfloat16)})
-    ref = oracle.combine(L, bf16_to_f64(o), oinv, w.double().numpy(), cfg.T)
+    ref = oracle.combine(L, o.double().numpy(), oinv, w.double().numpy(), cfg.T)
     assert_close_rel(bf16_to_f64(y), ref, rtol=2.0 ** -8, atol=1e-5 * rms(ref), what="y")
 
 
