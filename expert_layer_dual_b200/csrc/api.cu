@@ -97,8 +97,8 @@ WsLayout ws_layout(const moe_shape& s) {
     L.inv = take(T * k * 4);
     L.seg = take((size_t)permute_segments((int64_t)(T * k)) * E * 4);
     if (s.wdtype == MOE_WDTYPE_FP8_BLOCK128) {
-        L.xq = take(T * d);
-        L.xs = take(T * (d / 128) * 4);
+        L.xq = take(R * d);                               // quantised x in permuted row order
+        L.xs = take(R * (d / 128) * 4);
         L.h = take(R * I);
         L.hs = take(R * (I / 128) * 4);
     } else {
@@ -246,8 +246,9 @@ moe_status forward_device(const moe_shape* s, const moe_weights* w, const uint16
     const void* a_in = x;
     const float* a_scale = nullptr;
     if (fp8) {
-        if ((r = cuda_status(launch_quant_act_fp8(x, s->T, s->d, at<uint8_t>(ws, L.xq),
-                                                  at<float>(ws, L.xs), st))) != MOE_OK)
+        if ((r = cuda_status(launch_quant_act_fp8_permuted(x, perm, s->T, s->k, s->I_shared > 0 ? 1 : 0,
+                                                           s->d, at<uint8_t>(ws, L.xq),
+                                                           at<float>(ws, L.xs), st))) != MOE_OK)
             return r;
         a_in = at<uint8_t>(ws, L.xq);
         a_scale = at<float>(ws, L.xs);
@@ -321,6 +322,18 @@ moe_status moe_quantize_act_fp8(const uint16_t* x, int64_t rows, int32_t cols, u
     return cuda_status(launch_quant_act_fp8(x, rows, cols, q, scale, as_stream(stream)));
 }
 
+moe_status moe_quantize_act_fp8_permuted(const uint16_t* x, const int32_t* perm, int32_t T,
+                                         int32_t k, int32_t with_shared, int32_t d, uint8_t* q,
+                                         float* scale, void* stream) {
+    if (T < 0 || k <= 0 || d <= 0) return MOE_ERR_INVALID_ARG;
+    if (d % 128 != 0 || (int64_t)T * k + T >= ((int64_t)1 << 31)) return MOE_ERR_UNSUPPORTED;
+    if (T == 0) return MOE_OK;
+    if (x == nullptr || perm == nullptr || q == nullptr || scale == nullptr) return MOE_ERR_INVALID_ARG;
+    if (!device_ok()) return MOE_ERR_UNSUPPORTED;
+    return cuda_status(launch_quant_act_fp8_permuted(x, perm, T, k, with_shared ? 1 : 0, d, q, scale,
+                                                     as_stream(stream)));
+}
+
 moe_status moe_router_logits(const uint16_t* x, const uint16_t* hi, const uint16_t* lo,
                              const float* bias, float* logits, int32_t T, int32_t d, int32_t E,
                              void* stream) {
@@ -368,7 +381,7 @@ moe_status moe_gemm_gateup(const moe_shape* shape, const moe_weights* weights, c
     if ((r = check_weights(shape, weights, true, false, false)) != MOE_OK) return r;
     if (shape->T == 0) return MOE_OK;
     const bool fp8 = shape->wdtype == MOE_WDTYPE_FP8_BLOCK128;
-    if (x == nullptr || perm == nullptr || offsets == nullptr || h == nullptr ||
+    if (x == nullptr || offsets == nullptr || h == nullptr || (!fp8 && perm == nullptr) ||
         (fp8 && (x_scale == nullptr || h_scale == nullptr)))
         return MOE_ERR_INVALID_ARG;
     if ((r = check_ws(ws, ws_bytes, kWsHeader)) != MOE_OK) return r;

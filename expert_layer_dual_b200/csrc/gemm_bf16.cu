@@ -23,8 +23,6 @@
 //    accumulators, so the epilogue of a tile overlaps the next tile's MMAs;
 //  - 4 epilogue warps read TMEM (tcgen05.ld), apply SiLU*mul (gate-up) and
 //    store rows (h in bf16, the MMA operand of the down GEMM; o in FP32);
-//  - the TMA warp also prefetches the weight tiles kPrefetch k-blocks ahead
-//    into L2, so the loads into the ring mostly hit L2.
 // Every wait is bounded; a timeout sets the device status word and all roles
 // stop, drain their copies in flight and free TMEM.
 #include "common.cuh"
@@ -35,7 +33,6 @@ namespace moe {
 namespace {
 
 constexpr int BM = 128, BK = 64, BN = 256, STAGES = 4;
-constexpr int kPrefetch = 8;  // k-blocks of weights prefetched into L2 ahead of the ring
 constexpr int A_BYTES = BM * BK * 2;      // 16 KB
 constexpr int B_HALF = 128 * BK * 2;      // 16 KB
 constexpr int B_BYTES = 2 * B_HALF;       // 32 KB
@@ -188,20 +185,7 @@ __global__ void __launch_bounds__(GATEUP_THREADS, 1)
                 const CUtensorMap* map;
                 int rg, ru;
                 rows_of(t, map, rg, ru);
-                const int next = tile + (int)gridDim.x;
-                const CUtensorMap* nmap = map;
-                int nrg = rg, nru = ru;
-                if (next < total) rows_of(decode_tile(sm.tt, G, n_tiles, next, BM), nmap, nrg, nru);
                 for (int kb = 0; kb < nk; ++kb, ++it) {
-                    // keep the L2 kPrefetch k-blocks ahead of the shared-memory ring
-                    const int pk = kb + kPrefetch;
-                    if (pk < nk) {
-                        tma_prefetch_l2_2d(map, pk * BK, rg);
-                        tma_prefetch_l2_2d(map, pk * BK, ru);
-                    } else if (next < total) {
-                        tma_prefetch_l2_2d(nmap, (pk - nk) * BK, nrg);
-                        tma_prefetch_l2_2d(nmap, (pk - nk) * BK, nru);
-                    }
                     const int s = it % STAGES;
                     const uint32_t ph = (it / STAGES) & 1;
                     if (!mbar_wait(&b->empty[s], ph ^ 1, a.timeout_ns, ab)) {
@@ -345,12 +329,6 @@ __global__ void __launch_bounds__(DOWN_THREADS, 1)
                 const int r0 = (shared ? 0 : t.g * a.d) + t.n * BN;
                 const bool two = t.n * BN + 128 < a.d;  // second 128-row half inside this matrix
                 for (int kb = 0; kb < nk; ++kb, ++it) {
-                    const int pk = kb + kPrefetch;
-                    if (pk < nk) {
-                        tma_prefetch_l2_2d(&tm_h, pk * BK, t.row0);
-                        tma_prefetch_l2_2d(map, pk * BK, r0);
-                        if (two) tma_prefetch_l2_2d(map, pk * BK, r0 + 128);
-                    }
                     const int s = it % STAGES;
                     const uint32_t ph = (it / STAGES) & 1;
                     if (!mbar_wait(&b->empty[s], ph ^ 1, a.timeout_ns, ab)) {

@@ -34,6 +34,9 @@ cudaError_t launch_combine(const float* o, const int32_t* inv, const float* w, u
                            int d, int k, int has_shared, cudaStream_t s);
 cudaError_t launch_quant_act_fp8(const uint16_t* x, int64_t rows, int cols, uint8_t* q,
                                  float* scale, cudaStream_t s);
+cudaError_t launch_quant_act_fp8_permuted(const uint16_t* x, const int32_t* perm, int T, int k,
+                                          int has_shared, int cols, uint8_t* q, float* scale,
+                                          cudaStream_t s);
 cudaError_t launch_quant_weights_fp8(const uint16_t* W, int64_t batch, int rows, int cols,
                                      uint8_t* q, float* scale, cudaStream_t s);
 cudaError_t launch_selftest_timeout(int32_t* status, uint64_t limit_ns, cudaStream_t s);

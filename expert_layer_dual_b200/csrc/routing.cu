@@ -343,6 +343,44 @@ __global__ void __launch_bounds__(256)
     if (lane == 0) scale[r * groups + g] = s;
 }
 
+// Same quantisation, written in the permuted row order of the grouped GEMMs:
+// row p < T*k holds token perm[p] / k, row T*k + t holds token t.  The FP8
+// gate-up GEMM then reads its A operand as plain TMA tiles; the gather
+// rides on this pass, which has to read x anyway.
+__global__ void __launch_bounds__(256)
+    k_quant_act_permuted(const uint16_t* __restrict__ x, const int32_t* __restrict__ perm, int T,
+                         int k, int64_t rows, int cols, uint8_t* __restrict__ q,
+                         float* __restrict__ scale) {
+    const int64_t gw = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    const int groups = cols / 128;
+    if (gw >= rows * groups) return;
+    const int64_t p = gw / groups;
+    const int g = (int)(gw % groups);
+    const int64_t Tk = (int64_t)T * k;
+    const int64_t tok = p < Tk ? (int64_t)(perm[p] / k) : p - Tk;
+    const uint2 raw = *reinterpret_cast<const uint2*>(x + tok * cols + g * 128 + lane * 4);
+    const float v0 = __uint_as_float(raw.x << 16), v1 = __uint_as_float(raw.x & 0xffff0000u);
+    const float v2 = __uint_as_float(raw.y << 16), v3 = __uint_as_float(raw.y & 0xffff0000u);
+    float amax = fmaxf(fmaxf(fabsf(v0), fabsf(v1)), fmaxf(fabsf(v2), fabsf(v3)));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const float s = group_scale(amax);
+    *reinterpret_cast<uint32_t*>(q + p * cols + g * 128 + lane * 4) = quant4_e4m3(v0, v1, v2, v3, s);
+    if (lane == 0) scale[p * groups + g] = s;
+}
+
+cudaError_t launch_quant_act_fp8_permuted(const uint16_t* x, const int32_t* perm, int T, int k,
+                                          int has_shared, int cols, uint8_t* q, float* scale,
+                                          cudaStream_t s) {
+    const int64_t rows = (int64_t)T * k + (has_shared ? T : 0);
+    const int64_t warps = rows * (cols / 128);
+    if (warps == 0) return cudaSuccess;
+    k_quant_act_permuted<<<(unsigned)((warps + 7) / 8), 256, 0, s>>>(x, perm, T, k, rows, cols, q,
+                                                                      scale);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_quant_act_fp8(const uint16_t* x, int64_t rows, int cols, uint8_t* q,
                                  float* scale, cudaStream_t s) {
     const int64_t warps = rows * (cols / 128);

@@ -32,6 +32,7 @@ WDTYPE_BF16, WDTYPE_FP8_BLOCK128 = 0, 1
 
 EXPORTS = ["moe_status_string", "moe_workspace_bytes", "moe_permute_workspace_bytes",
            "moe_router_split", "moe_quantize_weights_fp8", "moe_quantize_act_fp8",
+           "moe_quantize_act_fp8_permuted",
            "moe_router_logits", "moe_route_topk", "moe_permute", "moe_gemm_gateup",
            "moe_gemm_down", "moe_combine", "moe_forward", "moe_forward_profiled", "moe_forward_host",
            "moe_read_device_status", "moe_selftest_timeout"]
@@ -58,6 +59,7 @@ _sig = {
     "moe_router_split": (_i32, [_vp, _vp, _vp, _i64, _vp]),
     "moe_quantize_weights_fp8": (_i32, [_vp, _i64, _i32, _i32, _vp, _vp, _vp]),
     "moe_quantize_act_fp8": (_i32, [_vp, _i64, _i32, _vp, _vp, _vp]),
+    "moe_quantize_act_fp8_permuted": (_i32, [_vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
     "moe_router_logits": (_i32, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _vp]),
     "moe_route_topk": (_i32, [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
     "moe_permute": (_i32, [_vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
@@ -133,6 +135,12 @@ def quantize_act_fp8(x, q, scale, stream=None):
     rows, cols = x.shape
     _check(_lib.moe_quantize_act_fp8(_p(x), rows, cols, _p(q), _p(scale), _stream(stream)),
            "moe_quantize_act_fp8")
+
+
+def quantize_act_fp8_permuted(x, perm, k, with_shared, q, scale, stream=None):
+    T, d = x.shape
+    _check(_lib.moe_quantize_act_fp8_permuted(_p(x), _p(perm), T, k, int(with_shared), d, _p(q), _p(scale),
+                                              _stream(stream)), "moe_quantize_act_fp8_permuted")
 
 
 def router_logits(x, hi, lo, bias, logits, stream=None):

@@ -127,6 +127,15 @@ moe_status moe_quantize_weights_fp8(const uint16_t* W, int64_t batch, int32_t ro
 moe_status moe_quantize_act_fp8(const uint16_t* x, int64_t rows, int32_t cols,
                                 uint8_t* q, float* scale, void* stream);
 
+/* [FM] The same activation quantisation, written in the permuted row order
+ * of the grouped GEMMs (the FP8 gate-up GEMM's A operand): row p < T*k holds
+ * token perm[p] / k, rows T*k .. T*k+T-1 (with_shared != 0) hold tokens
+ * 0 .. T-1.  x [T][d] bf16 -> q [R][d] e4m3, scale [R][d/128],
+ * R = T*k + (with_shared ? T : 0). */
+moe_status moe_quantize_act_fp8_permuted(const uint16_t* x, const int32_t* perm, int32_t T,
+                                         int32_t k, int32_t with_shared, int32_t d, uint8_t* q,
+                                         float* scale, void* stream);
+
 /* [RG] Router logits on tensor cores:
  *   logits[t][e] = acc_hi + acc_lo / 256 (+ bias[e]),
  *   acc_* = sum_i x[t][i] * {hi,lo}[e][i] accumulated in FP32.
@@ -158,9 +167,10 @@ moe_status moe_permute(const int32_t* ids, int32_t T, int32_t E, int32_t k,
  * the shared expert on token p - T*k.
  *   h[p][n] = silu(x_t . Wg[e][n]) * (x_t . Wu[e][n]),  FP32 accumulation.
  * wdtype 0: x [T][d] bf16, x_scale NULL; h [R][I] bf16, h_scale NULL.
- * wdtype 1: x [T][d] e4m3 with x_scale [T][d/128] (moe_quantize_act_fp8);
- *           h [R][I] e4m3 with h_scale [R][I/128] (1x128 quantisation of the
- *           FP32 h in the epilogue).
+ * wdtype 1: x [R][d] e4m3 rows already in permuted order with x_scale
+ *           [R][d/128] (moe_quantize_act_fp8_permuted; perm is then not read
+ *           and may be NULL); h [R][I] e4m3 with h_scale [R][I/128] (1x128
+ *           quantisation of the FP32 h in the epilogue).
  * R = T*k + (I_shared ? T : 0).  ws: at least 256 bytes (the status word). */
 moe_status moe_gemm_gateup(const moe_shape* shape, const moe_weights* weights,
                            const void* x, const float* x_scale, const int32_t* perm,

@@ -199,3 +199,85 @@ def test_quantize_weights_fp8_bit_exact(batch, rows, cols):
     M.quantize_weights_fp8(_u16(W.to(DEV)), q, s)
     oq, os_ = oracle.quant_fp8_blocks(bits(W))
     assert np.array_equal(q.cpu().numpy(), oq) and np.array_equal(s.cpu().numpy(), os_)
+
+
+# ---------------------------------------------------------------- FP8 path
+FP8 = [
+    MoEConfig("fp8small", T=200, d=512, E=16, k=4, I=256, Is=256, wdtype=1, seed=31),
+    MoEConfig("fp8odd", T=77, d=384, E=8, k=2, I=128, Is=0, wdtype=1, seed=32),
+]
+FP8_IDS = [c.name for c in FP8]
+
+
+def _permuted_quant(x_dev, perm, cfg):
+    R = cfg.rows()
+    q = torch.empty((R, cfg.d), dtype=torch.uint8, device=DEV)
+    s = torch.empty((R, cfg.d // 128), dtype=torch.float32, device=DEV)
+    M.quantize_act_fp8_permuted(_u16(x_dev), perm, cfg.k, cfg.Is > 0, q, s)
+    return q, s
+
+
+@pytest.mark.parametrize("cfg", FP8, ids=FP8_IDS)
+def test_quantize_act_fp8_permuted_bit_exact(cfg):
+    x = make_layer(cfg)["x"]
+    ids = random_ids(cfg.T, cfg.E, cfg.k, seed=cfg.seed + 400)
+    _, _, perm, _ = _gpu_permute(ids.to(DEV), cfg.E)
+    q, s = _permuted_quant(x.to(DEV), perm, cfg)
+    _, _, operm, _ = oracle.permute(ids.numpy(), cfg.E)
+    tok = np.concatenate([operm // cfg.k, np.arange(cfg.T) if cfg.Is else np.zeros(0, np.int64)])
+    oq, os_ = oracle.quant_fp8_rows(x.float().numpy()[tok])
+    assert np.array_equal(q.cpu().numpy(), oq) and np.array_equal(s.cpu().numpy(), os_)
+
+
+@pytest.mark.parametrize("cfg", FP8, ids=FP8_IDS)
+def test_weights_fp8_match_oracle_quantisation(cfg):
+    inp = make_layer(cfg)
+    layer = M.MoELayer(cfg, inp)
+    q, s = oracle.quant_fp8_blocks(bits(inp["w_gu"]))
+    assert np.array_equal(layer.mats["w_gu"].cpu().numpy(), q)
+    assert np.array_equal(layer.scales["w_gu"].cpu().numpy(), s)
+
+
+@pytest.mark.parametrize("cfg", FP8, ids=FP8_IDS)
+def test_gemm_gateup_fp8(cfg):
+    inp = make_layer(cfg)
+    layer = M.MoELayer(cfg, inp)
+    ids = random_ids(cfg.T, cfg.E, cfg.k, seed=cfg.seed + 100)
+    _, offsets, perm, _ = _gpu_permute(ids.to(DEV), cfg.E)
+    xq, xs = _permuted_quant(inp["x"].to(DEV), perm, cfg)
+    R = cfg.rows()
+    hq = torch.empty((R, cfg.I), dtype=torch.uint8, device=DEV)
+    hs = torch.empty((R, cfg.I // 128), dtype=torch.float32, device=DEV)
+    M.gemm_gateup(layer.shape(cfg.T), layer.weights, xq, xs, None, offsets, hq, hs, layer.ws)
+    assert M.read_device_status(layer.ws) == M.OK
+    _, ooff, operm, _ = oracle.permute(ids.numpy(), cfg.E)
+    ref = oracle.gateup(oracle_layer(cfg, inp), bits(inp["x"]), operm, ooff)   # FP64 h, pre-quantisation
+    gq, gs = hq.cpu().numpy(), hs.cpu().numpy()
+    deq = oracle.e4m3_decode(gq) * np.repeat(gs.astype(np.float64), 128, axis=1)
+    sfull = np.repeat(gs.astype(np.float64), 128, axis=1)
+    # one e4m3 rounding of the row group (relative 2^-4, or 2^-10 s near zero) plus FP32 noise
+    bound = 2.0 ** -4 * np.abs(ref) + 2.0 ** -10 * sfull + 1e-5 * rms(ref)
+    assert np.all(np.abs(deq - ref) <= bound * (1 + 1e-6))
+    # codes and scales against the oracle's own quantisation of its h
+    oq, os_ = oracle.quant_fp8_rows(ref.astype(np.float32))
+    assert np.mean(gq == oq) >= 0.99
+    np.testing.assert_allclose(gs, os_, rtol=1e-5)
+
+
+@pytest.mark.parametrize("cfg", FP8, ids=FP8_IDS)
+def test_gemm_down_fp8(cfg):
+    inp = make_layer(cfg)
+    layer = M.MoELayer(cfg, inp)
+    ids = random_ids(cfg.T, cfg.E, cfg.k, seed=cfg.seed + 200)
+    _, offsets, _, _ = _gpu_permute(ids.to(DEV), cfg.E)
+    R = cfg.rows()
+    hin = random_bf16((R, cfg.I), seed=cfg.seed, idx=5, std=0.5)
+    hq = torch.empty((R, cfg.I), dtype=torch.uint8, device=DEV)
+    hs = torch.empty((R, cfg.I // 128), dtype=torch.float32, device=DEV)
+    M.quantize_act_fp8(_u16(hin.to(DEV)), hq, hs)
+    o = torch.empty((R, cfg.d), dtype=torch.float32, device=DEV)
+    M.gemm_down(layer.shape(cfg.T), layer.weights, hq, hs, offsets, o, layer.ws)
+    assert M.read_device_status(layer.ws) == M.OK
+    _, ooff, _, _ = oracle.permute(ids.numpy(), cfg.E)
+    ref = oracle.down(oracle_layer(cfg, inp), bf16_to_f64(hin), ooff, cfg.T)
+    assert_close_rel(o.cpu().double().numpy(), ref, rtol=1e-4, atol=1e-4 * rms(ref), what="o")
