@@ -33,7 +33,8 @@ WDTYPE_BF16, WDTYPE_FP8_BLOCK128 = 0, 1
 EXPORTS = ["moe_status_string", "moe_workspace_bytes", "moe_permute_workspace_bytes",
            "moe_router_split", "moe_quantize_weights_fp8", "moe_quantize_act_fp8",
            "moe_quantize_act_fp8_permuted",
-           "moe_router_logits", "moe_route_topk", "moe_permute", "moe_gemm_gateup",
+           "moe_router_logits", "moe_route_topk", "moe_permute", "moe_permute_noalloc",
+           "moe_gemm_gateup",
            "moe_gemm_down", "moe_combine", "moe_forward", "moe_forward_profiled", "moe_forward_host",
            "moe_read_device_status", "moe_selftest_timeout"]
 
@@ -63,6 +64,7 @@ _sig = {
     "moe_router_logits": (_i32, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _vp]),
     "moe_route_topk": (_i32, [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
     "moe_permute": (_i32, [_vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "moe_permute_noalloc": (_i32, [_vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp]),
     "moe_gemm_gateup": (_i32, [_S, _W, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_gemm_down": (_i32, [_S, _W, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_combine": (_i32, [_S, _vp, _vp, _vp, _vp, _vp]),
@@ -159,6 +161,14 @@ def permute(ids, E, counts, offsets, perm, inv, ws, stream=None):
     T, k = ids.shape
     _check(_lib.moe_permute(_p(ids), T, E, k, _p(counts), _p(offsets), _p(perm), _p(inv), _p(ws),
                             ws.numel() * ws.element_size(), _stream(stream)), "moe_permute")
+
+
+def permute_noalloc(ids, E, counts, offsets, perm, inv, stream=None):
+    """moe_permute without a workspace, for callers that cannot allocate:
+    the library's own fixed device scratch is used (see include/moe.h)."""
+    T, k = ids.shape
+    _check(_lib.moe_permute_noalloc(_p(ids), T, E, k, _p(counts), _p(offsets), _p(perm), _p(inv),
+                                    _stream(stream)), "moe_permute_noalloc")
 
 
 def gemm_gateup(shape, weights, x, x_scale, perm, offsets, h, h_scale, ws, stream=None):

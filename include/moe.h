@@ -161,6 +161,27 @@ moe_status moe_permute(const int32_t* ids, int32_t T, int32_t E, int32_t k,
                        int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv,
                        void* ws, size_t ws_bytes, void* stream);
 
+/* moe_permute for callers that cannot allocate device memory (no counterpart
+ * on the pages: an addition of this library).  Same inputs, outputs and
+ * results as moe_permute, but no workspace argument: the scratch lives in a
+ * fixed 256 KiB device array inside the library, which every GPU that loads
+ * the library holds until the process exits.
+ *  - Size limit: permute_segments * E <= 65536 with one segment per 1024
+ *    assignments, i.e. ceil(T*k / 1024) * E <= 65536 (T*k <= 262144 at
+ *    E = 256); larger calls return MOE_ERR_WORKSPACE_TOO_SMALL before any
+ *    launch.
+ *  - The first call on a device looks up the array's device address (once
+ *    per device, with that device current); make that first call before any
+ *    stream capture.
+ *  - All calls share the one array: calls that overlap on the GPU (different
+ *    streams without ordering, or concurrent host threads) race and must be
+ *    serialised by the caller.
+ *  - An expert id outside [0, E) is not placed and, with no workspace to hold
+ *    a status word, not reported; use moe_permute to get the report. */
+moe_status moe_permute_noalloc(const int32_t* ids, int32_t T, int32_t E, int32_t k,
+                               int32_t* counts, int32_t* offsets, int32_t* perm,
+                               int32_t* inv, void* stream);
+
 /* [FM][FP][G8] Grouped Gate-Up GEMM with SiLU*mul epilogue.  Row p < T*k of
  * expert e (offsets[e] <= p < offsets[e+1]) reads token perm[p] / k straight
  * from x (no separate gather); rows T*k .. T*k+T-1 (when I_shared > 0) are
