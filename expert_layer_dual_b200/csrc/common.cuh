@@ -87,6 +87,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64
     }
 }
 
+// Warp-collective form of mbar_wait: every lane waits (and so acquires), and
+// the warp agrees on one outcome, so a timeout makes the whole warp leave
+// its loop together (its later __syncwarp / per-warp arrivals stay matched).
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint64_t timeout_ns,
+                                          const volatile int* abort) {
+    const bool ok = mbar_wait(bar, parity, timeout_ns, abort);
+    return __all_sync(0xffffffffu, ok);
+}
+
 // ------------------------------------------------------------------ TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");

@@ -43,11 +43,11 @@ constexpr int GATEUP_THREADS = 32 * (GATHER_WARP0 + GATHER_WARPS);  // 320
 constexpr int DOWN_THREADS = 32 * (TMA_WARP + 1);                    // 192
 
 struct Bars {
-    uint64_t full_a[STAGES];  // gate-up: 128 gather arrivals; down: unused
+    uint64_t full_a[STAGES];  // gate-up: one arrival per gather warp; down: unused
     uint64_t full_b[STAGES];  // TMA arrival + transaction bytes
     uint64_t empty[STAGES];   // MMA commit
     uint64_t tfull[2];        // accumulator ready (MMA commit)
-    uint64_t tempty[2];       // accumulator drained (128 epilogue arrivals)
+    uint64_t tempty[2];       // accumulator drained (one arrival per epilogue warp)
     uint32_t tmem_slot;
     int abort_flag;
 };
@@ -69,6 +69,12 @@ __device__ __forceinline__ Smem carve_smem(uint8_t* raw) {
     return s;
 }
 
+// All lanes of the warp are done with their part: one lane arrives for it.
+__device__ __forceinline__ void warp_arrive(uint64_t* bar) {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
+
 __device__ __forceinline__ void fail(Bars* b, int32_t* status) {
     report_status(status, MOE_ERR_DEVICE_TIMEOUT);
     *reinterpret_cast<volatile int*>(&b->abort_flag) = 1;
@@ -87,7 +93,7 @@ __device__ __forceinline__ uint32_t prologue(Smem& sm, const GroupedGemmArgs& a,
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&b->tfull[i], 1);
-            mbar_init(&b->tempty[i], EPI_WARPS * 32);
+            mbar_init(&b->tempty[i], EPI_WARPS);
         }
         b->abort_flag = 0;
         fence_barrier_init();
@@ -158,7 +164,7 @@ __global__ void __launch_bounds__(GATEUP_THREADS, 1)
     Bars* b = sm.bars;
     const volatile int* ab = &b->abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const uint32_t tmem = prologue(sm, a, GATHER_WARPS * 32);
+    const uint32_t tmem = prologue(sm, a, GATHER_WARPS);
     const int G = a.E + a.has_shared;
     const int n_tiles = a.I / 128;
     const int total = sm.tt->mstart[G] * n_tiles;
@@ -237,7 +243,7 @@ __global__ void __launch_bounds__(GATEUP_THREADS, 1)
             for (int kb = 0; kb < nk; ++kb, ++it) {
                 const int s = it % STAGES;
                 const uint32_t ph = (it / STAGES) & 1;
-                if (!mbar_wait(&b->empty[s], ph ^ 1, a.timeout_ns, ab)) {
+                if (!warp_wait(&b->empty[s], ph ^ 1, a.timeout_ns, ab)) {
                     fail(b, a.status);
                     ok = false;
                     break;
@@ -250,7 +256,7 @@ __global__ void __launch_bounds__(GATEUP_THREADS, 1)
                 if (pend0 >= 0) {
                     cp_async_wait<2>();  // the oldest of the three groups in flight is done
                     fence_proxy_async_smem();
-                    mbar_arrive(&b->full_a[pend0]);
+                    warp_arrive(&b->full_a[pend0]);
                 }
                 pend0 = pend1;
                 pend1 = s;
@@ -258,8 +264,8 @@ __global__ void __launch_bounds__(GATEUP_THREADS, 1)
         }
         cp_async_wait<0>();
         fence_proxy_async_smem();
-        if (pend0 >= 0) mbar_arrive(&b->full_a[pend0]);
-        if (pend1 >= 0) mbar_arrive(&b->full_a[pend1]);
+        if (pend0 >= 0) warp_arrive(&b->full_a[pend0]);
+        if (pend1 >= 0) warp_arrive(&b->full_a[pend1]);
     } else if (warp == MMA_WARP) {
         if (lane == 0) mma_role(sm, a, tmem, G, n_tiles, true);
     } else {
@@ -269,7 +275,7 @@ __global__ void __launch_bounds__(GATEUP_THREADS, 1)
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++lt) {
             const Tile t = decode_tile(sm.tt, G, n_tiles, tile, BM);
             const uint32_t buf = lt & 1, tph = (lt >> 1) & 1;
-            if (!mbar_wait(&b->tfull[buf], tph, a.timeout_ns, ab)) { fail(b, a.status); break; }
+            if (!warp_wait(&b->tfull[buf], tph, a.timeout_ns, ab)) { fail(b, a.status); break; }
             tc_fence_after_sync();
             const uint32_t taddr = tmem + (static_cast<uint32_t>(warp * 32) << 16) + buf * BN;
             uint16_t* dst = h + (int64_t)(t.row0 + row) * a.I + t.n * 128;
@@ -290,7 +296,7 @@ __global__ void __launch_bounds__(GATEUP_THREADS, 1)
                 }
             }
             tc_fence_before_sync();
-            mbar_arrive(&b->tempty[buf]);
+            warp_arrive(&b->tempty[buf]);
         }
     }
     teardown(sm, tmem);
@@ -357,7 +363,7 @@ __global__ void __launch_bounds__(DOWN_THREADS, 1)
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++lt) {
             const Tile t = decode_tile(sm.tt, G, n_tiles, tile, BM);
             const uint32_t buf = lt & 1, tph = (lt >> 1) & 1;
-            if (!mbar_wait(&b->tfull[buf], tph, a.timeout_ns, ab)) { fail(b, a.status); break; }
+            if (!warp_wait(&b->tfull[buf], tph, a.timeout_ns, ab)) { fail(b, a.status); break; }
             tc_fence_after_sync();
             const uint32_t taddr = tmem + (static_cast<uint32_t>(warp * 32) << 16) + buf * BN;
             const int ncols = min(BN, a.d - t.n * BN);
@@ -376,7 +382,7 @@ __global__ void __launch_bounds__(DOWN_THREADS, 1)
                 }
             }
             tc_fence_before_sync();
-            mbar_arrive(&b->tempty[buf]);
+            warp_arrive(&b->tempty[buf]);
         }
     }
     teardown(sm, tmem);

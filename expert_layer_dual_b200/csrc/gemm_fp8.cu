@@ -14,16 +14,17 @@
 //  - one thread issues four kind::f8f6f4 MMAs (K = 32 each) that write a
 //    fresh partial product of the k-block into one of two 256-column TMEM
 //    buffers, so the next k-block's MMAs run while this one is promoted;
-//  - eight epilogue warps (two per TMEM lane quadrant, each owning half of
-//    the columns) read the partial with tcgen05.ld and accumulate
-//    s_a[row] * s_w * P into FP32 registers;
+//  - sixteen epilogue warps (four per TMEM lane quadrant, each owning a
+//    quarter of the columns, so four warps per scheduler hide the TMEM load
+//    latency) read the partial with tcgen05.ld and accumulate
+//    s_a[row] * s_w * P into 64 FP32 registers per thread;
 //  - operands arrive by TMA into a 4-stage ring (128-byte swizzle).  The
 //    gate-up A rows are the activation quantisation's output, already
 //    written in permuted row order, so both operands are plain tiles.
 // Gate-up's tile is 128 rows x (128 gate + 128 up) columns: each row's 128
 // h values form exactly one 1x128 quantisation group, so the epilogue
-// computes h = silu(g) * u, the group's amax (combining the two column
-// halves through shared memory) and writes e4m3 h with its scale.  Down's
+// computes h = silu(g) * u, the group's amax (combining the four column
+// quarters through shared memory) and writes e4m3 h with its scale.  Down's
 // tile is 128 rows x 256 output columns (two weight scale blocks) and writes
 // FP32 o.  Every wait is bounded, as in the BF16 kernels.
 #include "common.cuh"
@@ -39,18 +40,18 @@ constexpr int B_HALF = 128 * BK;       // 16 KB
 constexpr int B_BYTES = 2 * B_HALF;    // 32 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr uint32_t TMEM_COLS = 512;    // two 256-column partial buffers
-constexpr int EPI_WARPS = 8, MMA_WARP = 8, TMA_WARP = 9;
-constexpr int THREADS = 32 * (TMA_WARP + 1);  // 320
+constexpr int EPI_WARPS = 16, MMA_WARP = 16, TMA_WARP = 17;
+constexpr int THREADS = 32 * (TMA_WARP + 1);  // 576
 
 struct Bars {
     uint64_t full[STAGES];   // TMA arrival + transaction bytes
     uint64_t empty[STAGES];  // MMA commit
     uint64_t pfull[2];       // partial ready (MMA commit)
-    uint64_t pempty[2];      // partial consumed (256 epilogue arrivals)
-    uint64_t amax_bar[2];    // gate-up: both column halves' amax written (256 arrivals)
+    uint64_t pempty[2];      // partial consumed (one arrival per epilogue warp)
+    uint64_t amax_bar[2];    // gate-up: the four quarters' amax written (one per warp)
     uint32_t tmem_slot;
     int abort_flag;
-    float amax[2][2][BM];    // [tile parity][column half][row]
+    float amax[2][4][BM];    // [tile parity][column quarter][row]
 };
 
 constexpr size_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + sizeof(Bars) + sizeof(TileTable) + 64;
@@ -85,8 +86,8 @@ __device__ __forceinline__ uint32_t prologue(Smem& sm, const GroupedGemmArgs& a)
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&b->pfull[i], 1);
-            mbar_init(&b->pempty[i], EPI_WARPS * 32);
-            mbar_init(&b->amax_bar[i], EPI_WARPS * 32);
+            mbar_init(&b->pempty[i], EPI_WARPS);
+            mbar_init(&b->amax_bar[i], EPI_WARPS);
         }
         b->abort_flag = 0;
         fence_barrier_init();
@@ -182,20 +183,27 @@ __device__ __forceinline__ void mma_role(Smem& sm, const GroupedGemmArgs& a, uin
     }
 }
 
-// One promotion step of an epilogue thread: acc[0..63] += f0 * cols c0..c0+63,
-// acc[64..127] += f1 * cols c1..c1+63 of its TMEM lane, 16 columns per load
-// to keep the register footprint at the 128 accumulators plus one chunk.
+// One promotion step of an epilogue thread: acc[0..31] += f0 * cols
+// c0..c0+31 and acc[32..63] += f1 * cols c1..c1+31 of its TMEM lane, 16
+// columns per load to keep the footprint at 64 accumulators plus one chunk.
 __device__ __forceinline__ void promote(uint32_t lane_base, int c0, int c1, float f0, float f1,
                                         float* acc) {
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
+    for (int q = 0; q < 4; ++q) {
         float v[16];
-        const int col = (q < 4 ? c0 : c1) + (q & 3) * 16;
-        const float f = q < 4 ? f0 : f1;
+        const int col = (q < 2 ? c0 : c1) + (q & 1) * 16;
+        const float f = q < 2 ? f0 : f1;
         tmem_load16(lane_base + col, v);
 #pragma unroll
         for (int i = 0; i < 16; ++i) acc[q * 16 + i] = fmaf(f, v[i], acc[q * 16 + i]);
     }
+}
+
+// All lanes of the warp are done with their part (TMEM loads waited for,
+// shared-memory writes issued): one lane arrives for the warp.
+__device__ __forceinline__ void warp_arrive(uint64_t* bar) {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
 }
 
 __device__ __forceinline__ uint32_t quant4(float a, float b, float c, float d, float s) {
@@ -241,8 +249,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     } else if (warp == MMA_WARP) {
         if (lane == 0) mma_role(sm, a, tmem, G, n_tiles, nk);
     } else {
-        // ---------------- 8 epilogue warps
-        const int quad = warp & 3, half = warp >> 2;
+        // ---------------- 16 epilogue warps
+        const int quad = warp & 3, qtr = warp >> 2;
         const int row = quad * 32 + lane;
         const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
         const int total = sm.tt->mstart[G] * n_tiles;
@@ -256,53 +264,60 @@ __global__ void __launch_bounds__(THREADS, 1)
                                       : wsc + ((int64_t)t.g * nbs + a.I / 128 + t.n) * kbs;
             const bool valid = row < t.nrows;
             const float* sa_row = xs + (int64_t)(valid ? t.row0 + row : 0) * kbs;
-            float acc[128];
+            float acc[64];
 #pragma unroll
-            for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
+            for (int i = 0; i < 64; ++i) acc[i] = 0.0f;
             bool ok = true;
+            // scales of the next k-block load while this one is promoted
+            float sa_n = valid ? __ldg(sa_row) : 0.0f, sg_n = __ldg(swg), su_n = __ldg(swu);
             for (int kb = 0; kb < nk; ++kb, ++it) {
                 const uint32_t pb = it & 1, pph = (it >> 1) & 1;
-                const float sa = valid ? __ldg(sa_row + kb) : 0.0f;
-                const float fg = sa * __ldg(swg + kb), fu = sa * __ldg(swu + kb);
-                if (!mbar_wait(&b->pfull[pb], pph, a.timeout_ns, ab)) {
+                const float fg = sa_n * sg_n, fu = sa_n * su_n;
+                if (kb + 1 < nk) {
+                    sa_n = valid ? __ldg(sa_row + kb + 1) : 0.0f;
+                    sg_n = __ldg(swg + kb + 1);
+                    su_n = __ldg(swu + kb + 1);
+                }
+                if (!warp_wait(&b->pfull[pb], pph, a.timeout_ns, ab)) {
                     fail(b, a.status);
                     ok = false;
                     break;
                 }
                 tc_fence_after_sync();
                 const uint32_t base = tmem + lane_off + pb * BN;
-                promote(base, half * 64, 128 + half * 64, fg, fu, acc);
+                promote(base, qtr * 32, 128 + qtr * 32, fg, fu, acc);
                 tc_fence_before_sync();
-                mbar_arrive(&b->pempty[pb]);
+                warp_arrive(&b->pempty[pb]);
             }
             if (!ok) break;
-            // h = silu(g) * u on this thread's 64 columns, then the row's group amax
+            // h = silu(g) * u on this thread's 32 columns, then the row's group amax
             float amax = 0.0f;
 #pragma unroll
-            for (int i = 0; i < 64; ++i) {
-                acc[i] = silu_f(acc[i]) * acc[64 + i];
+            for (int i = 0; i < 32; ++i) {
+                acc[i] = silu_f(acc[i]) * acc[32 + i];
                 amax = fmaxf(amax, fabsf(acc[i]));
             }
-            // the two column halves of a row meet in shared memory; the
+            // the four column quarters of a row meet in shared memory; the
             // exchange waits on an mbarrier (bounded), double-buffered by tile
             const int par = lt & 1;
-            b->amax[par][half][row] = amax;
-            mbar_arrive(&b->amax_bar[par]);
-            if (!mbar_wait(&b->amax_bar[par], (lt >> 1) & 1, a.timeout_ns, ab)) {
+            b->amax[par][qtr][row] = amax;
+            warp_arrive(&b->amax_bar[par]);
+            if (!warp_wait(&b->amax_bar[par], (lt >> 1) & 1, a.timeout_ns, ab)) {
                 fail(b, a.status);
                 break;
             }
-            amax = fmaxf(b->amax[par][0][row], b->amax[par][1][row]);
+            amax = fmaxf(fmaxf(b->amax[par][0][row], b->amax[par][1][row]),
+                         fmaxf(b->amax[par][2][row], b->amax[par][3][row]));
             const float s = amax == 0.0f ? 1.0f : __fdiv_rn(amax, 448.0f);
             if (valid) {
-                uint8_t* dst = hq + (int64_t)(t.row0 + row) * a.I + t.n * 128 + half * 64;
+                uint8_t* dst = hq + (int64_t)(t.row0 + row) * a.I + t.n * 128 + qtr * 32;
 #pragma unroll
-                for (int q = 0; q < 4; ++q)
+                for (int q = 0; q < 2; ++q)
                     st_global_v4(dst + q * 16, quant4(acc[16 * q], acc[16 * q + 1], acc[16 * q + 2], acc[16 * q + 3], s),
                                  quant4(acc[16 * q + 4], acc[16 * q + 5], acc[16 * q + 6], acc[16 * q + 7], s),
                                  quant4(acc[16 * q + 8], acc[16 * q + 9], acc[16 * q + 10], acc[16 * q + 11], s),
                                  quant4(acc[16 * q + 12], acc[16 * q + 13], acc[16 * q + 14], acc[16 * q + 15], s));
-                if (half == 0) hs[(int64_t)(t.row0 + row) * (a.I / 128) + t.n] = s;
+                if (qtr == 0) hs[(int64_t)(t.row0 + row) * (a.I / 128) + t.n] = s;
             }
         }
     }
@@ -343,7 +358,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     } else if (warp == MMA_WARP) {
         if (lane == 0) mma_role(sm, a, tmem, G, n_tiles, nk);
     } else {
-        const int quad = warp & 3, half = warp >> 2;
+        const int quad = warp & 3, qtr = warp >> 2;
         const int row = quad * 32 + lane;
         const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
         const int total = sm.tt->mstart[G] * n_tiles;
@@ -351,35 +366,38 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
             const Tile t = decode_tile(sm.tt, G, n_tiles, tile, BM);
             const bool shared = t.g >= a.E;
-            const int nb = 2 * t.n + half;                 // this half's weight scale block
-            const bool live = nb < nbs;                     // inside d
+            const int nb = 2 * t.n + (qtr >> 1);             // this quarter's weight scale block
+            const bool live = nb < nbs;                       // inside d
             const float* sw = shared ? wssc + (int64_t)(live ? nb : 0) * kbs
                                      : wsc + ((int64_t)t.g * nbs + (live ? nb : 0)) * kbs;
             const bool valid = row < t.nrows;
             const float* sa_row = hs + (int64_t)(valid ? t.row0 + row : 0) * kbs;
-            float acc[128];
+            float acc[64];
 #pragma unroll
-            for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
+            for (int i = 0; i < 64; ++i) acc[i] = 0.0f;
             bool ok = true;
+            const bool use = valid && live;
+            float f_n = use ? __ldg(sa_row) * __ldg(sw) : 0.0f;
             for (int kb = 0; kb < nk; ++kb, ++it) {
                 const uint32_t pb = it & 1, pph = (it >> 1) & 1;
-                const float f = (valid && live) ? __ldg(sa_row + kb) * __ldg(sw + kb) : 0.0f;
-                if (!mbar_wait(&b->pfull[pb], pph, a.timeout_ns, ab)) {
+                const float f = f_n;
+                if (kb + 1 < nk) f_n = use ? __ldg(sa_row + kb + 1) * __ldg(sw + kb + 1) : 0.0f;
+                if (!warp_wait(&b->pfull[pb], pph, a.timeout_ns, ab)) {
                     fail(b, a.status);
                     ok = false;
                     break;
                 }
                 tc_fence_after_sync();
                 const uint32_t base = tmem + lane_off + pb * BN;
-                promote(base, half * 128, half * 128 + 64, f, f, acc);
+                promote(base, qtr * 64, qtr * 64 + 32, f, f, acc);
                 tc_fence_before_sync();
-                mbar_arrive(&b->pempty[pb]);
+                warp_arrive(&b->pempty[pb]);
             }
             if (!ok) break;
             if (valid && live) {
-                float* dst = o + (int64_t)(t.row0 + row) * a.d + t.n * BN + half * 128;
+                float* dst = o + (int64_t)(t.row0 + row) * a.d + t.n * BN + qtr * 64;
 #pragma unroll
-                for (int q = 0; q < 32; ++q)
+                for (int q = 0; q < 16; ++q)
                     st_global_v4(dst + 4 * q, __float_as_uint(acc[4 * q]), __float_as_uint(acc[4 * q + 1]),
                                  __float_as_uint(acc[4 * q + 2]), __float_as_uint(acc[4 * q + 3]));
             }

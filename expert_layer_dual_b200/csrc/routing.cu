@@ -321,26 +321,43 @@ __device__ __forceinline__ float group_scale(float amax) {
     return amax == 0.0f ? 1.0f : __fdiv_rn(amax, 448.0f);
 }
 
-// one warp per (row, 128-column group); lane holds 4 consecutive values
+// One warp quantises one row: each step covers two 128-column groups, lanes
+// 0-15 the first and 16-31 the second, 8 values (16 bytes) per lane; the
+// group amax is a 16-lane shuffle reduction.
+__device__ __forceinline__ void quant_row(const uint16_t* __restrict__ src, int cols,
+                                          uint8_t* __restrict__ qrow, float* __restrict__ srow) {
+    const int lane = threadIdx.x & 31;
+    const int groups = cols / 128;
+    const int half = lane >> 4, l16 = lane & 15;
+    for (int g0 = 0; g0 < groups; g0 += 2) {
+        const int g = g0 + half;
+        const bool active = g < groups;
+        uint4 u = make_uint4(0, 0, 0, 0);
+        if (active) u = *reinterpret_cast<const uint4*>(src + g * 128 + l16 * 8);
+        float f[8];
+        bf16x8_to_f32(u, f);
+        float amax = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        const float s = group_scale(amax);
+        if (active) {
+            uint2 q;
+            q.x = quant4_e4m3(f[0], f[1], f[2], f[3], s);
+            q.y = quant4_e4m3(f[4], f[5], f[6], f[7], s);
+            *reinterpret_cast<uint2*>(qrow + g * 128 + l16 * 8) = q;
+            if (l16 == 0) srow[g] = s;
+        }
+    }
+}
+
 __global__ void __launch_bounds__(256)
     k_quant_act(const uint16_t* __restrict__ x, int64_t rows, int cols, uint8_t* __restrict__ q,
                 float* __restrict__ scale) {
-    const int64_t gw = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
-    const int lane = threadIdx.x & 31;
-    const int groups = cols / 128;
-    if (gw >= rows * groups) return;
-    const int64_t r = gw / groups;
-    const int g = (int)(gw % groups);
-    const int64_t off = r * cols + g * 128 + lane * 4;
-    const uint2 raw = *reinterpret_cast<const uint2*>(x + off);
-    const float v0 = __uint_as_float(raw.x << 16), v1 = __uint_as_float(raw.x & 0xffff0000u);
-    const float v2 = __uint_as_float(raw.y << 16), v3 = __uint_as_float(raw.y & 0xffff0000u);
-    float amax = fmaxf(fmaxf(fabsf(v0), fabsf(v1)), fmaxf(fabsf(v2), fabsf(v3)));
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    const float s = group_scale(amax);
-    *reinterpret_cast<uint32_t*>(q + off) = quant4_e4m3(v0, v1, v2, v3, s);
-    if (lane == 0) scale[r * groups + g] = s;
+    const int64_t r = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+    if (r >= rows) return;
+    quant_row(x + r * cols, cols, q + r * cols, scale + r * (cols / 128));
 }
 
 // Same quantisation, written in the permuted row order of the grouped GEMMs:
@@ -351,42 +368,27 @@ __global__ void __launch_bounds__(256)
     k_quant_act_permuted(const uint16_t* __restrict__ x, const int32_t* __restrict__ perm, int T,
                          int k, int64_t rows, int cols, uint8_t* __restrict__ q,
                          float* __restrict__ scale) {
-    const int64_t gw = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
-    const int lane = threadIdx.x & 31;
-    const int groups = cols / 128;
-    if (gw >= rows * groups) return;
-    const int64_t p = gw / groups;
-    const int g = (int)(gw % groups);
+    const int64_t p = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+    if (p >= rows) return;
     const int64_t Tk = (int64_t)T * k;
     const int64_t tok = p < Tk ? (int64_t)(perm[p] / k) : p - Tk;
-    const uint2 raw = *reinterpret_cast<const uint2*>(x + tok * cols + g * 128 + lane * 4);
-    const float v0 = __uint_as_float(raw.x << 16), v1 = __uint_as_float(raw.x & 0xffff0000u);
-    const float v2 = __uint_as_float(raw.y << 16), v3 = __uint_as_float(raw.y & 0xffff0000u);
-    float amax = fmaxf(fmaxf(fabsf(v0), fabsf(v1)), fmaxf(fabsf(v2), fabsf(v3)));
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    const float s = group_scale(amax);
-    *reinterpret_cast<uint32_t*>(q + p * cols + g * 128 + lane * 4) = quant4_e4m3(v0, v1, v2, v3, s);
-    if (lane == 0) scale[p * groups + g] = s;
+    quant_row(x + tok * cols, cols, q + p * cols, scale + p * (cols / 128));
 }
 
 cudaError_t launch_quant_act_fp8_permuted(const uint16_t* x, const int32_t* perm, int T, int k,
                                           int has_shared, int cols, uint8_t* q, float* scale,
                                           cudaStream_t s) {
     const int64_t rows = (int64_t)T * k + (has_shared ? T : 0);
-    const int64_t warps = rows * (cols / 128);
-    if (warps == 0) return cudaSuccess;
-    k_quant_act_permuted<<<(unsigned)((warps + 7) / 8), 256, 0, s>>>(x, perm, T, k, rows, cols, q,
-                                                                      scale);
+    if (rows == 0) return cudaSuccess;
+    k_quant_act_permuted<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(x, perm, T, k, rows, cols, q,
+                                                                     scale);
     return cudaGetLastError();
 }
 
 cudaError_t launch_quant_act_fp8(const uint16_t* x, int64_t rows, int cols, uint8_t* q,
                                  float* scale, cudaStream_t s) {
-    const int64_t warps = rows * (cols / 128);
-    if (warps == 0) return cudaSuccess;
-    const int64_t blocks = (warps + 7) / 8;
-    k_quant_act<<<(unsigned)blocks, 256, 0, s>>>(x, rows, cols, q, scale);
+    if (rows == 0) return cudaSuccess;
+    k_quant_act<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(x, rows, cols, q, scale);
     return cudaGetLastError();
 }
 
