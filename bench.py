@@ -45,7 +45,7 @@ from expert_layer_dual_b200.inputs import make_layer  # noqa: E402
 METRIC = "fused MoE layer tokens/s"
 UNIT = "tokens/s"
 # oracle token sample per step of the CPU baseline / reference arm
-CPU_SAMPLE = {"tiny": 16, "decode": 16, "prefill": 8, "fp8": 4, "skew": 8}
+CPU_SAMPLE = {"tiny": 16, "decode": 64, "prefill": 16, "fp8": 8, "skew": 16}
 
 
 def cpu_sample(cfg: MoEConfig) -> int:
@@ -161,6 +161,39 @@ def load_peaks():
     return 6650.0, 1590.0, "fallback"
 
 
+# DRAM traffic of the dominant kernel, from an ncu capture (dram__bytes_read.sum +
+# dram__bytes_write.sum of one launch) recorded in profiles/dram_traffic.txt with a
+# hash of the kernel's sources; reported only while the sources still match.
+KERNEL_SOURCES = {
+    "k_gateup_bf16": ["csrc/gemm_bf16.cu", "csrc/common.cuh", "csrc/grouped_common.cuh"],
+    "k_gateup_fp8": ["csrc/gemm_fp8.cu", "csrc/common.cuh", "csrc/grouped_common.cuh"],
+}
+
+
+def kernel_source_hash(kernel: str) -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(ROOT, "expert_layer_dual_b200", rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """(bytes per launch, note) if profiles/dram_traffic.txt holds a capture of
+    `kernel` on `workload` taken from the current sources, else (None, why)."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(path):
+        return None, "no capture recorded"
+    for line in open(path):
+        parts = line.split()
+        if len(parts) >= 4 and not line.startswith("#") and parts[0] == kernel and parts[1] == workload:
+            if parts[3] != kernel_source_hash(kernel):
+                return None, "kernel changed since the capture"
+            return int(parts[2]), "ncu capture, profiles/dram_traffic.txt"
+    return None, "no capture for this workload"
+
+
 def gateup_algorithmic(cfg: MoEConfig, T: int, n_active: int):
     """Algorithmic work of one gate-up launch: FLOPs, and bytes = the weights
     of every expert that received tokens (+ shared) read once, x read once,
@@ -187,9 +220,9 @@ def _bits(t):
     return t.detach().contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
 
 
-def oracle_sample_time(cfg: MoEConfig, inp: dict, n_tokens: int, repeats: int = 1):
-    """Seconds the oracle takes for the whole layer on n_tokens of the
-    workload (host copies made first, outside the timing)."""
+def oracle_sample(cfg: MoEConfig, inp: dict, n_tokens: int):
+    """Host inputs of the oracle for the first n_tokens of the workload: x rows,
+    the router weight and the experts the oracle's own routing selects."""
     import oracle
     oracle.build()
     n = min(n_tokens, cfg.T)
@@ -208,12 +241,18 @@ def oracle_sample_time(cfg: MoEConfig, inp: dict, n_tokens: int, repeats: int = 
                      ws_gu=None if inp.get("ws_gu") is None else _bits(inp["ws_gu"]),
                      ws_d=None if inp.get("ws_d") is None else _bits(inp["ws_d"]),
                      router_w=rw, router_bias=bias, wdtype=cfg.wdtype, renorm=cfg.renorm)
+    return L, xs
+
+
+def oracle_times(L, xs, repeats: int):
+    """Seconds of each of `repeats` whole-layer oracle runs on the sample."""
+    import oracle
     times = []
     for _ in range(repeats):
         t0 = time.perf_counter()
         oracle.forward(L, xs)
         times.append(time.perf_counter() - t0)
-    return times, n, oracle.num_threads()
+    return times
 
 
 def run_reference(args, cfg: MoEConfig):
@@ -221,11 +260,15 @@ def run_reference(args, cfg: MoEConfig):
     if rank != 0:
         return
     inp = make_layer(cfg, device="cuda" if torch.cuda.is_available() else "cpu")
+    import oracle
     # size the per-step sample so the whole run stays within a few minutes
-    t1, _, _ = oracle_sample_time(cfg, inp, 1, repeats=1)
+    L1, x1 = oracle_sample(cfg, inp, 1)
+    t1 = oracle_times(L1, x1, 1)
     budget = 150.0 / (args.warmup + args.steps)
     n = int(max(1, min(cpu_sample(cfg), budget / max(t1[0], 1e-3))))
-    times, n, cores = oracle_sample_time(cfg, inp, n, repeats=args.warmup + args.steps)
+    L, xs = oracle_sample(cfg, inp, n)
+    n = xs.shape[0]
+    times, cores = oracle_times(L, xs, args.warmup + args.steps), oracle.num_threads()
     timed = times[args.warmup:]
     tps = n * len(timed) / sum(timed)
     sample = f"{n} tokens of the {cfg.name} workload per step (whole layer, FP64)"
@@ -324,7 +367,7 @@ def run_ours(args, cfg: MoEConfig):
     roof["peak_source"] = (f"{peak_kind} MEASURED_PEAKS.json "
                            + ("hbm_gbs" if roof["bound"] == "hbm" else "bf16_tflops (burst: the timed loop is well under a second)"
                               + (" x2 (e4m3 nominal ratio)" if cfg.wdtype else "")))
-    roof["traffic"] = None
+    roof["traffic"], roof["traffic_source"] = recorded_traffic(roof["kernel"], cfg.name)
     roof["algorithmic_bytes"] = gu_bytes
     roof["algorithmic_flops"] = gu_flops
     roof["launch_ms"] = gu_ms
@@ -351,11 +394,17 @@ def run_ours(args, cfg: MoEConfig):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        n = cpu_sample(cfg)
-        times, n, cores = oracle_sample_time(cfg, inp, n, repeats=1)
-        cpu = {"value": n / times[0], "unit": UNIT, "cores": cores, "kind": "oracle",
-               "sample": f"first {n} tokens of the {cfg.name} batch, whole layer in FP64 "
-                         f"({times[0]:.1f} s)"}
+        import oracle
+        L, xs = oracle_sample(cfg, inp, cpu_sample(cfg))
+        n, cores = xs.shape[0], oracle.num_threads()
+        times = oracle_times(L, xs, 1)
+        # repeat up to about 10 s of CPU work (at most 30 s)
+        reps = int(min(30.0, max(10.0, times[0])) // max(times[0], 1e-3))
+        if reps > 1:
+            times += oracle_times(L, xs, reps - 1)
+        cpu = {"value": n * len(times) / sum(times), "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": f"first {n} tokens of the {cfg.name} batch, whole layer in FP64, "
+                         f"{len(times)} runs, {sum(times):.1f} s of CPU time"}
 
     kernels_per_step = 8 + (1 if cfg.wdtype else 0)
     if rank == 0:
