@@ -74,7 +74,8 @@ namespace {
 inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 struct WsLayout {
-    size_t logits, ids, w, counts, offsets, perm, inv, seg, xq, xs, h, hs, o, xin, yout, total;
+    size_t logits, part, ids, w, counts, offsets, perm, inv, seg, xq, xs, h, hs, o, xin, yout, total;
+    int ksplit;
 };
 
 WsLayout ws_layout(const moe_shape& s) {
@@ -89,6 +90,8 @@ WsLayout ws_layout(const moe_shape& s) {
                  I = (size_t)s.I;
     const size_t R = T * k + (s.I_shared > 0 ? T : 0);
     L.logits = take(T * E * 4);
+    L.ksplit = router_ksplit(s.T, s.d, s.E);
+    L.part = L.ksplit > 1 ? take(2 * (size_t)L.ksplit * T * E * 4) : 0;  // split-K router partials
     L.ids = take(T * k * 4);
     L.w = take(T * k * 4);
     L.counts = take(E * 4);
@@ -231,13 +234,27 @@ moe_status forward_device(const moe_shape* s, const moe_weights* w, const uint16
     moe_status r;
     if (cudaMemsetAsync(status, 0, sizeof(int32_t), st) != cudaSuccess) return MOE_ERR_CUDA;
     if (!mark(0)) return MOE_ERR_CUDA;
-    if ((r = cuda_status(launch_router_logits(x, w->router_hi, w->router_lo, w->router_bias, logits,
-                                              s->T, s->d, s->E, status, st))) != MOE_OK)
-        return r;
-    if (!mark(1)) return MOE_ERR_CUDA;
-    if ((r = cuda_status(launch_route_topk(logits, s->T, s->E, s->k, s->renormalize, ids, rw, st))) !=
-        MOE_OK)
-        return r;
+    if (L.ksplit == 1) {
+        if ((r = cuda_status(launch_router_logits(x, w->router_hi, w->router_lo, w->router_bias,
+                                                  logits, s->T, s->d, s->E, status, st))) != MOE_OK)
+            return r;
+        if (!mark(1)) return MOE_ERR_CUDA;
+        if ((r = cuda_status(launch_route_topk(logits, s->T, s->E, s->k, s->renormalize, ids, rw,
+                                               st))) != MOE_OK)
+            return r;
+    } else {
+        // few tokens: K split across CTAs, partials combined inside the top-k kernel
+        float* ph = at<float>(ws, L.part);
+        float* pl = ph + (size_t)L.ksplit * s->T * s->E;
+        if ((r = cuda_status(launch_router_partials(x, w->router_hi, w->router_lo, ph, pl, L.ksplit,
+                                                    s->T, s->d, s->E, status, st))) != MOE_OK)
+            return r;
+        if (!mark(1)) return MOE_ERR_CUDA;
+        if ((r = cuda_status(launch_route_topk_partials(ph, pl, L.ksplit, w->router_bias, logits,
+                                                        s->T, s->E, s->k, s->renormalize, ids, rw,
+                                                        st))) != MOE_OK)
+            return r;
+    }
     if (!mark(2)) return MOE_ERR_CUDA;
     if ((r = cuda_status(launch_permute(ids, s->T, s->E, s->k, counts, offsets, perm, inv, seg,
                                         status, st))) != MOE_OK)

@@ -24,6 +24,11 @@ cudaError_t launch_router_split(const float* W, uint16_t* hi, uint16_t* lo, int6
                                 cudaStream_t s);
 cudaError_t launch_route_topk(const float* logits, int T, int E, int k, int renorm, int32_t* ids,
                               float* w, cudaStream_t s);
+// Top-k on router partial sums (split-K router): logits = sum_ks part_hi (pairwise)
+// + sum_ks part_lo / 256 + bias, also written to `logits`.
+cudaError_t launch_route_topk_partials(const float* part_hi, const float* part_lo, int ksplit,
+                                       const float* bias, float* logits, int T, int E, int k,
+                                       int renorm, int32_t* ids, float* w, cudaStream_t s);
 // Scratch: seg_hist [nseg][E] int32, nseg = permute_segments(T*k).
 int permute_segments(int64_t n_assign);
 cudaError_t launch_permute(const int32_t* ids, int T, int E, int k, int32_t* counts,
@@ -45,6 +50,13 @@ cudaError_t launch_selftest_timeout(int32_t* status, uint64_t limit_ns, cudaStre
 cudaError_t launch_router_logits(const uint16_t* x, const uint16_t* hi, const uint16_t* lo,
                                  const float* bias, float* logits, int T, int d, int E,
                                  int32_t* status, cudaStream_t s);
+
+// K split of the router GEMM for T tokens (1 = one CTA per tile covers all of d).
+int router_ksplit(int T, int d, int E);
+// Partial sums [ksplit][T][E] of the hi and lo products (no bias, no combination).
+cudaError_t launch_router_partials(const uint16_t* x, const uint16_t* hi, const uint16_t* lo,
+                                   float* part_hi, float* part_lo, int ksplit, int T, int d, int E,
+                                   int32_t* status, cudaStream_t s);
 
 // ---- gemm_bf16.cu (tcgen05 grouped GEMMs)
 struct GroupedGemmArgs {

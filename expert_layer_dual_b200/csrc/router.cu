@@ -21,6 +21,11 @@
 // of the k-blocks, summed pairwise in FP32 by the epilogue before the single
 // correcting FMA; lo (already scaled down by 256) keeps one accumulator.
 // TMEM columns: hi chunk c at c*64 .. c*64+63, lo at C*64 .. C*64+63.
+//
+// Few tokens (decode): one 128-token tile row gives only E/64 CTAs, so the
+// K dimension is also split across CTAs (grid z = ksplit); each CTA then
+// writes its partial hi and lo sums, and the top-k kernel adds the ksplit
+// partials in a fixed pairwise order before the correcting FMA.
 #include "common.cuh"
 #include "launch.h"
 
@@ -39,7 +44,8 @@ constexpr size_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
 __global__ void __launch_bounds__(THREADS, 1)
     k_router_dual(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_hi,
                   const __grid_constant__ CUtensorMap tm_lo, const float* __restrict__ bias,
-                  float* __restrict__ logits, int T, int d, int E, int32_t* status,
+                  float* __restrict__ logits, float* __restrict__ part_hi,
+                  float* __restrict__ part_lo, int T, int d, int E, int32_t* status,
                   uint64_t timeout_ns) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -52,7 +58,10 @@ __global__ void __launch_bounds__(THREADS, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int m0 = blockIdx.x * BM, e0 = blockIdx.y * BN;
-    const int nk = d / BK;
+    const int ksplit = gridDim.z, ks = blockIdx.z;
+    const int nk_all = d / BK;
+    const int kb0 = ks * nk_all / ksplit;                // this CTA's k-blocks: kb0 .. kb0+nk-1
+    const int nk = (ks + 1) * nk_all / ksplit - kb0;
     const int nchunks = nk < MAX_CHUNKS ? nk : MAX_CHUNKS;
 
     if (threadIdx.x == 0) {
@@ -86,9 +95,9 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
             uint8_t* st = smem + s * STAGE_BYTES;
             mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
-            tma_load_2d(st, &tm_x, &full[s], kb * BK, m0);
-            tma_load_2d(st + A_BYTES, &tm_hi, &full[s], kb * BK, e0);
-            tma_load_2d(st + A_BYTES + B_BYTES, &tm_lo, &full[s], kb * BK, e0);
+            tma_load_2d(st, &tm_x, &full[s], (kb0 + kb) * BK, m0);
+            tma_load_2d(st + A_BYTES, &tm_hi, &full[s], (kb0 + kb) * BK, e0);
+            tma_load_2d(st + A_BYTES + B_BYTES, &tm_lo, &full[s], (kb0 + kb) * BK, e0);
             ++issued;
         }
         if (*abort_flag) {  // let the copies still in flight land before the block exits
@@ -148,7 +157,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
                     for (int i = 0; i < 32; ++i) h[i] += (nchunks == 4) ? (h2[i] + h3[i]) : h2[i];
                 }
-                if (t < T) {
+                if (t < T && ksplit == 1) {
                     float* dst = logits + (int64_t)t * E;
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
@@ -157,6 +166,17 @@ __global__ void __launch_bounds__(THREADS, 1)
                             float v = fmaf(l[i], 0.00390625f, h[i]);
                             if (bias != nullptr) v += bias[e];
                             dst[e] = v;
+                        }
+                    }
+                } else if (t < T) {
+                    float* dh = part_hi + ((int64_t)ks * T + t) * E;
+                    float* dl = part_lo + ((int64_t)ks * T + t) * E;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const int e = e0 + c * 32 + i;
+                        if (e < E) {
+                            dh[e] = h[i];
+                            dl[e] = l[i];
                         }
                     }
                 }
@@ -173,9 +193,19 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 }  // namespace
 
-cudaError_t launch_router_logits(const uint16_t* x, const uint16_t* hi, const uint16_t* lo,
-                                 const float* bias, float* logits, int T, int d, int E,
-                                 int32_t* status, cudaStream_t s) {
+int router_ksplit(int T, int d, int E) {
+    const int tiles = ((T + BM - 1) / BM) * ((E + BN - 1) / BN);
+    const int nk = d / BK;
+    int ks = 1;
+    // split K while the grid fills less than half the SMs, keeping >= 4 k-blocks per CTA
+    while (ks < 8 && tiles * ks * 2 <= 148 && nk / (ks * 2) >= 4) ks *= 2;
+    return ks;
+}
+
+static cudaError_t launch_router_impl(const uint16_t* x, const uint16_t* hi, const uint16_t* lo,
+                                      const float* bias, float* logits, float* part_hi,
+                                      float* part_lo, int ksplit, int T, int d, int E,
+                                      int32_t* status, cudaStream_t s) {
     if (T == 0) return cudaSuccess;
     CUtensorMap tx, th, tl;
     if (!make_tmap_2d(&tx, x, 2, (uint64_t)T, (uint64_t)d, BM, BK) ||
@@ -190,10 +220,23 @@ cudaError_t launch_router_logits(const uint16_t* x, const uint16_t* hi, const ui
         if (e != cudaSuccess) return e;
         attr_set[dev] = true;
     }
-    dim3 grid((T + BM - 1) / BM, (E + BN - 1) / BN);
-    k_router_dual<<<grid, THREADS, SMEM_BYTES, s>>>(tx, th, tl, bias, logits, T, d, E, status,
-                                                    kDefaultTimeoutNs);
+    dim3 grid((T + BM - 1) / BM, (E + BN - 1) / BN, ksplit);
+    k_router_dual<<<grid, THREADS, SMEM_BYTES, s>>>(tx, th, tl, bias, logits, part_hi, part_lo, T, d,
+                                                    E, status, kDefaultTimeoutNs);
     return cudaGetLastError();
+}
+
+cudaError_t launch_router_logits(const uint16_t* x, const uint16_t* hi, const uint16_t* lo,
+                                 const float* bias, float* logits, int T, int d, int E,
+                                 int32_t* status, cudaStream_t s) {
+    return launch_router_impl(x, hi, lo, bias, logits, nullptr, nullptr, 1, T, d, E, status, s);
+}
+
+cudaError_t launch_router_partials(const uint16_t* x, const uint16_t* hi, const uint16_t* lo,
+                                   float* part_hi, float* part_lo, int ksplit, int T, int d, int E,
+                                   int32_t* status, cudaStream_t s) {
+    return launch_router_impl(x, hi, lo, nullptr, nullptr, part_hi, part_lo, ksplit, T, d, E,
+                              status, s);
 }
 
 }  // namespace moe

@@ -56,20 +56,45 @@ cudaError_t launch_router_split(const float* W, uint16_t* hi, uint16_t* lo, int6
 // ---------------------------------------------------------------------------
 constexpr int kTopkWarps = 8;
 
+// Sum of the split-K router partials of one logit, in a fixed pairwise order.
+__device__ __forceinline__ float sum_partials(const float* p, int64_t stride, int n) {
+    if (n == 1) return p[0];
+    if (n == 2) return p[0] + p[stride];
+    if (n == 4) return (p[0] + p[stride]) + (p[2 * stride] + p[3 * stride]);
+    return ((p[0] + p[stride]) + (p[2 * stride] + p[3 * stride])) +
+           ((p[4 * stride] + p[5 * stride]) + (p[6 * stride] + p[7 * stride]));
+}
+
 __global__ void __launch_bounds__(kTopkWarps * 32)
-    k_route_topk(const float* __restrict__ logits, int T, int E, int k, int renorm,
+    k_route_topk(const float* __restrict__ logits_in, const float* __restrict__ part_hi,
+                 const float* __restrict__ part_lo, int ksplit, const float* __restrict__ bias,
+                 float* __restrict__ logits_out, int T, int E, int k, int renorm,
                  int32_t* __restrict__ ids, float* __restrict__ w) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int t = blockIdx.x * kTopkWarps + warp;
     if (t >= T) return;
-    const float* l = logits + (int64_t)t * E;
     float v[8];
     uint32_t taken = 0;
+    const int64_t pstride = (int64_t)T * E;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         const int e = lane + 32 * i;
-        v[i] = (e < E) ? l[e] : 0.0f;
-        if (e >= E) taken |= 1u << i;
+        if (e < E) {
+            if (part_hi != nullptr) {
+                // split-K router: hi sums + lo sums / 256 (one FMA) + bias
+                const int64_t off = (int64_t)t * E + e;
+                float x = fmaf(sum_partials(part_lo + off, pstride, ksplit), 0.00390625f,
+                               sum_partials(part_hi + off, pstride, ksplit));
+                if (bias != nullptr) x += bias[e];
+                logits_out[off] = x;
+                v[i] = x;
+            } else {
+                v[i] = logits_in[(int64_t)t * E + e];
+            }
+        } else {
+            v[i] = 0.0f;
+            taken |= 1u << i;
+        }
     }
     float my_v = 0.0f;
     int my_e = 0;
@@ -123,8 +148,17 @@ __global__ void __launch_bounds__(kTopkWarps * 32)
 cudaError_t launch_route_topk(const float* logits, int T, int E, int k, int renorm, int32_t* ids,
                               float* w, cudaStream_t s) {
     if (T == 0) return cudaSuccess;
-    k_route_topk<<<(T + kTopkWarps - 1) / kTopkWarps, kTopkWarps * 32, 0, s>>>(logits, T, E, k,
-                                                                              renorm, ids, w);
+    k_route_topk<<<(T + kTopkWarps - 1) / kTopkWarps, kTopkWarps * 32, 0, s>>>(
+        logits, nullptr, nullptr, 1, nullptr, nullptr, T, E, k, renorm, ids, w);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_route_topk_partials(const float* part_hi, const float* part_lo, int ksplit,
+                                       const float* bias, float* logits, int T, int E, int k,
+                                       int renorm, int32_t* ids, float* w, cudaStream_t s) {
+    if (T == 0) return cudaSuccess;
+    k_route_topk<<<(T + kTopkWarps - 1) / kTopkWarps, kTopkWarps * 32, 0, s>>>(
+        nullptr, part_hi, part_lo, ksplit, bias, logits, T, E, k, renorm, ids, w);
     return cudaGetLastError();
 }
 
