@@ -203,9 +203,10 @@ moe_status run_down(const moe_shape* s, const moe_weights* w, const void* h, con
                     const int32_t* offsets, float* o, int32_t* status, cudaStream_t st) {
     const GroupedGemmArgs a = gemm_args(s, offsets, nullptr, status);
     if (s->wdtype == MOE_WDTYPE_BF16)
-        return cuda_status(launch_down_bf16(a, static_cast<const uint16_t*>(h),
-                                            static_cast<const uint16_t*>(w->w_d),
-                                            static_cast<const uint16_t*>(w->ws_d), o, st));
+        return cuda_status((use_pair_tiles(s->T, s->E, s->k) ? launch_down_bf16_2sm
+                                                             : launch_down_bf16)(
+            a, static_cast<const uint16_t*>(h), static_cast<const uint16_t*>(w->w_d),
+            static_cast<const uint16_t*>(w->ws_d), o, st));
     return cuda_status(launch_down_fp8(a, static_cast<const uint8_t*>(h), hs,
                                        static_cast<const uint8_t*>(w->w_d), w->w_d_scale,
                                        static_cast<const uint8_t*>(w->ws_d), w->ws_d_scale, o, st));
