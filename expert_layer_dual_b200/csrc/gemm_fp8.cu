@@ -17,7 +17,8 @@
 //  - sixteen epilogue warps (four per TMEM lane quadrant, each owning a
 //    quarter of the columns, so four warps per scheduler hide the TMEM load
 //    latency) read the partial with tcgen05.ld and accumulate
-//    s_a[row] * s_w * P into 64 FP32 registers per thread;
+//    s_a[row] * s_w * P into 64 FP32 values per thread, held as 32 pairs for
+//    the paired FMA (fma.rn.f32x2), which halves the promotion's FMA count;
 //  - operands arrive by TMA into a 4-stage ring (128-byte swizzle).  The
 //    gate-up A rows are the activation quantisation's output, already
 //    written in permuted row order, so both operands are plain tiles.
@@ -183,20 +184,36 @@ __device__ __forceinline__ void mma_role(Smem& sm, const GroupedGemmArgs& a, uin
     }
 }
 
-// One promotion step of an epilogue thread: acc[0..31] += f0 * cols
-// c0..c0+31 and acc[32..63] += f1 * cols c1..c1+31 of its TMEM lane, 16
-// columns per load to keep the footprint at 64 accumulators plus one chunk.
+__device__ __forceinline__ uint64_t f32x2_pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f32x2_unpack(uint64_t r, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(r));
+}
+__device__ __forceinline__ uint64_t f32x2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
 __device__ __forceinline__ void promote(uint32_t lane_base, int c0, int c1, float f0, float f1,
-                                        float* acc) {
+                                        uint64_t* acc) {
+    const uint64_t ff0 = f32x2_pack(f0, f0), ff1 = f32x2_pack(f1, f1);
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
         float v[16];
         const int col = (q < 2 ? c0 : c1) + (q & 1) * 16;
-        const float f = q < 2 ? f0 : f1;
+        const uint64_t ff = q < 2 ? ff0 : ff1;
         tmem_load16(lane_base + col, v);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) acc[q * 16 + i] = fmaf(f, v[i], acc[q * 16 + i]);
+        for (int i = 0; i < 8; ++i)
+            acc[q * 8 + i] = f32x2_fma(ff, f32x2_pack(v[2 * i], v[2 * i + 1]), acc[q * 8 + i]);
     }
+}
+__device__ __forceinline__ void unpack_acc(const uint64_t* acc2, float* acc) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) f32x2_unpack(acc2[i], acc[2 * i], acc[2 * i + 1]);
 }
 
 // All lanes of the warp are done with their part (TMEM loads waited for,
@@ -264,9 +281,9 @@ __global__ void __launch_bounds__(THREADS, 1)
                                       : wsc + ((int64_t)t.g * nbs + a.I / 128 + t.n) * kbs;
             const bool valid = row < t.nrows;
             const float* sa_row = xs + (int64_t)(valid ? t.row0 + row : 0) * kbs;
-            float acc[64];
+            uint64_t acc2[32];
 #pragma unroll
-            for (int i = 0; i < 64; ++i) acc[i] = 0.0f;
+            for (int i = 0; i < 32; ++i) acc2[i] = 0ull;
             bool ok = true;
             // scales of the next k-block load while this one is promoted
             float sa_n = valid ? __ldg(sa_row) : 0.0f, sg_n = __ldg(swg), su_n = __ldg(swu);
@@ -285,12 +302,13 @@ __global__ void __launch_bounds__(THREADS, 1)
                 }
                 tc_fence_after_sync();
                 const uint32_t base = tmem + lane_off + pb * BN;
-                promote(base, qtr * 32, 128 + qtr * 32, fg, fu, acc);
+                promote(base, qtr * 32, 128 + qtr * 32, fg, fu, acc2);
                 tc_fence_before_sync();
                 warp_arrive(&b->pempty[pb]);
             }
             if (!ok) break;
-            // h = silu(g) * u on this thread's 32 columns, then the row's group amax
+            float acc[64];
+            unpack_acc(acc2, acc);
             float amax = 0.0f;
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
@@ -372,9 +390,9 @@ __global__ void __launch_bounds__(THREADS, 1)
                                      : wsc + ((int64_t)t.g * nbs + (live ? nb : 0)) * kbs;
             const bool valid = row < t.nrows;
             const float* sa_row = hs + (int64_t)(valid ? t.row0 + row : 0) * kbs;
-            float acc[64];
+            uint64_t acc2[32];
 #pragma unroll
-            for (int i = 0; i < 64; ++i) acc[i] = 0.0f;
+            for (int i = 0; i < 32; ++i) acc2[i] = 0ull;
             bool ok = true;
             const bool use = valid && live;
             float f_n = use ? __ldg(sa_row) * __ldg(sw) : 0.0f;
@@ -389,12 +407,14 @@ __global__ void __launch_bounds__(THREADS, 1)
                 }
                 tc_fence_after_sync();
                 const uint32_t base = tmem + lane_off + pb * BN;
-                promote(base, qtr * 64, qtr * 64 + 32, f, f, acc);
+                promote(base, qtr * 64, qtr * 64 + 32, f, f, acc2);
                 tc_fence_before_sync();
                 warp_arrive(&b->pempty[pb]);
             }
             if (!ok) break;
             if (valid && live) {
+                float acc[64];
+                unpack_acc(acc2, acc);
                 float* dst = o + (int64_t)(t.row0 + row) * a.d + t.n * BN + qtr * 64;
 #pragma unroll
                 for (int q = 0; q < 16; ++q)
