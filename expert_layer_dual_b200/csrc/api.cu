@@ -175,6 +175,7 @@ GroupedGemmArgs gemm_args(const moe_shape* s, const int32_t* offsets, const int3
     a.offsets = offsets;
     a.perm = perm;
     a.status = status;
+    a.tile_counter = status + kWsTileCounter;
     a.timeout_ns = kDefaultTimeoutNs;
     return a;
 }

@@ -19,8 +19,10 @@
 namespace moe {
 
 // Bytes reserved at the start of every workspace; the device status word is
-// its first int32.
+// its first int32, the grouped GEMMs' tile counter the int32 at index
+// kWsTileCounter.
 constexpr size_t kWsHeader = 256;
+constexpr int kWsTileCounter = 32;
 
 // Default bound of every device-side wait: far above any legitimate wait in
 // these kernels (the longest is one k-block of one tile), far below a hang.
@@ -202,6 +204,12 @@ __device__ __forceinline__ uint64_t l2_policy_evict_last() {
 // 16-byte global -> shared copy; src_bytes == 0 fills the 16 bytes with zeros.
 __device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+                 "r"(src_bytes)
+                 : "memory");
+}
+// 4-byte global -> shared copy; src_bytes == 0 writes a zero.
+__device__ __forceinline__ void cp_async_4(uint32_t dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src),
                  "r"(src_bytes)
                  : "memory");
 }

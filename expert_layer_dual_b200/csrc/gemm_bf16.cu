@@ -10,7 +10,8 @@
 // on cross-CTA scheduling; on sm_100a the MMA is issued by one thread and
 // runs asynchronously from its operand loads, so the kernel is warp
 // specialised instead):
-//  - persistent: one CTA per SM walks the device-side tile list;
+//  - persistent: one CTA per SM takes tiles from the dynamic schedule of
+//    grouped_common.cuh (m-tiles that share a weight tile start together);
 //  - tile 128 rows x 256 columns x 64-wide k-blocks, 4-stage shared-memory
 //    ring, 128-byte swizzled K-major operands;
 //  - gate-up: the 256 B columns are 128 gate rows and the matching 128 up
@@ -48,6 +49,7 @@ struct Bars {
     uint64_t empty[STAGES];   // MMA commit
     uint64_t tfull[2];        // accumulator ready (MMA commit)
     uint64_t tempty[2];       // accumulator drained (one arrival per epilogue warp)
+    TileRing ring;            // tile numbers from the producer to the other roles
     uint32_t tmem_slot;
     int abort_flag;
 };
@@ -81,8 +83,10 @@ __device__ __forceinline__ void fail(Bars* b, int32_t* status) {
 }
 
 // Shared prologue: barriers, tile table, TMEM.  full_a_count = 0 means the
-// A operand also arrives by TMA (full_a unused).
-__device__ __forceinline__ uint32_t prologue(Smem& sm, const GroupedGemmArgs& a, int full_a_count) {
+// A operand also arrives by TMA (full_a unused); `consumers` is the number of
+// arrivals that release a tile-ring slot.
+__device__ __forceinline__ uint32_t prologue(Smem& sm, const GroupedGemmArgs& a, int full_a_count,
+                                             uint32_t consumers) {
     const int warp = threadIdx.x >> 5;
     Bars* b = sm.bars;
     if (threadIdx.x == 0) {
@@ -95,6 +99,7 @@ __device__ __forceinline__ uint32_t prologue(Smem& sm, const GroupedGemmArgs& a,
             mbar_init(&b->tfull[i], 1);
             mbar_init(&b->tempty[i], EPI_WARPS);
         }
+        tile_ring_init(&b->ring, consumers);
         b->abort_flag = 0;
         fence_barrier_init();
     }
@@ -122,11 +127,14 @@ __device__ __forceinline__ void mma_role(Smem& sm, const GroupedGemmArgs& a, uin
     Bars* b = sm.bars;
     const volatile int* ab = &b->abort_flag;
     constexpr uint32_t idesc = idesc_bf16(BM, BN);
-    const int total = sm.tt->mstart[G] * n_tiles;
     const int nk = (wait_a ? a.d : a.I) / BK;
     uint32_t it = 0, lt = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x, ++lt) {
+    for (;; ++lt) {
+        if (tile_ring_pop(&b->ring, lt, a.timeout_ns, ab, ok) < 0) {
+            if (!ok) fail(b, a.status);
+            break;
+        }
         const uint32_t buf = lt & 1, tph = (lt >> 1) & 1;
         if (!mbar_wait(&b->tempty[buf], tph ^ 1, a.timeout_ns, ab)) { fail(b, a.status); break; }
         tc_fence_after_sync();
@@ -150,6 +158,7 @@ __device__ __forceinline__ void mma_role(Smem& sm, const GroupedGemmArgs& a, uin
             umma_commit(&b->empty[s]);
         }
         umma_commit(&b->tfull[buf]);  // also after an abort: arrives when issued MMAs finish
+        if (!ok) break;
     }
 }
 
@@ -164,7 +173,8 @@ __global__ void __launch_bounds__(GATEUP_THREADS, 1)
     Bars* b = sm.bars;
     const volatile int* ab = &b->abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const uint32_t tmem = prologue(sm, a, GATHER_WARPS);
+    // ring consumers: the MMA thread, 4 epilogue warps, 4 gather warps
+    const uint32_t tmem = prologue(sm, a, GATHER_WARPS, 1 + EPI_WARPS + GATHER_WARPS);
     const int G = a.E + a.has_shared;
     const int n_tiles = a.I / 128;
     const int total = sm.tt->mstart[G] * n_tiles;
@@ -186,7 +196,13 @@ __global__ void __launch_bounds__(GATEUP_THREADS, 1)
                 rg = rbase + t.n * 128;
                 ru = rbase + a.I + t.n * 128;
             };
-            for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+            for (uint32_t ti = 0; ok; ++ti) {
+                const int tile = tile_ring_push(&b->ring, ti, a.tile_counter, total, a.timeout_ns,
+                                                ab, ok);
+                if (tile < 0) {
+                    if (!ok) fail(b, a.status);
+                    break;
+                }
                 const Tile t = decode_tile(sm.tt, G, n_tiles, tile, BM);
                 const CUtensorMap* map;
                 int rg, ru;
@@ -225,7 +241,12 @@ __global__ void __launch_bounds__(GATEUP_THREADS, 1)
         uint32_t it = 0;
         int pend0 = -1, pend1 = -1;  // stages issued but not yet published, oldest first
         bool ok = true;
-        for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+        for (uint32_t ti = 0; ok; ++ti) {
+            const int tile = tile_ring_pop_warp(&b->ring, ti, a.timeout_ns, ab, ok);
+            if (tile < 0) {
+                if (!ok && lane == 0) fail(b, a.status);
+                break;
+            }
             const Tile t = decode_tile(sm.tt, G, n_tiles, tile, BM);
             const uint16_t* src[8];
             uint32_t valid = 0;
@@ -271,8 +292,13 @@ __global__ void __launch_bounds__(GATEUP_THREADS, 1)
     } else {
         // ---------------- epilogue warps 0-3: TMEM -> silu(g) * u -> bf16
         const int row = warp * 32 + lane;
-        uint32_t lt = 0;
-        for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++lt) {
+        bool ok = true;
+        for (uint32_t lt = 0;; ++lt) {
+            const int tile = tile_ring_pop_warp(&b->ring, lt, a.timeout_ns, ab, ok);
+            if (tile < 0) {
+                if (!ok && lane == 0) fail(b, a.status);
+                break;
+            }
             const Tile t = decode_tile(sm.tt, G, n_tiles, tile, BM);
             const uint32_t buf = lt & 1, tph = (lt >> 1) & 1;
             if (!warp_wait(&b->tfull[buf], tph, a.timeout_ns, ab)) { fail(b, a.status); break; }
@@ -315,7 +341,8 @@ __global__ void __launch_bounds__(DOWN_THREADS, 1)
     Bars* b = sm.bars;
     const volatile int* ab = &b->abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const uint32_t tmem = prologue(sm, a, 0);
+    // ring consumers: the MMA thread and 4 epilogue warps
+    const uint32_t tmem = prologue(sm, a, 0, 1 + EPI_WARPS);
     const int G = a.E + a.has_shared;
     const int n_tiles = (a.d + BN - 1) / BN;
     const int total = sm.tt->mstart[G] * n_tiles;
@@ -328,7 +355,13 @@ __global__ void __launch_bounds__(DOWN_THREADS, 1)
             tma_prefetch_desc(&tm_ws);
             uint32_t it = 0, issued = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+            for (uint32_t ti = 0; ok; ++ti) {
+                const int tile = tile_ring_push(&b->ring, ti, a.tile_counter, total, a.timeout_ns,
+                                                ab, ok);
+                if (tile < 0) {
+                    if (!ok) fail(b, a.status);
+                    break;
+                }
                 const Tile t = decode_tile(sm.tt, G, n_tiles, tile, BM);
                 const bool shared = t.g >= a.E;
                 const CUtensorMap* map = shared ? &tm_ws : &tm_w;
@@ -359,8 +392,13 @@ __global__ void __launch_bounds__(DOWN_THREADS, 1)
         if (lane == 0) mma_role(sm, a, tmem, G, n_tiles, false);
     } else {
         const int row = warp * 32 + lane;
-        uint32_t lt = 0;
-        for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++lt) {
+        bool ok = true;
+        for (uint32_t lt = 0;; ++lt) {
+            const int tile = tile_ring_pop_warp(&b->ring, lt, a.timeout_ns, ab, ok);
+            if (tile < 0) {
+                if (!ok && lane == 0) fail(b, a.status);
+                break;
+            }
             const Tile t = decode_tile(sm.tt, G, n_tiles, tile, BM);
             const uint32_t buf = lt & 1, tph = (lt >> 1) & 1;
             if (!warp_wait(&b->tfull[buf], tph, a.timeout_ns, ab)) { fail(b, a.status); break; }
@@ -411,6 +449,7 @@ cudaError_t launch_gateup_bf16(const GroupedGemmArgs& a, const uint16_t* x, cons
     static bool flags[64] = {false};
     cudaError_t e = set_smem_once(k_gateup_bf16, flags);
     if (e != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(a.tile_counter, 0, sizeof(int32_t), s)) != cudaSuccess) return e;
     k_gateup_bf16<<<current_device_info().num_sms, GATEUP_THREADS, SMEM_BYTES, s>>>(tw, tws, a, x, h);
     return cudaGetLastError();
 }
@@ -427,6 +466,7 @@ cudaError_t launch_down_bf16(const GroupedGemmArgs& a, const uint16_t* h, const 
     static bool flags[64] = {false};
     cudaError_t e = set_smem_once(k_down_bf16, flags);
     if (e != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(a.tile_counter, 0, sizeof(int32_t), s)) != cudaSuccess) return e;
     k_down_bf16<<<current_device_info().num_sms, DOWN_THREADS, SMEM_BYTES, s>>>(th, tw, tws, a, o);
     return cudaGetLastError();
 }

@@ -21,7 +21,17 @@
 //    the paired FMA (fma.rn.f32x2), which halves the promotion's FMA count;
 //  - operands arrive by TMA into a 4-stage ring (128-byte swizzle).  The
 //    gate-up A rows are the activation quantisation's output, already
-//    written in permuted row order, so both operands are plain tiles.
+//    written in permuted row order, so both operands are plain tiles;
+//  - tiles come from the dynamic schedule of grouped_common.cuh, so the
+//    m-tiles of one expert read its weight tile from DRAM once (with the
+//    static round-robin order the FP8 gate-up read 1.4x its weight bytes);
+//  - gate-up: a scale warp stages the tile's activation and weight scales in
+//    shared memory, 16 k-blocks per chunk, double-buffered and issued as
+//    cp.async copies, so the promotion never waits on a global load (a
+//    per-k-block register prefetch left the epilogue warps stalled on those
+//    loads a third of the time).  Down has one chunk per tile, where the
+//    staging latency would fall on every tile start, so its epilogue keeps
+//    the one-k-block-ahead register prefetch.
 // Gate-up's tile is 128 rows x (128 gate + 128 up) columns: each row's 128
 // h values form exactly one 1x128 quantisation group, so the epilogue
 // computes h = silu(g) * u, the group's amax (combining the four column
@@ -41,8 +51,13 @@ constexpr int B_HALF = 128 * BK;       // 16 KB
 constexpr int B_BYTES = 2 * B_HALF;    // 32 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr uint32_t TMEM_COLS = 512;    // two 256-column partial buffers
-constexpr int EPI_WARPS = 16, MMA_WARP = 16, TMA_WARP = 17;
-constexpr int THREADS = 32 * (TMA_WARP + 1);  // 576
+constexpr int EPI_WARPS = 16, MMA_WARP = 16, TMA_WARP = 17, SCALE_WARP = 18;
+constexpr int THREADS = 32 * (SCALE_WARP + 1);  // 608
+// Scales are staged in chunks of SC_KB k-blocks: activation scales [k][row]
+// with a padded row pitch (conflict-free reads by the 32 rows of a warp),
+// then the chunk's scales of weight block 0 and weight block 1.
+constexpr int SC_KB = 16, SA_PITCH = BM + 1;
+constexpr int SC_FLOATS = SC_KB * SA_PITCH + 2 * SC_KB;  // one chunk buffer
 
 struct Bars {
     uint64_t full[STAGES];   // TMA arrival + transaction bytes
@@ -50,15 +65,20 @@ struct Bars {
     uint64_t pfull[2];       // partial ready (MMA commit)
     uint64_t pempty[2];      // partial consumed (one arrival per epilogue warp)
     uint64_t amax_bar[2];    // gate-up: the four quarters' amax written (one per warp)
+    uint64_t sfull[2];       // scale chunk staged (scale warp)
+    uint64_t sempty[2];      // scale chunk read (one arrival per epilogue warp)
+    TileRing ring;           // tile numbers from the producer to the other roles
     uint32_t tmem_slot;
     int abort_flag;
     float amax[2][4][BM];    // [tile parity][column quarter][row]
 };
 
-constexpr size_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + sizeof(Bars) + sizeof(TileTable) + 64;
+constexpr size_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 2 * SC_FLOATS * sizeof(float) +
+                              sizeof(Bars) + sizeof(TileTable) + 64;
 
 struct Smem {
     uint8_t* stages;
+    float* scales;  // two chunk buffers of SC_FLOATS
     Bars* bars;
     TileTable* tt;
 };
@@ -67,7 +87,8 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
     Smem s;
     s.stages = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) &
                                           ~static_cast<uintptr_t>(1023));
-    s.bars = reinterpret_cast<Bars*>(s.stages + STAGES * STAGE_BYTES);
+    s.scales = reinterpret_cast<float*>(s.stages + STAGES * STAGE_BYTES);
+    s.bars = reinterpret_cast<Bars*>(s.scales + 2 * SC_FLOATS);
     s.tt = reinterpret_cast<TileTable*>(s.bars + 1);
     return s;
 }
@@ -77,7 +98,8 @@ __device__ __forceinline__ void fail(Bars* b, int32_t* status) {
     *reinterpret_cast<volatile int*>(&b->abort_flag) = 1;
 }
 
-__device__ __forceinline__ uint32_t prologue(Smem& sm, const GroupedGemmArgs& a) {
+__device__ __forceinline__ uint32_t prologue(Smem& sm, const GroupedGemmArgs& a,
+                                             uint32_t ring_consumers) {
     const int warp = threadIdx.x >> 5;
     Bars* b = sm.bars;
     if (threadIdx.x == 0) {
@@ -89,7 +111,10 @@ __device__ __forceinline__ uint32_t prologue(Smem& sm, const GroupedGemmArgs& a)
             mbar_init(&b->pfull[i], 1);
             mbar_init(&b->pempty[i], EPI_WARPS);
             mbar_init(&b->amax_bar[i], EPI_WARPS);
+            mbar_init(&b->sfull[i], 1);
+            mbar_init(&b->sempty[i], EPI_WARPS);
         }
+        tile_ring_init(&b->ring, ring_consumers);
         b->abort_flag = 0;
         fence_barrier_init();
     }
@@ -126,7 +151,12 @@ __device__ __forceinline__ void tma_role(Smem& sm, const GroupedGemmArgs& a, con
     const int total = sm.tt->mstart[G] * n_tiles;
     uint32_t it = 0, issued = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+    for (uint32_t ti = 0; ok; ++ti) {
+        const int tile = tile_ring_push(&b->ring, ti, a.tile_counter, total, a.timeout_ns, ab, ok);
+        if (tile < 0) {
+            if (!ok) fail(b, a.status);
+            break;
+        }
         const Tile t = decode_tile(sm.tt, G, n_tiles, tile, BM);
         const Loads L = rows_of(t);
         for (int kb = 0; kb < nk; ++kb, ++it) {
@@ -157,10 +187,13 @@ __device__ __forceinline__ void mma_role(Smem& sm, const GroupedGemmArgs& a, uin
     Bars* b = sm.bars;
     const volatile int* ab = &b->abort_flag;
     constexpr uint32_t idesc = idesc_e4m3(BM, BN);
-    const int total = sm.tt->mstart[G] * n_tiles;
     uint32_t it = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+    for (uint32_t ti = 0; ok; ++ti) {
+        if (tile_ring_pop(&b->ring, ti, a.timeout_ns, ab, ok) < 0) {
+            if (!ok) fail(b, a.status);
+            break;
+        }
         for (int kb = 0; kb < nk; ++kb, ++it) {
             const int s = it % STAGES;
             const uint32_t ph = (it / STAGES) & 1;
@@ -183,6 +216,89 @@ __device__ __forceinline__ void mma_role(Smem& sm, const GroupedGemmArgs& a, uin
         }
     }
 }
+
+// Scale warp: for every tile (from the ring), stages its scales chunk by
+// chunk into the two chunk buffers, SC_KB k-blocks at a time.  The
+// activation scales of rows row0 .. row0+127 are one contiguous run of
+// 128 * nk floats in global memory (consecutive rows); each chunk reads
+// 16-float row segments coalesced and writes them transposed.  Rows past the
+// tile's valid rows get 0.  `weight_rows(t, w0, w1)` gives the nk scales of
+// the tile's two weight blocks.
+template <typename WeightRows>
+__device__ __forceinline__ void scale_role(Smem& sm, const GroupedGemmArgs& a, int G, int n_tiles,
+                                           int nk, const float* __restrict__ act_scale,
+                                           WeightRows weight_rows) {
+    Bars* b = sm.bars;
+    const volatile int* ab = &b->abort_flag;
+    const int lane = threadIdx.x & 31;
+    uint32_t cc = 0;  // chunks staged so far
+    bool ok = true;
+    for (uint32_t lt = 0; ok; ++lt) {
+        const int tile = tile_ring_pop_warp(&b->ring, lt, a.timeout_ns, ab, ok);
+        if (tile < 0) break;
+        const Tile t = decode_tile(sm.tt, G, n_tiles, tile, BM);
+        const float* src = act_scale + (int64_t)t.row0 * nk;
+        const float* w0;
+        const float* w1;
+        weight_rows(t, w0, w1);
+        for (int k0 = 0; k0 < nk; k0 += SC_KB, ++cc) {
+            const int buf = cc & 1;
+            if (!warp_wait(&b->sempty[buf], ((cc >> 1) & 1) ^ 1, a.timeout_ns, ab)) {
+                ok = false;
+                break;
+            }
+            const int nkb = min(SC_KB, nk - k0);
+            const uint32_t dst = smem_u32(sm.scales + buf * SC_FLOATS);
+            // every copy of the chunk in flight at once (4-byte cp.async,
+            // zero-filled past the valid rows), then one wait
+            for (int idx = lane; idx < BM * SC_KB; idx += 32) {
+                const int row = idx / SC_KB, kk = idx % SC_KB;
+                if (kk < nkb) {
+                    const bool in = row < t.nrows;
+                    cp_async_4(dst + 4u * (kk * SA_PITCH + row),
+                               src + (in ? (int64_t)row * nk + k0 + kk : 0), in ? 4u : 0u);
+                }
+            }
+            if (lane < nkb) {
+                cp_async_4(dst + 4u * (SC_KB * SA_PITCH + lane), w0 + k0 + lane, 4u);
+                cp_async_4(dst + 4u * (SC_KB * SA_PITCH + SC_KB + lane), w1 + k0 + lane, 4u);
+            }
+            cp_async_commit();
+            cp_async_wait<0>();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&b->sfull[buf]);
+        }
+    }
+    if (!ok && lane == 0) fail(b, a.status);
+}
+
+// Epilogue side of the scale chunks: the scales of k-block kb (chunk cc
+// counted over all of the CTA's tiles).  Waits for the chunk at its first
+// k-block and releases it after its last.
+struct ScaleReader {
+    uint32_t cc = 0;
+    const float* buf = nullptr;
+    __device__ __forceinline__ bool fetch(Smem& sm, const GroupedGemmArgs& a, int kb, int nk,
+                                          int row, float& sa, float& s0, float& s1) {
+        Bars* b = sm.bars;
+        const int kk = kb % SC_KB;
+        if (kk == 0) {
+            if (!warp_wait(&b->sfull[cc & 1], (cc >> 1) & 1, a.timeout_ns, &b->abort_flag))
+                return false;
+            buf = sm.scales + (cc & 1) * SC_FLOATS;
+        }
+        sa = buf[kk * SA_PITCH + row];
+        s0 = buf[SC_KB * SA_PITCH + kk];
+        s1 = buf[SC_KB * SA_PITCH + SC_KB + kk];
+        if (kk == SC_KB - 1 || kb == nk - 1) {
+            // the chunk's last k-block: its scales are in registers now
+            __syncwarp();
+            if ((threadIdx.x & 31) == 0) mbar_arrive(&b->sempty[cc & 1]);
+            ++cc;
+        }
+        return true;
+    }
+};
 
 __device__ __forceinline__ uint64_t f32x2_pack(float lo, float hi) {
     uint64_t r;
@@ -245,7 +361,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     Bars* b = sm.bars;
     const volatile int* ab = &b->abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const uint32_t tmem = prologue(sm, a);
+    // ring consumers: the MMA thread, the epilogue warps, the scale warp
+    const uint32_t tmem = prologue(sm, a, 1 + EPI_WARPS + 1);
     const int G = a.E + a.has_shared;
     const int n_tiles = a.I / 128;
     const int nk = a.d / BK;
@@ -265,36 +382,42 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
     } else if (warp == MMA_WARP) {
         if (lane == 0) mma_role(sm, a, tmem, G, n_tiles, nk);
-    } else {
+    } else if (warp == SCALE_WARP) {
+        scale_role(sm, a, G, n_tiles, nk, xs, [&](const Tile& t, const float*& w0, const float*& w1) {
+            const bool shared = t.g >= a.E;
+            const float* base = shared ? wssc : wsc + (int64_t)t.g * nbs * kbs;
+            w0 = base + (int64_t)t.n * kbs;
+            w1 = base + (int64_t)(a.I / 128 + t.n) * kbs;
+        });
+    } else if (warp < EPI_WARPS) {
         // ---------------- 16 epilogue warps
         const int quad = warp & 3, qtr = warp >> 2;
         const int row = quad * 32 + lane;
         const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-        const int total = sm.tt->mstart[G] * n_tiles;
-        uint32_t it = 0, lt = 0;
-        for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++lt) {
+        uint32_t it = 0;
+        ScaleReader sr;
+        bool rok = true;
+        for (uint32_t lt = 0;; ++lt) {
+            const int tile = tile_ring_pop_warp(&b->ring, lt, a.timeout_ns, ab, rok);
+            if (tile < 0) {
+                if (!rok && lane == 0) fail(b, a.status);
+                break;
+            }
             const Tile t = decode_tile(sm.tt, G, n_tiles, tile, BM);
-            const bool shared = t.g >= a.E;
-            const float* swg = shared ? wssc + (int64_t)t.n * kbs
-                                      : wsc + ((int64_t)t.g * nbs + t.n) * kbs;
-            const float* swu = shared ? wssc + (int64_t)(a.I / 128 + t.n) * kbs
-                                      : wsc + ((int64_t)t.g * nbs + a.I / 128 + t.n) * kbs;
             const bool valid = row < t.nrows;
-            const float* sa_row = xs + (int64_t)(valid ? t.row0 + row : 0) * kbs;
             uint64_t acc2[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) acc2[i] = 0ull;
             bool ok = true;
-            // scales of the next k-block load while this one is promoted
-            float sa_n = valid ? __ldg(sa_row) : 0.0f, sg_n = __ldg(swg), su_n = __ldg(swu);
             for (int kb = 0; kb < nk; ++kb, ++it) {
                 const uint32_t pb = it & 1, pph = (it >> 1) & 1;
-                const float fg = sa_n * sg_n, fu = sa_n * su_n;
-                if (kb + 1 < nk) {
-                    sa_n = valid ? __ldg(sa_row + kb + 1) : 0.0f;
-                    sg_n = __ldg(swg + kb + 1);
-                    su_n = __ldg(swu + kb + 1);
+                float sa, sg, su;
+                if (!sr.fetch(sm, a, kb, nk, row, sa, sg, su)) {
+                    fail(b, a.status);
+                    ok = false;
+                    break;
                 }
+                const float fg = sa * sg, fu = sa * su;
                 if (!warp_wait(&b->pfull[pb], pph, a.timeout_ns, ab)) {
                     fail(b, a.status);
                     ok = false;
@@ -355,7 +478,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     Bars* b = sm.bars;
     const volatile int* ab = &b->abort_flag;
-    const uint32_t tmem = prologue(sm, a);
+    // ring consumers: the MMA thread and the epilogue warps (the scale warp idles:
+    // with one chunk per tile its staging latency would sit at every tile start)
+    const uint32_t tmem = prologue(sm, a, 1 + EPI_WARPS);
     const int G = a.E + a.has_shared;
     const int n_tiles = (a.d + BN - 1) / BN;
     const int nk = a.I / BK;
@@ -375,13 +500,18 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
     } else if (warp == MMA_WARP) {
         if (lane == 0) mma_role(sm, a, tmem, G, n_tiles, nk);
-    } else {
+    } else if (warp < EPI_WARPS) {
         const int quad = warp & 3, qtr = warp >> 2;
         const int row = quad * 32 + lane;
         const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-        const int total = sm.tt->mstart[G] * n_tiles;
         uint32_t it = 0;
-        for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+        bool rok = true;
+        for (uint32_t lt = 0;; ++lt) {
+            const int tile = tile_ring_pop_warp(&b->ring, lt, a.timeout_ns, ab, rok);
+            if (tile < 0) {
+                if (!rok && lane == 0) fail(b, a.status);
+                break;
+            }
             const Tile t = decode_tile(sm.tt, G, n_tiles, tile, BM);
             const bool shared = t.g >= a.E;
             const int nb = 2 * t.n + (qtr >> 1);             // this quarter's weight scale block
@@ -395,6 +525,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             for (int i = 0; i < 32; ++i) acc2[i] = 0ull;
             bool ok = true;
             const bool use = valid && live;
+            // the next k-block's scale product loads while this one is promoted
             float f_n = use ? __ldg(sa_row) * __ldg(sw) : 0.0f;
             for (int kb = 0; kb < nk; ++kb, ++it) {
                 const uint32_t pb = it & 1, pph = (it >> 1) & 1;
@@ -451,6 +582,7 @@ cudaError_t launch_gateup_fp8(const GroupedGemmArgs& a, const uint8_t* xq, const
     static bool flags[64] = {false};
     cudaError_t e = set_smem_once(k_gateup_fp8, flags);
     if (e != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(a.tile_counter, 0, sizeof(int32_t), s)) != cudaSuccess) return e;
     k_gateup_fp8<<<current_device_info().num_sms, THREADS, SMEM_BYTES, s>>>(
         ta, tw, tws, a, xs, w_gu_s, a.has_shared ? ws_gu_s : w_gu_s, hq, hs);
     return cudaGetLastError();
@@ -469,6 +601,7 @@ cudaError_t launch_down_fp8(const GroupedGemmArgs& a, const uint8_t* hq, const f
     static bool flags[64] = {false};
     cudaError_t e = set_smem_once(k_down_fp8, flags);
     if (e != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(a.tile_counter, 0, sizeof(int32_t), s)) != cudaSuccess) return e;
     k_down_fp8<<<current_device_info().num_sms, THREADS, SMEM_BYTES, s>>>(
         ta, tw, tws, a, hs, w_d_s, a.has_shared ? ws_d_s : w_d_s, o);
     return cudaGetLastError();

@@ -5,9 +5,17 @@
 // of the routing stage), the shared expert owns rows T*k .. T*k+T-1.  A group
 // of n rows has ceil(n / 128) m-tiles; every group has the same number of
 // n-tiles.  Tiles are numbered group by group, and inside a group n-tile by
-// n-tile with the m-tiles innermost, so CTAs that run at the same time share
-// weight tiles through L2.  The host never learns the counts: each CTA
-// rebuilds the m-tile prefix from `offsets` in its prologue.
+// n-tile with the m-tiles innermost, so tiles with neighbouring numbers share
+// weight tiles.  The host never learns the counts: each CTA rebuilds the
+// m-tile prefix from `offsets` in its prologue.
+//
+// Tiles are handed out dynamically: the producer of each CTA takes the next
+// number from a global counter when it is ready for a new tile and publishes
+// it to the CTA's other roles through a small ring in shared memory.  Tiles
+// that share a weight tile are therefore started at about the same time by
+// whichever CTAs are free, and the second reader of a weight tile finds it
+// in L2; a static round-robin order lets the CTAs drift apart over the waves
+// until those second reads miss L2 and go to DRAM again.
 #pragma once
 
 #include "common.cuh"
@@ -71,6 +79,67 @@ __device__ __forceinline__ Tile decode_tile(const TileTable* tt, int G, int n_ti
     t.row0 = tt->goff[lo] + m * BM;
     const int rows = tt->goff[lo + 1] - tt->goff[lo];
     t.nrows = min(BM, rows - m * BM);
+    return t;
+}
+
+// ---------------------------------------------------------------- tile ring
+constexpr int kTileRing = 8;
+
+struct TileRing {
+    uint64_t full[kTileRing];   // producer published the slot (one arrival)
+    uint64_t empty[kTileRing];  // every consumer read it
+    int32_t tile[kTileRing];    // tile number, or -1 past the end
+};
+
+__device__ __forceinline__ void tile_ring_init(TileRing* r, uint32_t consumers) {
+    for (int i = 0; i < kTileRing; ++i) {
+        mbar_init(&r->full[i], 1);
+        mbar_init(&r->empty[i], consumers);
+    }
+}
+
+// Producer thread: takes the next tile number (its i-th) from the global
+// counter and publishes it; returns it, or -1 past the last tile.  Sets
+// `ok` false when the wait for a free slot runs out.
+__device__ __forceinline__ int tile_ring_push(TileRing* r, uint32_t i, int32_t* counter, int total,
+                                              uint64_t timeout_ns, const volatile int* abort,
+                                              bool& ok) {
+    const int slot = i % kTileRing;
+    if (!mbar_wait(&r->empty[slot], ((i / kTileRing) & 1) ^ 1, timeout_ns, abort)) {
+        ok = false;
+        return -1;
+    }
+    int t = atomicAdd(counter, 1);
+    if (t >= total) t = -1;
+    *reinterpret_cast<volatile int32_t*>(&r->tile[slot]) = t;
+    mbar_arrive(&r->full[slot]);  // release: the number is visible to the waiters
+    return t;
+}
+
+// Consumer, one thread: the i-th tile number; the slot is released at once.
+__device__ __forceinline__ int tile_ring_pop(TileRing* r, uint32_t i, uint64_t timeout_ns,
+                                             const volatile int* abort, bool& ok) {
+    const int slot = i % kTileRing;
+    if (!mbar_wait(&r->full[slot], (i / kTileRing) & 1, timeout_ns, abort)) {
+        ok = false;
+        return -1;
+    }
+    const int t = *reinterpret_cast<volatile int32_t*>(&r->tile[slot]);
+    mbar_arrive(&r->empty[slot]);
+    return t;
+}
+
+// Consumer, a whole warp (one arrival for the warp): the i-th tile number.
+__device__ __forceinline__ int tile_ring_pop_warp(TileRing* r, uint32_t i, uint64_t timeout_ns,
+                                                  const volatile int* abort, bool& ok) {
+    const int slot = i % kTileRing;
+    if (!warp_wait(&r->full[slot], (i / kTileRing) & 1, timeout_ns, abort)) {
+        ok = false;
+        return -1;
+    }
+    const int t = *reinterpret_cast<volatile int32_t*>(&r->tile[slot]);
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(&r->empty[slot]);
     return t;
 }
 

@@ -64,6 +64,7 @@ struct GroupedGemmArgs {
     const int32_t* offsets;  // [E+1]
     const int32_t* perm;     // [T*k]
     int32_t* status;
+    int32_t* tile_counter;   // next tile number of the dynamic schedule (zeroed by the launcher)
     uint64_t timeout_ns;
 };
 cudaError_t launch_gateup_bf16(const GroupedGemmArgs& a, const uint16_t* x, const uint16_t* w_gu,
