@@ -74,6 +74,12 @@ def lib():
         L.orc_permute.argtypes = [vp, i32, i32, i32, vp, vp, vp, vp]
         L.orc_quant_fp8_blocks.argtypes = [vp, i64, i32, i32, vp, vp]
         L.orc_quant_fp8_rows.argtypes = [vp, i64, i32, vp, vp]
+        L.orc_e8m0_decode.restype = ctypes.c_double
+        L.orc_e8m0_decode.argtypes = [ctypes.c_uint8]
+        L.orc_mx_scale_byte.restype = ctypes.c_uint8
+        L.orc_mx_scale_byte.argtypes = [ctypes.c_float]
+        L.orc_quant_mx_rows.argtypes = [vp, i64, i32, vp, vp]
+        L.orc_quant_mx_bf16.argtypes = [vp, i64, i32, i32, vp, vp]
         L.orc_gateup.argtypes = [ctypes.POINTER(_Layer), vp, vp, vp, vp]
         L.orc_down.argtypes = [ctypes.POINTER(_Layer), vp, vp, vp]
         L.orc_combine.argtypes = [ctypes.POINTER(_Layer), vp, vp, vp, vp]
@@ -182,6 +188,35 @@ def quant_fp8_rows(v: np.ndarray):
     return q, s
 
 
+def e8m0_decode(b: int) -> float:
+    return lib().orc_e8m0_decode(int(b))
+
+
+def mx_scale_byte(amax: float) -> int:
+    return int(lib().orc_mx_scale_byte(float(amax)))
+
+
+def quant_mx_rows(v: np.ndarray):
+    """v: float32 [rows, cols] -> (q uint8 [rows, cols], s uint8 E8M0 [rows, cols/32])."""
+    v = _c(v, np.float32)
+    rows, cols = v.shape
+    q = np.empty(v.shape, np.uint8)
+    s = np.empty((rows, cols // 32), np.uint8)
+    lib().orc_quant_mx_rows(_p(v), rows, cols, _p(q), _p(s))
+    return q, s
+
+
+def quant_mx_bf16(W: np.ndarray):
+    """W: bf16 bits [..., rows, cols] -> (q uint8, s uint8 E8M0 [..., rows, cols/32])."""
+    W = _c(W, np.uint16)
+    rows, cols = W.shape[-2:]
+    batch = int(np.prod(W.shape[:-2])) if W.ndim > 2 else 1
+    q = np.empty(W.shape, np.uint8)
+    s = np.empty(W.shape[:-1] + (cols // 32,), np.uint8)
+    lib().orc_quant_mx_bf16(_p(W), batch, rows, cols, _p(q), _p(s))
+    return q, s
+
+
 @dataclass
 class Layer:
     """Host copy of one MoE layer's weights, as the oracle consumes them."""
@@ -197,7 +232,7 @@ class Layer:
     ws_gu: Optional[np.ndarray] = None   # bf16 bits [2Is, d]
     ws_d: Optional[np.ndarray] = None    # bf16 bits [d, Is]
     router_bias: Optional[np.ndarray] = None
-    wdtype: int = 0             # 0 bf16, 1 fp8 e4m3 with 128x128 block scales
+    wdtype: int = 0             # 0 bf16, 1 fp8 e4m3 with 128x128 block scales, 2 mxfp8
     renorm: bool = True
 
     def _struct(self, T: Optional[int] = None):

@@ -117,6 +117,60 @@ static float quant_group(const float* v, int n, int64_t stride, uint8_t* q, int6
 }
 
 /* ---------------------------------------------------------------------------
+ * [MX] MXFP8: E8M0 shared scale per block of 32, e4m3 elements
+ * ------------------------------------------------------------------------- */
+
+double orc_e8m0_decode(uint8_t b) {
+    if (b == 255) return NAN;
+    return ldexp(1.0, (int)b - 127);
+}
+
+/* shared_exp = floor(log2(amax)) - 8, clamped to [-127, 127] (amax == 0 ->
+ * -127); the byte is shared_exp + 127. */
+uint8_t orc_mx_scale_byte(float amax) {
+    if (!(amax > 0.0f)) return 0;
+    int e;
+    frexp((double)amax, &e);            /* amax in [2^(e-1), 2^e)           */
+    int se = (e - 1) - 8;
+    if (se < -127) se = -127;
+    if (se > 127) se = 127;
+    return (uint8_t)(se + 127);
+}
+
+static void quant_mx_block(const float* v, int n, uint8_t* q, uint8_t* sb) {
+    float amax = 0.0f;
+    for (int i = 0; i < n; ++i) {
+        float a = fabsf(v[i]);
+        if (a > amax) amax = a;
+    }
+    uint8_t b = orc_mx_scale_byte(amax);
+    double X = orc_e8m0_decode(b);
+    for (int i = 0; i < n; ++i) q[i] = orc_e4m3_round((double)v[i] / X);
+    *sb = b;
+}
+
+void orc_quant_mx_rows(const float* v, int64_t rows, int cols, uint8_t* q, uint8_t* s) {
+    int g = cols / 32;
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r)
+        for (int j = 0; j < g; ++j)
+            quant_mx_block(v + r * cols + j * 32, 32, q + r * cols + j * 32, s + r * g + j);
+}
+
+void orc_quant_mx_bf16(const uint16_t* W, int64_t batch, int rows, int cols, uint8_t* q,
+                       uint8_t* s) {
+    int64_t n = batch * rows;
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < n; ++r) {
+        float f[32];
+        for (int j = 0; j < cols / 32; ++j) {
+            for (int i = 0; i < 32; ++i) f[i] = (float)orc_bf16_decode(W[r * cols + j * 32 + i]);
+            quant_mx_block(f, 32, q + r * cols + j * 32, s + r * (cols / 32) + j);
+        }
+    }
+}
+
+/* ---------------------------------------------------------------------------
  * [RG] router split and logits
  * ------------------------------------------------------------------------- */
 
@@ -249,6 +303,15 @@ static double* group_weights(const orc_layer* L, const uint16_t* W, int rows, in
         for (int64_t i = 0; i < n; ++i) out[i] = orc_bf16_decode(W[i]);
         return out;
     }
+    if (L->wdtype == 2) {
+        uint8_t* q = (uint8_t*)malloc((size_t)n);
+        uint8_t* sb = (uint8_t*)malloc((size_t)(n / 32 + 1));
+        orc_quant_mx_bf16(W, 1, rows, cols, q, sb);
+        for (int64_t i = 0; i < n; ++i) out[i] = orc_e4m3_decode(q[i]) * orc_e8m0_decode(sb[i / 32]);
+        free(q);
+        free(sb);
+        return out;
+    }
     int rb = rows / 128, cb = cols / 128;
     uint8_t* q = (uint8_t*)malloc((size_t)n);
     float* s = (float*)malloc(sizeof(float) * (size_t)rb * cb);
@@ -271,8 +334,17 @@ static void activation_row(const orc_layer* L, const double* v, int n, double* o
     }
     float* f = (float*)malloc(sizeof(float) * (size_t)n);
     uint8_t* q = (uint8_t*)malloc((size_t)n);
-    float* s = (float*)malloc(sizeof(float) * (size_t)(n / 128));
     for (int i = 0; i < n; ++i) f[i] = (float)v[i];
+    if (L->wdtype == 2) {
+        uint8_t* sb = (uint8_t*)malloc((size_t)(n / 32 + 1));
+        orc_quant_mx_rows(f, 1, n, q, sb);
+        for (int i = 0; i < n; ++i) out[i] = orc_e4m3_decode(q[i]) * orc_e8m0_decode(sb[i / 32]);
+        free(f);
+        free(q);
+        free(sb);
+        return;
+    }
+    float* s = (float*)malloc(sizeof(float) * (size_t)(n / 128));
     orc_quant_fp8_rows(f, 1, n, q, s);
     for (int i = 0; i < n; ++i) out[i] = orc_e4m3_decode(q[i]) * (double)s[i / 128];
     free(f);

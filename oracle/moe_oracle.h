@@ -83,9 +83,28 @@ void orc_quant_fp8_blocks(const uint16_t* W, int64_t batch, int rows, int cols,
  * q [rows][cols], s [rows][cols/128]. */
 void orc_quant_fp8_rows(const float* v, int64_t rows, int cols, uint8_t* q, float* s);
 
+/* [MX] MXFP8 (OCP Microscaling formats v1.0, "MXFP8 E4M3"): blocks of 32
+ * consecutive elements along K share one E8M0 scale X = 2^(b - 127) (byte b;
+ * 255 is NaN).  For a block with amax = max |v| (taken in FP32):
+ * shared_exp = floor(log2(amax)) - 8 (8 = exponent of the largest e4m3
+ * normal, 448 = 1.75 * 2^8), clamped to [-127, 127]; amax == 0 -> -127.
+ * q_i = e4m3_rne_satfinite(v_i / X) (exact power-of-two scaling, so FP32 and
+ * FP64 take the same decision).  The pages name the format ("PR #54160 完整报告",
+ * section 实现拆解 item 4: FP8 blockwise 128x128 and MXFP8 scale parameters);
+ * its definition is the OCP one. */
+double  orc_e8m0_decode(uint8_t b);
+uint8_t orc_mx_scale_byte(float amax);
+/* Rows of an FP32 matrix: q [rows][cols], s [rows][cols/32] (E8M0 bytes). */
+void orc_quant_mx_rows(const float* v, int64_t rows, int cols, uint8_t* q, uint8_t* s);
+/* Rows of `batch` bf16 matrices [rows][cols] (weights; K = cols):
+ * q [batch][rows][cols], s [batch][rows][cols/32]. */
+void orc_quant_mx_bf16(const uint16_t* W, int64_t batch, int rows, int cols, uint8_t* q,
+                       uint8_t* s);
+
 typedef struct {
     int T, d, E, k, I, Is;     /* Is = 0: no shared expert                     */
-    int wdtype;                /* 0: BF16 weights; 1: FP8 e4m3, 128x128 blocks
+    int wdtype;                /* 0: BF16 weights; 1: FP8 e4m3, 128x128 blocks;
+                                  2: MXFP8 (e4m3, E8M0 scale per 1x32 along K)
                                   (the oracle quantises the BF16 weights itself) */
     int renorm;
     const uint16_t* w_gu;      /* bf16 [E][2I][d]: gate rows 0..I-1, up I..2I-1 */
@@ -100,12 +119,14 @@ typedef struct {
  * expert whose offsets interval holds p and read token perm[p] / k; rows
  * T*k .. T*k+T-1 are the shared expert and read token p - T*k.
  * h: [T*k + (Is ? T : 0)][max(I, Is)] FP64, row stride hs = max(I, Is).
- * FP8 (wdtype 1): each input row is quantised per 1x128 group first.       */
+ * FP8 (wdtype 1): each input row is quantised per 1x128 group first;
+ * MXFP8 (wdtype 2): per 1x32 block (MX).                                     */
 void orc_gateup(const orc_layer* L, const uint16_t* x, const int32_t* perm,
                 const int32_t* offsets, double* h);
 
 /* [FM] Down stage: o[p] = h[p] Wd[e]^T, same row grouping as orc_gateup.
- * FP8: each h row is quantised per 1x128 group (FP32 decision) first.       */
+ * FP8: each h row is quantised per 1x128 group (FP32 decision) first;
+ * MXFP8: per 1x32 block of the FP32-rounded h row.                           */
 void orc_down(const orc_layer* L, const double* h, const int32_t* offsets, double* o);
 
 /* [FM] Top-K weighted aggregation: y[t] = sum_j w[t][j] o[inv[t*k+j]] + o[T*k+t]. */
