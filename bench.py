@@ -1,6 +1,6 @@
 """Benchmark of the fused MoE layer forward (one JSON line on rank 0).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config decode|prefill|fp8|skew|tiny]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config decode|prefill|fp8|mxfp8|skew|tiny]
                     [--impl ours|reference] [--no-cpu-baseline]
 
 A step is one moe_forward over one batch of the workload's T tokens (router
@@ -45,7 +45,7 @@ from expert_layer_dual_b200.inputs import make_layer  # noqa: E402
 METRIC = "fused MoE layer tokens/s"
 UNIT = "tokens/s"
 # oracle token sample per step of the CPU baseline / reference arm
-CPU_SAMPLE = {"tiny": 16, "decode": 64, "prefill": 16, "fp8": 8, "skew": 16}
+CPU_SAMPLE = {"tiny": 16, "decode": 64, "prefill": 16, "fp8": 8, "mxfp8": 8, "skew": 16}
 
 
 def cpu_sample(cfg: MoEConfig) -> int:
@@ -55,7 +55,8 @@ def cpu_sample(cfg: MoEConfig) -> int:
 def describe(cfg: MoEConfig) -> str:
     s = f"{cfg.name}: T={cfg.T} d={cfg.d} E={cfg.E} top-{cfg.k}"
     s += f" + shared I={cfg.I}" if cfg.Is else f" I={cfg.I}"
-    s += ", FP8 e4m3 128x128 block-scaled weights" if cfg.wdtype else ", BF16 weights"
+    s += {0: ", BF16 weights", 1: ", FP8 e4m3 128x128 block-scaled weights",
+          2: ", MXFP8 (e4m3, E8M0 scale per 1x32) weights and activations"}[cfg.wdtype]
     if cfg.zipf_bias:
         s += ", Zipf(1.2)-biased routing"
     return s
@@ -167,6 +168,7 @@ def load_peaks():
 KERNEL_SOURCES = {
     "k_gateup_bf16": ["csrc/gemm_bf16.cu", "csrc/common.cuh", "csrc/grouped_common.cuh"],
     "k_gateup_fp8": ["csrc/gemm_fp8.cu", "csrc/common.cuh", "csrc/grouped_common.cuh"],
+    "k_gateup_mx": ["csrc/gemm_mx.cu", "csrc/common.cuh", "csrc/grouped_common.cuh"],
 }
 
 
@@ -203,6 +205,8 @@ def gateup_algorithmic(cfg: MoEConfig, T: int, n_active: int):
     groups = n_active + (1 if cfg.Is else 0)
     flops = 2.0 * R * cfg.d * 2 * cfg.I
     byts = groups * 2 * cfg.I * cfg.d * wbytes + T * cfg.d * wbytes + R * cfg.I * wbytes
+    if cfg.wdtype == 2:  # MXFP8: one scale byte per 32 elements of weights, x and h
+        byts += (groups * 2 * cfg.I * cfg.d + T * cfg.d + R * cfg.I) // 32
     return flops, byts
 
 
@@ -212,6 +216,8 @@ def down_algorithmic(cfg: MoEConfig, T: int, n_active: int):
     groups = n_active + (1 if cfg.Is else 0)
     flops = 2.0 * R * cfg.I * cfg.d
     byts = groups * cfg.d * cfg.I * wbytes + R * cfg.I * wbytes + R * cfg.d * 2
+    if cfg.wdtype == 2:
+        byts += (groups * cfg.d * cfg.I + R * cfg.I) // 32
     return flops, byts
 
 
@@ -363,7 +369,7 @@ def run_ours(args, cfg: MoEConfig):
         roof = {"bound": "tensor", "achieved": gu_flops / (gu_ms / 1e3) / 1e12, "peak": peak,
                 "unit": "TFLOP/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["kernel"] = "k_gateup_" + ("fp8" if cfg.wdtype else "bf16")
+    roof["kernel"] = "k_gateup_" + {0: "bf16", 1: "fp8", 2: "mx"}[cfg.wdtype]
     roof["peak_source"] = (f"{peak_kind} MEASURED_PEAKS.json "
                            + ("hbm_gbs" if roof["bound"] == "hbm" else "bf16_tflops (burst: the timed loop is well under a second)"
                               + (" x2 (e4m3 nominal ratio)" if cfg.wdtype else "")))
@@ -411,7 +417,7 @@ def run_ours(args, cfg: MoEConfig):
         out = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f8e4m3" if cfg.wdtype else "bf16",
+            "scaling": "weak", "vs_baseline": None, "dtype": {0: "bf16", 1: "f8e4m3", 2: "mxf8e4m3"}[cfg.wdtype],
             "data": "synthetic",
             "config": {"workload": describe(cfg), "tokens_per_gpu": cfg.T,
                        "active_experts": n_active,

@@ -104,6 +104,11 @@ WsLayout ws_layout(const moe_shape& s) {
         L.xs = take(R * (d / 128) * 4);
         L.h = take(R * I);
         L.hs = take(R * (I / 128) * 4);
+    } else if (s.wdtype == MOE_WDTYPE_MXFP8) {
+        L.xq = take(R * d);                               // e4m3 x, permuted rows
+        L.xs = take(R * (d / 32));                        // E8M0 byte per 1x32 block
+        L.h = take(R * I);
+        L.hs = take(R * (I / 32));
     } else {
         L.xq = L.xs = L.hs = 0;
         L.h = take(R * I * 2);
@@ -127,7 +132,8 @@ moe_status check_shape(const moe_shape* s) {
     if (s->d % 128 != 0 || s->I % 128 != 0 || s->E > 256 || s->k > 8 || s->k > s->E)
         return MOE_ERR_UNSUPPORTED;
     if (s->I_shared != 0 && s->I_shared != s->I) return MOE_ERR_UNSUPPORTED;
-    if (s->wdtype != MOE_WDTYPE_BF16 && s->wdtype != MOE_WDTYPE_FP8_BLOCK128)
+    if (s->wdtype != MOE_WDTYPE_BF16 && s->wdtype != MOE_WDTYPE_FP8_BLOCK128 &&
+        s->wdtype != MOE_WDTYPE_MXFP8)
         return MOE_ERR_UNSUPPORTED;
     if ((int64_t)s->T * s->k + s->T >= (int64_t)1 << 31) return MOE_ERR_UNSUPPORTED;
     if ((int64_t)s->E * 2 * s->I >= (int64_t)1 << 31 || (int64_t)s->E * s->d >= (int64_t)1 << 31)
@@ -138,7 +144,7 @@ moe_status check_shape(const moe_shape* s) {
 moe_status check_weights(const moe_shape* s, const moe_weights* w, bool need_gateup,
                          bool need_down, bool need_router) {
     if (w == nullptr) return MOE_ERR_INVALID_ARG;
-    const bool fp8 = s->wdtype == MOE_WDTYPE_FP8_BLOCK128;
+    const bool fp8 = s->wdtype != MOE_WDTYPE_BF16;  // scaled weights (FP8 or MXFP8)
     const bool sh = s->I_shared > 0;
     if (need_gateup && (w->w_gu == nullptr || (fp8 && w->w_gu_scale == nullptr) ||
                         (sh && (w->ws_gu == nullptr || (fp8 && w->ws_gu_scale == nullptr)))))
@@ -185,8 +191,8 @@ inline P* at(void* ws, size_t off) {
     return reinterpret_cast<P*>(static_cast<uint8_t*>(ws) + off);
 }
 
-moe_status run_gateup(const moe_shape* s, const moe_weights* w, const void* x, const float* xs,
-                      const int32_t* perm, const int32_t* offsets, void* h, float* hs,
+moe_status run_gateup(const moe_shape* s, const moe_weights* w, const void* x, const void* xs,
+                      const int32_t* perm, const int32_t* offsets, void* h, void* hs,
                       int32_t* status, cudaStream_t st) {
     const GroupedGemmArgs a = gemm_args(s, offsets, perm, status);
     if (s->wdtype == MOE_WDTYPE_BF16)
@@ -194,13 +200,20 @@ moe_status run_gateup(const moe_shape* s, const moe_weights* w, const void* x, c
                                               static_cast<const uint16_t*>(w->w_gu),
                                               static_cast<const uint16_t*>(w->ws_gu),
                                               static_cast<uint16_t*>(h), st));
-    return cuda_status(launch_gateup_fp8(a, static_cast<const uint8_t*>(x), xs,
-                                         static_cast<const uint8_t*>(w->w_gu), w->w_gu_scale,
-                                         static_cast<const uint8_t*>(w->ws_gu), w->ws_gu_scale,
-                                         static_cast<uint8_t*>(h), hs, st));
+    if (s->wdtype == MOE_WDTYPE_MXFP8)
+        return cuda_status(launch_gateup_mx(
+            a, static_cast<const uint8_t*>(x), static_cast<const uint8_t*>(xs),
+            static_cast<const uint8_t*>(w->w_gu), static_cast<const uint8_t*>(w->w_gu_scale),
+            static_cast<const uint8_t*>(w->ws_gu), static_cast<const uint8_t*>(w->ws_gu_scale),
+            static_cast<uint8_t*>(h), static_cast<uint8_t*>(hs), st));
+    return cuda_status(launch_gateup_fp8(
+        a, static_cast<const uint8_t*>(x), static_cast<const float*>(xs),
+        static_cast<const uint8_t*>(w->w_gu), static_cast<const float*>(w->w_gu_scale),
+        static_cast<const uint8_t*>(w->ws_gu), static_cast<const float*>(w->ws_gu_scale),
+        static_cast<uint8_t*>(h), static_cast<float*>(hs), st));
 }
 
-moe_status run_down(const moe_shape* s, const moe_weights* w, const void* h, const float* hs,
+moe_status run_down(const moe_shape* s, const moe_weights* w, const void* h, const void* hs,
                     const int32_t* offsets, float* o, int32_t* status, cudaStream_t st) {
     const GroupedGemmArgs a = gemm_args(s, offsets, nullptr, status);
     if (s->wdtype == MOE_WDTYPE_BF16)
@@ -208,9 +221,15 @@ moe_status run_down(const moe_shape* s, const moe_weights* w, const void* h, con
                                                              : launch_down_bf16)(
             a, static_cast<const uint16_t*>(h), static_cast<const uint16_t*>(w->w_d),
             static_cast<const uint16_t*>(w->ws_d), o, st));
-    return cuda_status(launch_down_fp8(a, static_cast<const uint8_t*>(h), hs,
-                                       static_cast<const uint8_t*>(w->w_d), w->w_d_scale,
-                                       static_cast<const uint8_t*>(w->ws_d), w->ws_d_scale, o, st));
+    if (s->wdtype == MOE_WDTYPE_MXFP8)
+        return cuda_status(launch_down_mx(
+            a, static_cast<const uint8_t*>(h), static_cast<const uint8_t*>(hs),
+            static_cast<const uint8_t*>(w->w_d), static_cast<const uint8_t*>(w->w_d_scale),
+            static_cast<const uint8_t*>(w->ws_d), static_cast<const uint8_t*>(w->ws_d_scale), o, st));
+    return cuda_status(launch_down_fp8(
+        a, static_cast<const uint8_t*>(h), static_cast<const float*>(hs),
+        static_cast<const uint8_t*>(w->w_d), static_cast<const float*>(w->w_d_scale),
+        static_cast<const uint8_t*>(w->ws_d), static_cast<const float*>(w->ws_d_scale), o, st));
 }
 
 // Records events[i] (when given) at the stage boundaries: 0 start, 1 router
@@ -233,6 +252,7 @@ moe_status forward_device(const moe_shape* s, const moe_weights* w, const uint16
     int32_t* inv = at<int32_t>(ws, L.inv);
     int32_t* seg = at<int32_t>(ws, L.seg);
     const bool fp8 = s->wdtype == MOE_WDTYPE_FP8_BLOCK128;
+    const bool mx = s->wdtype == MOE_WDTYPE_MXFP8;
     moe_status r;
     if (cudaMemsetAsync(status, 0, sizeof(int32_t), st) != cudaSuccess) return MOE_ERR_CUDA;
     if (!mark(0)) return MOE_ERR_CUDA;
@@ -263,7 +283,15 @@ moe_status forward_device(const moe_shape* s, const moe_weights* w, const uint16
         return r;
     if (!mark(3)) return MOE_ERR_CUDA;
     const void* a_in = x;
-    const float* a_scale = nullptr;
+    const void* a_scale = nullptr;
+    if (mx) {
+        if ((r = cuda_status(launch_quant_mx_permuted(x, perm, s->T, s->k, s->I_shared > 0 ? 1 : 0,
+                                                      s->d, at<uint8_t>(ws, L.xq),
+                                                      at<uint8_t>(ws, L.xs), st))) != MOE_OK)
+            return r;
+        a_in = at<uint8_t>(ws, L.xq);
+        a_scale = at<uint8_t>(ws, L.xs);
+    }
     if (fp8) {
         if ((r = cuda_status(launch_quant_act_fp8_permuted(x, perm, s->T, s->k, s->I_shared > 0 ? 1 : 0,
                                                            s->d, at<uint8_t>(ws, L.xq),
@@ -274,7 +302,7 @@ moe_status forward_device(const moe_shape* s, const moe_weights* w, const uint16
     }
     if (!mark(4)) return MOE_ERR_CUDA;
     void* h = at<uint8_t>(ws, L.h);
-    float* hs = fp8 ? at<float>(ws, L.hs) : nullptr;
+    void* hs = (fp8 || mx) ? at<uint8_t>(ws, L.hs) : nullptr;
     float* o = at<float>(ws, L.o);
     if ((r = run_gateup(s, w, a_in, a_scale, perm, offsets, h, hs, status, st)) != MOE_OK) return r;
     if (!mark(5)) return MOE_ERR_CUDA;
@@ -341,6 +369,38 @@ moe_status moe_quantize_act_fp8(const uint16_t* x, int64_t rows, int32_t cols, u
     return cuda_status(launch_quant_act_fp8(x, rows, cols, q, scale, as_stream(stream)));
 }
 
+moe_status moe_quantize_weights_mxfp8(const uint16_t* W, int64_t batch, int32_t rows, int32_t cols,
+                                      uint8_t* q, uint8_t* scale, void* stream) {
+    if (batch < 0 || rows < 0 || cols < 0) return MOE_ERR_INVALID_ARG;
+    if (cols % 128 != 0) return MOE_ERR_UNSUPPORTED;
+    if (batch * rows * (int64_t)cols == 0) return MOE_OK;
+    if (W == nullptr || q == nullptr || scale == nullptr) return MOE_ERR_INVALID_ARG;
+    if (!device_ok()) return MOE_ERR_UNSUPPORTED;
+    return cuda_status(launch_quant_mx_rows(W, batch * rows, cols, q, scale, as_stream(stream)));
+}
+
+moe_status moe_quantize_act_mxfp8(const uint16_t* x, int64_t rows, int32_t cols, uint8_t* q,
+                                  uint8_t* scale, void* stream) {
+    if (rows < 0 || cols <= 0) return MOE_ERR_INVALID_ARG;
+    if (cols % 128 != 0) return MOE_ERR_UNSUPPORTED;
+    if (rows == 0) return MOE_OK;
+    if (x == nullptr || q == nullptr || scale == nullptr) return MOE_ERR_INVALID_ARG;
+    if (!device_ok()) return MOE_ERR_UNSUPPORTED;
+    return cuda_status(launch_quant_mx_rows(x, rows, cols, q, scale, as_stream(stream)));
+}
+
+moe_status moe_quantize_act_mxfp8_permuted(const uint16_t* x, const int32_t* perm, int32_t T,
+                                           int32_t k, int32_t with_shared, int32_t d, uint8_t* q,
+                                           uint8_t* scale, void* stream) {
+    if (T < 0 || k <= 0 || d <= 0) return MOE_ERR_INVALID_ARG;
+    if (d % 128 != 0 || (int64_t)T * k + T >= ((int64_t)1 << 31)) return MOE_ERR_UNSUPPORTED;
+    if (T == 0) return MOE_OK;
+    if (x == nullptr || perm == nullptr || q == nullptr || scale == nullptr) return MOE_ERR_INVALID_ARG;
+    if (!device_ok()) return MOE_ERR_UNSUPPORTED;
+    return cuda_status(launch_quant_mx_permuted(x, perm, T, k, with_shared ? 1 : 0, d, q, scale,
+                                                as_stream(stream)));
+}
+
 moe_status moe_quantize_act_fp8_permuted(const uint16_t* x, const int32_t* perm, int32_t T,
                                          int32_t k, int32_t with_shared, int32_t d, uint8_t* q,
                                          float* scale, void* stream) {
@@ -393,13 +453,13 @@ moe_status moe_permute(const int32_t* ids, int32_t T, int32_t E, int32_t k, int3
 }
 
 moe_status moe_gemm_gateup(const moe_shape* shape, const moe_weights* weights, const void* x,
-                           const float* x_scale, const int32_t* perm, const int32_t* offsets,
-                           void* h, float* h_scale, void* ws, size_t ws_bytes, void* stream) {
+                           const void* x_scale, const int32_t* perm, const int32_t* offsets,
+                           void* h, void* h_scale, void* ws, size_t ws_bytes, void* stream) {
     moe_status r = check_shape(shape);
     if (r != MOE_OK) return r;
     if ((r = check_weights(shape, weights, true, false, false)) != MOE_OK) return r;
     if (shape->T == 0) return MOE_OK;
-    const bool fp8 = shape->wdtype == MOE_WDTYPE_FP8_BLOCK128;
+    const bool fp8 = shape->wdtype != MOE_WDTYPE_BF16;  // FP8 or MXFP8: permuted e4m3 rows
     if (x == nullptr || offsets == nullptr || h == nullptr || (!fp8 && perm == nullptr) ||
         (fp8 && (x_scale == nullptr || h_scale == nullptr)))
         return MOE_ERR_INVALID_ARG;
@@ -412,13 +472,13 @@ moe_status moe_gemm_gateup(const moe_shape* shape, const moe_weights* weights, c
 }
 
 moe_status moe_gemm_down(const moe_shape* shape, const moe_weights* weights, const void* h,
-                         const float* h_scale, const int32_t* offsets, float* o, void* ws,
+                         const void* h_scale, const int32_t* offsets, float* o, void* ws,
                          size_t ws_bytes, void* stream) {
     moe_status r = check_shape(shape);
     if (r != MOE_OK) return r;
     if ((r = check_weights(shape, weights, false, true, false)) != MOE_OK) return r;
     if (shape->T == 0) return MOE_OK;
-    const bool fp8 = shape->wdtype == MOE_WDTYPE_FP8_BLOCK128;
+    const bool fp8 = shape->wdtype != MOE_WDTYPE_BF16;
     if (h == nullptr || offsets == nullptr || o == nullptr || (fp8 && h_scale == nullptr))
         return MOE_ERR_INVALID_ARG;
     if ((r = check_ws(ws, ws_bytes, kWsHeader)) != MOE_OK) return r;

@@ -213,6 +213,12 @@ __device__ __forceinline__ void cp_async_4(uint32_t dst, const void* src, uint32
                  "r"(src_bytes)
                  : "memory");
 }
+// Arrives on `bar` (without raising its expected count) once all of this
+// thread's earlier cp.async copies have landed.
+__device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t* bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() {
     asm volatile("cp.async.commit_group;" ::: "memory");
 }
@@ -274,6 +280,54 @@ __device__ __forceinline__ void umma_e4m3(uint32_t d_tmem, uint64_t a_desc, uint
         "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
+}
+
+// ------------------------------------------------------------ block-scaled
+// Instruction descriptor of kind::mxf8f6f4 with block scaling (E8M0 scales,
+// one per 32 K-elements): A/B format 0 = e4m3 (bits 7-9, 10-12), both
+// K-major, N >> 3 (17-22), scale format 1 = E8M0 (bit 23), M >> 4 (24-28);
+// the B and A scale-factor ids (bits 4-5, 29-30) pick the byte of the
+// 32-bit TMEM scale cells that this MMA reads.  D is always FP32.
+__host__ __device__ constexpr uint32_t idesc_mx_e4m3(int M, int N) {
+    return (static_cast<uint32_t>(N >> 3) << 17) | (1u << 23) |
+           (static_cast<uint32_t>(M >> 4) << 24);
+}
+__device__ __forceinline__ uint32_t idesc_with_sf_id(uint32_t idesc, uint32_t id) {
+    return idesc | (id << 4) | (id << 29);
+}
+
+// D[tmem] (+)= (A * 2^sfa) (B * 2^sfb)^T with per-32 E8M0 scales read from
+// TMEM at sfa / sfb (the top two address bits select the byte, matching the
+// descriptor's scale-factor ids).
+__device__ __forceinline__ void umma_mx_e4m3(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                             uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                             uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+        : "memory");
+}
+
+// Shared-memory descriptor of a K-major operand without swizzle: core
+// matrices of 8 rows x 16 bytes stored contiguously (128 bytes), the next 8
+// rows `sbo` bytes on; one core matrix along K (the 16-byte rows of the
+// scale-factor copies below).
+__device__ __forceinline__ uint64_t sdesc_k_noswizzle(uint32_t saddr, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>(128u >> 4) << 16;
+    d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+    d |= static_cast<uint64_t>(1u) << 46;
+    return d;
+}
+
+// Copies 32 rows x 16 bytes from shared memory into TMEM lanes 0-31, columns
+// taddr .. taddr+3, and the same data into lanes 32-63, 64-95 and 96-127
+// (the replication the block-scaled MMA expects of its scale factors).
+__device__ __forceinline__ void tmem_cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+                 : "memory");
 }
 
 // CTA-pair MMA (issued by the pair leader): A rows from both CTAs' shared
@@ -378,6 +432,30 @@ __device__ __forceinline__ void tmem_load16(uint32_t taddr, float* v) {
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// Two 16-column loads (e.g. matching gate and up columns) behind one wait.
+__device__ __forceinline__ void tmem_load16x2(uint32_t taddr0, uint32_t taddr1, float* v0,
+                                              float* v1) {
+    uint32_t a[16], b[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%32];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%33];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3]), "=r"(a[4]), "=r"(a[5]), "=r"(a[6]),
+          "=r"(a[7]), "=r"(a[8]), "=r"(a[9]), "=r"(a[10]), "=r"(a[11]), "=r"(a[12]),
+          "=r"(a[13]), "=r"(a[14]), "=r"(a[15]), "=r"(b[0]), "=r"(b[1]), "=r"(b[2]), "=r"(b[3]),
+          "=r"(b[4]), "=r"(b[5]), "=r"(b[6]), "=r"(b[7]), "=r"(b[8]), "=r"(b[9]), "=r"(b[10]),
+          "=r"(b[11]), "=r"(b[12]), "=r"(b[13]), "=r"(b[14]), "=r"(b[15])
+        : "r"(taddr0), "r"(taddr1)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        v0[i] = __uint_as_float(a[i]);
+        v1[i] = __uint_as_float(b[i]);
+    }
+}
+
 // Two 32-column loads (e.g. gate and up halves) behind one wait.
 __device__ __forceinline__ void tmem_load32x2(uint32_t taddr0, uint32_t taddr1, float* v0,
                                               float* v1) {
@@ -417,6 +495,25 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 __device__ __forceinline__ float silu_f(float z) { return z / (1.0f + expf(-z)); }
+
+// MXFP8 element quantisation of one block of 32 values with FP32 amax: the
+// E8M0 byte b = (exponent field of amax) - 8, clamped to [0, 254] (0 for a
+// zero or subnormal amax), i.e. shared_exp = floor(log2 amax) - 8; codes are
+// e4m3 cvt.rn.satfinite of v * 2^(127 - b), an exact power-of-two scaling.
+__device__ __forceinline__ uint32_t mx_scale_byte(float amax) {
+    const int ef = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFFu);
+    if (ef == 0) return 0u;
+    const int b = ef - 8;
+    return static_cast<uint32_t>(b < 0 ? 0 : (b > 254 ? 254 : b));
+}
+
+__device__ __forceinline__ uint32_t mx_quant4(const float* f, float inv) {
+    const __nv_fp8x2_storage_t lo =
+        __nv_cvt_float2_to_fp8x2(make_float2(f[0] * inv, f[1] * inv), __NV_SATFINITE, __NV_E4M3);
+    const __nv_fp8x2_storage_t hi =
+        __nv_cvt_float2_to_fp8x2(make_float2(f[2] * inv, f[3] * inv), __NV_SATFINITE, __NV_E4M3);
+    return (uint32_t)lo | ((uint32_t)hi << 16);
+}
 
 // 16-byte global store
 __device__ __forceinline__ void st_global_v4(void* p, uint32_t a, uint32_t b, uint32_t c,

@@ -44,6 +44,13 @@ cudaError_t launch_quant_act_fp8_permuted(const uint16_t* x, const int32_t* perm
                                           cudaStream_t s);
 cudaError_t launch_quant_weights_fp8(const uint16_t* W, int64_t batch, int rows, int cols,
                                      uint8_t* q, float* scale, cudaStream_t s);
+// MXFP8 (e4m3 + E8M0 scale per 1x32 along the row): rows as they are, or in
+// the permuted row order of the grouped GEMMs.  scale [rows][cols/32] bytes.
+cudaError_t launch_quant_mx_rows(const uint16_t* x, int64_t rows, int cols, uint8_t* q,
+                                 uint8_t* scale, cudaStream_t s);
+cudaError_t launch_quant_mx_permuted(const uint16_t* x, const int32_t* perm, int T, int k,
+                                     int has_shared, int cols, uint8_t* q, uint8_t* scale,
+                                     cudaStream_t s);
 cudaError_t launch_selftest_timeout(int32_t* status, uint64_t limit_ns, cudaStream_t s);
 
 // ---- router.cu (tcgen05 dual-BF16 GEMM)
@@ -85,6 +92,15 @@ cudaError_t launch_gateup_fp8(const GroupedGemmArgs& a, const uint8_t* xq, const
 cudaError_t launch_down_fp8(const GroupedGemmArgs& a, const uint8_t* hq, const float* hs,
                             const uint8_t* w_d, const float* w_d_s, const uint8_t* ws_d,
                             const float* ws_d_s, float* o, cudaStream_t s);
+
+// ---- gemm_mx.cu (tcgen05 block-scaled grouped GEMMs, MXFP8: e4m3 + E8M0 per 1x32)
+// Scales are bytes [rows][K/32]; h / o as in the FP8 path.
+cudaError_t launch_gateup_mx(const GroupedGemmArgs& a, const uint8_t* xq, const uint8_t* xs,
+                             const uint8_t* w_gu, const uint8_t* w_gu_s, const uint8_t* ws_gu,
+                             const uint8_t* ws_gu_s, uint8_t* hq, uint8_t* hs, cudaStream_t s);
+cudaError_t launch_down_mx(const GroupedGemmArgs& a, const uint8_t* hq, const uint8_t* hs,
+                           const uint8_t* w_d, const uint8_t* w_d_s, const uint8_t* ws_d,
+                           const uint8_t* ws_d_s, float* o, cudaStream_t s);
 
 // ---- tensor maps (api.cu)
 // 2-D row-major tensor [rows][cols] of `elem_bytes`-sized elements, box

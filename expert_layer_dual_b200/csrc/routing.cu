@@ -426,6 +426,81 @@ cudaError_t launch_quant_act_fp8(const uint16_t* x, int64_t rows, int cols, uint
     return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------------------
+// MXFP8 quantisation (OCP microscaling): each block of 32 consecutive values
+// along a row shares one E8M0 scale X = 2^(b - 127).  For the block's FP32
+// amax, b = (exponent field of amax) - 8, i.e. shared_exp = floor(log2 amax)
+// - 8 (8 = exponent of e4m3's largest normal), clamped to [0, 254] (0 for a
+// zero or subnormal amax).  q = e4m3 cvt.rn.satfinite of v * 2^(127 - b): a
+// power-of-two scaling, exact in FP32, so the decision is the oracle's.
+// ---------------------------------------------------------------------------
+// One warp quantises one row: each step covers 256 columns (8 blocks), 8
+// values (16 bytes) per lane; a block's amax is a 4-lane shuffle reduction.
+__device__ __forceinline__ void mx_row(const uint16_t* __restrict__ src, int cols,
+                                       uint8_t* __restrict__ qrow, uint8_t* __restrict__ srow) {
+    const int lane = threadIdx.x & 31;
+    for (int c0 = 0; c0 < cols; c0 += 256) {
+        const int c = c0 + lane * 8;
+        const bool active = c < cols;
+        uint4 u = make_uint4(0, 0, 0, 0);
+        if (active) u = *reinterpret_cast<const uint4*>(src + c);
+        float f[8];
+        bf16x8_to_f32(u, f);
+        float amax = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+        const uint32_t b = mx_scale_byte(amax);
+        const float inv = __uint_as_float((254u - b) << 23);  // 2^(127 - b), b <= 253 here
+        if (active) {
+            uint2 q;
+            q.x = mx_quant4(f, inv);
+            q.y = mx_quant4(f + 4, inv);
+            *reinterpret_cast<uint2*>(qrow + c) = q;
+            if ((lane & 3) == 0) srow[c / 32] = static_cast<uint8_t>(b);
+        }
+    }
+}
+
+__global__ void __launch_bounds__(256)
+    k_quant_mx_rows(const uint16_t* __restrict__ x, int64_t rows, int cols, uint8_t* __restrict__ q,
+                    uint8_t* __restrict__ scale) {
+    const int64_t r = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+    if (r >= rows) return;
+    mx_row(x + r * cols, cols, q + r * cols, scale + r * (cols / 32));
+}
+
+// Same, written in the permuted row order of the grouped GEMMs (row p < T*k
+// holds token perm[p] / k, row T*k + t holds token t).
+__global__ void __launch_bounds__(256)
+    k_quant_mx_permuted(const uint16_t* __restrict__ x, const int32_t* __restrict__ perm, int T,
+                        int k, int64_t rows, int cols, uint8_t* __restrict__ q,
+                        uint8_t* __restrict__ scale) {
+    const int64_t p = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+    if (p >= rows) return;
+    const int64_t Tk = (int64_t)T * k;
+    const int64_t tok = p < Tk ? (int64_t)(perm[p] / k) : p - Tk;
+    mx_row(x + tok * cols, cols, q + p * cols, scale + p * (cols / 32));
+}
+
+cudaError_t launch_quant_mx_rows(const uint16_t* x, int64_t rows, int cols, uint8_t* q,
+                                 uint8_t* scale, cudaStream_t s) {
+    if (rows == 0) return cudaSuccess;
+    k_quant_mx_rows<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(x, rows, cols, q, scale);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quant_mx_permuted(const uint16_t* x, const int32_t* perm, int T, int k,
+                                     int has_shared, int cols, uint8_t* q, uint8_t* scale,
+                                     cudaStream_t s) {
+    const int64_t rows = (int64_t)T * k + (has_shared ? T : 0);
+    if (rows == 0) return cudaSuccess;
+    k_quant_mx_permuted<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(x, perm, T, k, rows, cols, q,
+                                                                   scale);
+    return cudaGetLastError();
+}
+
 // one block of 256 threads per 128x128 block; thread = half a row (64 values)
 __global__ void __launch_bounds__(256)
     k_quant_w(const uint16_t* __restrict__ W, int rows, int cols, uint8_t* __restrict__ q,

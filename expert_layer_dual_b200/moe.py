@@ -28,11 +28,12 @@ if not os.path.exists(LIB_PATH):
 _lib = ctypes.CDLL(LIB_PATH)
 
 OK, INVALID_ARG, UNSUPPORTED, CUDA_ERROR, WORKSPACE_TOO_SMALL, DEVICE_TIMEOUT, DEVICE_BAD_INDEX = range(7)
-WDTYPE_BF16, WDTYPE_FP8_BLOCK128 = 0, 1
+WDTYPE_BF16, WDTYPE_FP8_BLOCK128, WDTYPE_MXFP8 = 0, 1, 2
 
 EXPORTS = ["moe_status_string", "moe_workspace_bytes", "moe_permute_workspace_bytes",
            "moe_router_split", "moe_quantize_weights_fp8", "moe_quantize_act_fp8",
-           "moe_quantize_act_fp8_permuted",
+           "moe_quantize_act_fp8_permuted", "moe_quantize_weights_mxfp8", "moe_quantize_act_mxfp8",
+           "moe_quantize_act_mxfp8_permuted",
            "moe_router_logits", "moe_route_topk", "moe_permute", "moe_permute_noalloc",
            "moe_gemm_gateup",
            "moe_gemm_down", "moe_combine", "moe_forward", "moe_forward_profiled", "moe_forward_host",
@@ -61,6 +62,9 @@ _sig = {
     "moe_quantize_weights_fp8": (_i32, [_vp, _i64, _i32, _i32, _vp, _vp, _vp]),
     "moe_quantize_act_fp8": (_i32, [_vp, _i64, _i32, _vp, _vp, _vp]),
     "moe_quantize_act_fp8_permuted": (_i32, [_vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
+    "moe_quantize_weights_mxfp8": (_i32, [_vp, _i64, _i32, _i32, _vp, _vp, _vp]),
+    "moe_quantize_act_mxfp8": (_i32, [_vp, _i64, _i32, _vp, _vp, _vp]),
+    "moe_quantize_act_mxfp8_permuted": (_i32, [_vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
     "moe_router_logits": (_i32, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _vp]),
     "moe_route_topk": (_i32, [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
     "moe_permute": (_i32, [_vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
@@ -137,6 +141,27 @@ def quantize_act_fp8(x, q, scale, stream=None):
     rows, cols = x.shape
     _check(_lib.moe_quantize_act_fp8(_p(x), rows, cols, _p(q), _p(scale), _stream(stream)),
            "moe_quantize_act_fp8")
+
+
+def quantize_weights_mxfp8(W, q, scale, stream=None):
+    """W bf16 bits [..., rows, cols] -> q e4m3 codes (same shape), scale E8M0 bytes [..., rows, cols/32]."""
+    rows, cols = W.shape[-2:]
+    batch = W.numel() // (rows * cols)
+    _check(_lib.moe_quantize_weights_mxfp8(_p(W), batch, rows, cols, _p(q), _p(scale), _stream(stream)),
+           "moe_quantize_weights_mxfp8")
+
+
+def quantize_act_mxfp8(x, q, scale, stream=None):
+    rows, cols = x.shape
+    _check(_lib.moe_quantize_act_mxfp8(_p(x), rows, cols, _p(q), _p(scale), _stream(stream)),
+           "moe_quantize_act_mxfp8")
+
+
+def quantize_act_mxfp8_permuted(x, perm, k, with_shared, q, scale, stream=None):
+    T, d = x.shape
+    _check(_lib.moe_quantize_act_mxfp8_permuted(_p(x), _p(perm), T, k, int(with_shared), d, _p(q),
+                                                _p(scale), _stream(stream)),
+           "moe_quantize_act_mxfp8_permuted")
 
 
 def quantize_act_fp8_permuted(x, perm, k, with_shared, q, scale, stream=None):
@@ -255,6 +280,11 @@ class MoELayer:
                 s = torch.empty(t.shape[:-2] + (t.shape[-2] // 128, t.shape[-1] // 128),
                                 dtype=torch.float32, device=dev)
                 quantize_weights_fp8(t.view(torch.uint16), q, s)
+                self.mats[name], self.scales[name] = q, s
+            elif cfg.wdtype == WDTYPE_MXFP8:
+                q = torch.empty(t.shape, dtype=torch.uint8, device=dev)
+                s = torch.empty(t.shape[:-1] + (t.shape[-1] // 32,), dtype=torch.uint8, device=dev)
+                quantize_weights_mxfp8(t.view(torch.uint16), q, s)
                 self.mats[name], self.scales[name] = q, s
             else:
                 self.mats[name], self.scales[name] = t.view(torch.uint16), None

@@ -67,6 +67,9 @@ typedef int32_t moe_status;
 #define MOE_WDTYPE_BF16 0           /* expert weights bf16                         */
 #define MOE_WDTYPE_FP8_BLOCK128 1   /* expert weights e4m3 + f32 scale per 128x128
                                        block; activations quantised per 1x128     */
+#define MOE_WDTYPE_MXFP8 2          /* MXFP8: weights and activations e4m3 with one
+                                       E8M0 (power-of-two) scale byte per 1x32
+                                       block along K; native block-scaled MMA      */
 
 /* Layer shape.  T tokens of hidden size d; E routed experts of intermediate
  * size I, top-k routing; I_shared = 0 (no shared expert) or I. */
@@ -77,21 +80,22 @@ typedef struct moe_shape {
 } moe_shape;
 
 /* Layer weights (device).  Gate rows come first in every gate-up matrix.
- *   w_gu  [E][2I][d]   bf16 (wdtype 0) or e4m3 (wdtype 1)
+ *   w_gu  [E][2I][d]   bf16 (wdtype 0) or e4m3 (wdtype 1, 2)
  *   w_d   [E][d][I]
- *   w_gu_scale [E][2I/128][d/128], w_d_scale [E][d/128][I/128]  (wdtype 1)
+ *   wdtype 1: w_gu_scale float [E][2I/128][d/128], w_d_scale float [E][d/128][I/128]
+ *   wdtype 2: w_gu_scale uint8 E8M0 [E][2I][d/32], w_d_scale uint8 [E][d][I/32]
  *   ws_gu [2I][d], ws_d [d][I], ws_*_scale likewise  (when I_shared > 0)
  *   router_hi, router_lo [E][d] bf16 from moe_router_split; router_bias [E]
  *   or NULL (added to the logits, so it steers both selection and weights). */
 typedef struct moe_weights {
     const void* w_gu;
     const void* w_d;
-    const float* w_gu_scale;
-    const float* w_d_scale;
+    const void* w_gu_scale;   /* float (wdtype 1) or uint8 E8M0 (wdtype 2) */
+    const void* w_d_scale;
     const void* ws_gu;
     const void* ws_d;
-    const float* ws_gu_scale;
-    const float* ws_d_scale;
+    const void* ws_gu_scale;
+    const void* ws_d_scale;
     const uint16_t* router_hi;
     const uint16_t* router_lo;
     const float* router_bias;
@@ -126,6 +130,26 @@ moe_status moe_quantize_weights_fp8(const uint16_t* W, int64_t batch, int32_t ro
  * [rows][cols/128]. */
 moe_status moe_quantize_act_fp8(const uint16_t* x, int64_t rows, int32_t cols,
                                 uint8_t* q, float* scale, void* stream);
+
+/* [MX] Offline MXFP8 quantisation ("PR #54160 完整报告", section 实现拆解 item 4:
+ * the MXFP8 weight format; the format itself is OCP microscaling MXFP8 E4M3):
+ * each row of `batch` bf16 matrices [rows][cols] (cols % 128 == 0; K = cols)
+ * in blocks of 32: b = E8M0 byte of floor(log2 amax) - 8 (clamped to
+ * [0, 254], 0 for an all-zero block), q = e4m3_rne_satfinite(W * 2^(127-b)).
+ * q [batch][rows][cols], scale uint8 [batch][rows][cols/32]. */
+moe_status moe_quantize_weights_mxfp8(const uint16_t* W, int64_t batch, int32_t rows,
+                                      int32_t cols, uint8_t* q, uint8_t* scale, void* stream);
+
+/* [MX] The same quantisation of activation rows: x [rows][cols] bf16 ->
+ * q [rows][cols] e4m3, scale [rows][cols/32] E8M0. */
+moe_status moe_quantize_act_mxfp8(const uint16_t* x, int64_t rows, int32_t cols, uint8_t* q,
+                                  uint8_t* scale, void* stream);
+
+/* [MX] The same, in the permuted row order of the grouped GEMMs (as
+ * moe_quantize_act_fp8_permuted): q [R][d], scale [R][d/32]. */
+moe_status moe_quantize_act_mxfp8_permuted(const uint16_t* x, const int32_t* perm, int32_t T,
+                                           int32_t k, int32_t with_shared, int32_t d,
+                                           uint8_t* q, uint8_t* scale, void* stream);
 
 /* [FM] The same activation quantisation, written in the permuted row order
  * of the grouped GEMMs (the FP8 gate-up GEMM's A operand): row p < T*k holds
@@ -188,14 +212,18 @@ moe_status moe_permute_noalloc(const int32_t* ids, int32_t T, int32_t E, int32_t
  * the shared expert on token p - T*k.
  *   h[p][n] = silu(x_t . Wg[e][n]) * (x_t . Wu[e][n]),  FP32 accumulation.
  * wdtype 0: x [T][d] bf16, x_scale NULL; h [R][I] bf16, h_scale NULL.
- * wdtype 1: x [R][d] e4m3 rows already in permuted order with x_scale
+ * wdtype 1: x [R][d] e4m3 rows already in permuted order with x_scale float
  *           [R][d/128] (moe_quantize_act_fp8_permuted; perm is then not read
- *           and may be NULL); h [R][I] e4m3 with h_scale [R][I/128] (1x128
- *           quantisation of the FP32 h in the epilogue).
- * R = T*k + (I_shared ? T : 0).  ws: at least 256 bytes (the status word). */
+ *           and may be NULL); h [R][I] e4m3 with h_scale float [R][I/128]
+ *           (1x128 quantisation of the FP32 h in the epilogue).
+ * wdtype 2: the same with MXFP8: x_scale uint8 E8M0 [R][d/32]
+ *           (moe_quantize_act_mxfp8_permuted), h_scale uint8 [R][I/32] (each
+ *           1x32 block of the FP32 h quantised in the epilogue).
+ * R = T*k + (I_shared ? T : 0).  ws: at least 256 bytes (the status word and
+ * the tile counter). */
 moe_status moe_gemm_gateup(const moe_shape* shape, const moe_weights* weights,
-                           const void* x, const float* x_scale, const int32_t* perm,
-                           const int32_t* offsets, void* h, float* h_scale,
+                           const void* x, const void* x_scale, const int32_t* perm,
+                           const int32_t* offsets, void* h, void* h_scale,
                            void* ws, size_t ws_bytes, void* stream);
 
 /* [FM][G8] Grouped Down GEMM: o[p] = h[p] . Wd[e]^T with FP32 accumulation,
@@ -203,7 +231,7 @@ moe_status moe_gemm_gateup(const moe_shape* shape, const moe_weights* weights,
  * rows stay FP32 until the weighted combine so the layer output is rounded
  * to bf16 once.)  ws: at least 256 bytes (the status word). */
 moe_status moe_gemm_down(const moe_shape* shape, const moe_weights* weights,
-                         const void* h, const float* h_scale, const int32_t* offsets,
+                         const void* h, const void* h_scale, const int32_t* offsets,
                          float* o, void* ws, size_t ws_bytes, void* stream);
 
 /* [FM] Top-K weighted aggregation plus the shared expert:

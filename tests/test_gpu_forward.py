@@ -33,6 +33,8 @@ SMALL = [
     MoEConfig("norenorm", T=64, d=256, E=32, k=4, I=128, Is=0, renorm=False, seed=26),
     MoEConfig("fp8small", T=200, d=512, E=16, k=4, I=256, Is=256, wdtype=1, seed=31),
     MoEConfig("fp8odd", T=77, d=384, E=8, k=2, I=128, Is=0, wdtype=1, seed=32),
+    MoEConfig("mxsmall", T=200, d=512, E=16, k=4, I=256, Is=256, wdtype=2, seed=33),
+    MoEConfig("mxodd", T=77, d=384, E=8, k=2, I=128, Is=0, wdtype=2, seed=34),
 ]
 
 
