@@ -372,11 +372,11 @@ moe_status moe_quantize_act_fp8(const uint16_t* x, int64_t rows, int32_t cols, u
 moe_status moe_quantize_weights_mxfp8(const uint16_t* W, int64_t batch, int32_t rows, int32_t cols,
                                       uint8_t* q, uint8_t* scale, void* stream) {
     if (batch < 0 || rows < 0 || cols < 0) return MOE_ERR_INVALID_ARG;
-    if (cols % 128 != 0) return MOE_ERR_UNSUPPORTED;
+    if (cols % 128 != 0 || rows % 128 != 0) return MOE_ERR_UNSUPPORTED;
     if (batch * rows * (int64_t)cols == 0) return MOE_OK;
     if (W == nullptr || q == nullptr || scale == nullptr) return MOE_ERR_INVALID_ARG;
     if (!device_ok()) return MOE_ERR_UNSUPPORTED;
-    return cuda_status(launch_quant_mx_rows(W, batch * rows, cols, q, scale, as_stream(stream)));
+    return cuda_status(launch_quant_mx_weights(W, batch, rows, cols, q, scale, as_stream(stream)));
 }
 
 moe_status moe_quantize_act_mxfp8(const uint16_t* x, int64_t rows, int32_t cols, uint8_t* q,

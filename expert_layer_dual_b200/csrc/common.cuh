@@ -167,6 +167,16 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
         : "memory");
 }
 
+// 1-D bulk copy global -> shared (no multicast) completing on `bar` with its
+// byte count; both addresses 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
 // Tile load of one CTA of a CTA pair: the bytes land in this CTA's shared
 // memory and are counted on the barrier at `bar_cluster` (the pair leader's).
 __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map,

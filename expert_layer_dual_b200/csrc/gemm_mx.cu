@@ -15,10 +15,16 @@
 //    256-column FP32 accumulator; the rest of TMEM holds the scale factors;
 //  - operands by TMA into a 4-stage ring (128-byte swizzle), as in the other
 //    grouped GEMMs, tiles from the dynamic schedule of grouped_common.cuh;
-//  - a scale warp gathers each k-block's scale bytes (4 per row: one per
-//    MMA) for the tile's 128 A rows and 256 B rows into shared memory with
-//    4-byte cp.async copies, in the layout tcgen05.cp reads: 32 rows of 16
-//    bytes, byte 4g + j of row l = scale j of tile row 32g + l;
+//  - each k-block needs 4 scale bytes (one per MMA) for each of the tile's
+//    128 A rows and 256 B rows, in shared memory in the layout tcgen05.cp
+//    reads: 32 rows of 16 bytes, byte 4g + j of row l = scale j of tile row
+//    32g + l.  Weight scales are stored offline in exactly that image (512
+//    bytes per k-block and 128-row block), so the TMA thread fetches them
+//    with two 1-D bulk copies beside the operand tiles; activation scales are
+//    k-block-major ([K/128][rows][4], written that way by the quantiser and
+//    by the gate-up epilogue) and a scale warp gathers the tile's 128 records
+//    with coalesced 4-byte cp.async copies (the tile's first row is arbitrary,
+//    so its 512 bytes are not 16-byte aligned for a bulk copy);
 //  - the MMA thread copies them into TMEM with tcgen05.cp (32x128b.warpx4:
 //    the 32 rows go to every 32-lane subpartition, as the block-scaled MMA
 //    expects), then issues the 4 MMAs, MMA j reading byte j of the 32-bit
@@ -118,10 +124,13 @@ __device__ __forceinline__ void teardown(uint32_t tmem) {
 
 // Weight rows of a tile's B operand: half 0 rows rb0.., half 1 rows rb1..
 // (`two` false: the second half lies past the matrix and is not loaded).
+// Their scales: the matrix's scale image, 128-row blocks lb0 / lb1 of the
+// matrix's mrows rows.
 struct BRows {
     const CUtensorMap* map;
-    const uint8_t* scale;  // E8M0 scales of the weight matrix, [rows][K/32]
+    const uint8_t* scale;
     int rb0, rb1;
+    int lb0, lb1, mrows;
     bool two;
 };
 
@@ -151,10 +160,16 @@ __device__ __forceinline__ void tma_role(Smem& sm, const GroupedGemmArgs& a, con
                 break;
             }
             uint8_t* st = sm.stages + s * STAGE_BYTES;
-            mbar_arrive_expect_tx(&b->full[s], A_BYTES + (L.two ? B_BYTES : B_HALF));
+            uint8_t* sf = sm.sf + s * SF_STAGE + SFA_BYTES;
+            const uint8_t* img = L.scale + (int64_t)kb * (L.mrows / 128) * 512;
+            mbar_arrive_expect_tx(&b->full[s], L.two ? B_BYTES + A_BYTES + 1024 : B_HALF + A_BYTES + 512);
             tma_load_2d(st, tm_a, &b->full[s], kb * BK, t.row0);
             tma_load_2d(st + A_BYTES, L.map, &b->full[s], kb * BK, L.rb0);
-            if (L.two) tma_load_2d(st + A_BYTES + B_HALF, L.map, &b->full[s], kb * BK, L.rb1);
+            bulk_load(sf, img + L.lb0 * 512, 512, &b->full[s]);
+            if (L.two) {
+                tma_load_2d(st + A_BYTES + B_HALF, L.map, &b->full[s], kb * BK, L.rb1);
+                bulk_load(sf + 512, img + L.lb1 * 512, 512, &b->full[s]);
+            }
             ++issued;
         }
     }
@@ -176,30 +191,27 @@ __device__ __forceinline__ uint32_t sf_offset(int r) {
     return static_cast<uint32_t>((r >> 7) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4);
 }
 
-// Scale warp: per k-block, 128 A rows and 256 B rows of 4 scale bytes each,
-// as 4-byte cp.async copies (12 per lane); rows past the tile (or past the
-// weight matrix) are zero-filled.  Each lane then arms an arrival on the
+// Scale warp: per k-block, the 128 A rows' 4-byte scale records (k-block-
+// major: contiguous across rows, so each warp copy reads 128 contiguous
+// bytes), 4 cp.async per lane; rows past the tile are zero-filled.  Each lane then arms an arrival on the
 // stage's sf_full barrier (32 arrivals) that fires when its copies land, so a
 // stage is published as soon as its bytes are in shared memory and the warp
 // never waits for its own copies.  (Publishing a stage only after waiting
 // for it, one or three stages later, starved the MMA: measured 1.72 and
 // 2.39 ms for the FP8-sized gate-up.)  The MMA thread orders the landed
 // bytes before its async-proxy reads with fence.proxy.async.
-template <typename RowsOf>
 __device__ __forceinline__ void scale_role(Smem& sm, const GroupedGemmArgs& a, int G, int n_tiles,
                                            int nk, const uint8_t* __restrict__ act_scale,
-                                           RowsOf rows_of) {
+                                           int64_t R) {
     Bars* b = sm.bars;
     const volatile int* ab = &b->abort_flag;
     const int lane = threadIdx.x & 31;
-    const int kbytes = nk * 4;  // scale bytes per row (K / 32)
     uint32_t it = 0;
     bool ok = true;
     for (uint32_t lt = 0; ok; ++lt) {
         const int tile = tile_ring_pop_warp(&b->ring, lt, a.timeout_ns, ab, ok);
         if (tile < 0) break;
         const Tile t = decode_tile(sm.tt, G, n_tiles, tile, BM);
-        const BRows L = rows_of(t);
         for (int kb = 0; kb < nk; ++kb, ++it) {
             const int s = it % STAGES;
             const uint32_t ph = (it / STAGES) & 1;
@@ -213,16 +225,7 @@ __device__ __forceinline__ void scale_role(Smem& sm, const GroupedGemmArgs& a, i
                 const int r = lane + 32 * i;
                 const bool in = r < t.nrows;
                 cp_async_4(dst + sf_offset(r),
-                           act_scale + (in ? (int64_t)(t.row0 + r) * kbytes + kb * 4 : 0),
-                           in ? 4u : 0u);
-            }
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int r = lane + 32 * i;  // B row of the tile: half r / 128
-                const bool in = r < 128 || L.two;
-                const int wr = (r < 128 ? L.rb0 : L.rb1) + (r & 127);
-                cp_async_4(dst + SFA_BYTES + sf_offset(r),
-                           L.scale + (in ? (int64_t)wr * kbytes + kb * 4 : 0), in ? 4u : 0u);
+                           act_scale + (in ? ((int64_t)kb * R + t.row0 + r) * 4 : 0), in ? 4u : 0u);
             }
             cp_async_mbar_arrive_noinc(&b->sf_full[s]);
         }
@@ -300,10 +303,12 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int G = a.E + a.has_shared;
     const int n_tiles = a.I / 128;
     const int nk = a.d / BK;
+    const int64_t R = (int64_t)a.T * a.k + (a.has_shared ? a.T : 0);
     auto rows_of = [&](const Tile& t) {
         const bool shared = t.g >= a.E;
         const int r0 = (shared ? 0 : t.g * 2 * a.I) + t.n * 128;
-        return BRows{shared ? &tm_ws : &tm_w, shared ? wssc : wsc, r0, r0 + a.I, true};
+        const uint8_t* img = shared ? wssc : wsc + (int64_t)t.g * 2 * a.I * (a.d / 32);
+        return BRows{shared ? &tm_ws : &tm_w, img, r0, r0 + a.I, t.n, a.I / 128 + t.n, 2 * a.I, true};
     };
     if (warp == TMA_WARP) {
         if (lane == 0) {
@@ -315,7 +320,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     } else if (warp == MMA_WARP) {
         if (lane == 0) mma_role(sm, a, tmem, nk);
     } else if (warp == SCALE_WARP) {
-        scale_role(sm, a, G, n_tiles, nk, xs, rows_of);
+        scale_role(sm, a, G, n_tiles, nk, xs, R);
     } else if (warp < EPI_WARPS) {
         const int quad = warp & 3, qtr = warp >> 2;
         const int row = quad * 32 + lane;
@@ -356,7 +361,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                     st_global_v4(dst + 16 * q, mx_quant4(h + 16 * q, inv),
                                  mx_quant4(h + 16 * q + 4, inv), mx_quant4(h + 16 * q + 8, inv),
                                  mx_quant4(h + 16 * q + 12, inv));
-                hs[p * (a.I / 32) + t.n * 4 + qtr] = static_cast<uint8_t>(sb);
+                hs[((int64_t)t.n * R + p) * 4 + qtr] = static_cast<uint8_t>(sb);  // k-block-major
             }
         }
     }
@@ -380,10 +385,12 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int G = a.E + a.has_shared;
     const int n_tiles = (a.d + BN - 1) / BN;
     const int nk = a.I / BK;
+    const int64_t R = (int64_t)a.T * a.k + (a.has_shared ? a.T : 0);
     auto rows_of = [&](const Tile& t) {
         const bool shared = t.g >= a.E;
         const int r0 = (shared ? 0 : t.g * a.d) + t.n * BN;
-        return BRows{shared ? &tm_ws : &tm_w, shared ? wssc : wsc, r0, r0 + 128,
+        const uint8_t* img = shared ? wssc : wsc + (int64_t)t.g * a.d * (a.I / 32);
+        return BRows{shared ? &tm_ws : &tm_w, img, r0, r0 + 128, 2 * t.n, 2 * t.n + 1, a.d,
                      t.n * BN + 128 < a.d};
     };
     if (warp == TMA_WARP) {
@@ -396,7 +403,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     } else if (warp == MMA_WARP) {
         if (lane == 0) mma_role(sm, a, tmem, nk);
     } else if (warp == SCALE_WARP) {
-        scale_role(sm, a, G, n_tiles, nk, hs, rows_of);
+        scale_role(sm, a, G, n_tiles, nk, hs, R);
     } else if (warp < EPI_WARPS) {
         const int quad = warp & 3, qtr = warp >> 2;
         const int row = quad * 32 + lane;

@@ -45,9 +45,13 @@ cudaError_t launch_quant_act_fp8_permuted(const uint16_t* x, const int32_t* perm
 cudaError_t launch_quant_weights_fp8(const uint16_t* W, int64_t batch, int rows, int cols,
                                      uint8_t* q, float* scale, cudaStream_t s);
 // MXFP8 (e4m3 + E8M0 scale per 1x32 along the row): rows as they are, or in
-// the permuted row order of the grouped GEMMs.  scale [rows][cols/32] bytes.
+// the permuted row order of the grouped GEMMs; scales k-block-major
+// [cols/128][rows][4].  Weights (rows % 128 == 0): scales in the per-matrix
+// image of the block-scaled MMA's scale copy (see routing.cu).
 cudaError_t launch_quant_mx_rows(const uint16_t* x, int64_t rows, int cols, uint8_t* q,
                                  uint8_t* scale, cudaStream_t s);
+cudaError_t launch_quant_mx_weights(const uint16_t* W, int64_t batch, int rows, int cols,
+                                    uint8_t* q, uint8_t* scale, cudaStream_t s);
 cudaError_t launch_quant_mx_permuted(const uint16_t* x, const int32_t* perm, int T, int k,
                                      int has_shared, int cols, uint8_t* q, uint8_t* scale,
                                      cudaStream_t s);

@@ -434,10 +434,30 @@ cudaError_t launch_quant_act_fp8(const uint16_t* x, int64_t rows, int cols, uint
 // zero or subnormal amax).  q = e4m3 cvt.rn.satfinite of v * 2^(127 - b): a
 // power-of-two scaling, exact in FP32, so the decision is the oracle's.
 // ---------------------------------------------------------------------------
+// Where the scale byte of block j (32 columns) of row r goes.  Activations:
+// k-block-major, [cols/128][rows][4] (byte j % 4 of row r's record for
+// k-block j / 4), so the GEMM's gathers of one k-block's rows are contiguous.
+// Weights: per matrix of `rows` rows, the image the block-scaled MMA's scale
+// copy reads: for each k-block and 128-row block, 512 bytes where row r of
+// the block is at (r % 32) * 16 + (r / 32) * 4 (+ j % 4).
+struct MxScaleLayout {
+    int64_t rows;  // rows of the k-block-major matrix, or of one weight matrix
+    int cols;
+    bool tiled;    // weights
+    __device__ __forceinline__ int64_t at(int64_t r, int j) const {
+        const int kb = j >> 2, kk = j & 3;
+        if (!tiled) return ((int64_t)kb * rows + r) * 4 + kk;
+        const int64_t m = r / rows, rl = r - m * rows;
+        return m * rows * (cols / 32) + ((int64_t)kb * (rows / 128) + rl / 128) * 512 +
+               (rl & 31) * 16 + ((rl & 127) >> 5) * 4 + kk;
+    }
+};
+
 // One warp quantises one row: each step covers 256 columns (8 blocks), 8
 // values (16 bytes) per lane; a block's amax is a 4-lane shuffle reduction.
 __device__ __forceinline__ void mx_row(const uint16_t* __restrict__ src, int cols,
-                                       uint8_t* __restrict__ qrow, uint8_t* __restrict__ srow) {
+                                       uint8_t* __restrict__ qrow, uint8_t* __restrict__ scale,
+                                       const MxScaleLayout& lay, int64_t r) {
     const int lane = threadIdx.x & 31;
     for (int c0 = 0; c0 < cols; c0 += 256) {
         const int c = c0 + lane * 8;
@@ -458,17 +478,17 @@ __device__ __forceinline__ void mx_row(const uint16_t* __restrict__ src, int col
             q.x = mx_quant4(f, inv);
             q.y = mx_quant4(f + 4, inv);
             *reinterpret_cast<uint2*>(qrow + c) = q;
-            if ((lane & 3) == 0) srow[c / 32] = static_cast<uint8_t>(b);
+            if ((lane & 3) == 0) scale[lay.at(r, c / 32)] = static_cast<uint8_t>(b);
         }
     }
 }
 
 __global__ void __launch_bounds__(256)
     k_quant_mx_rows(const uint16_t* __restrict__ x, int64_t rows, int cols, uint8_t* __restrict__ q,
-                    uint8_t* __restrict__ scale) {
+                    uint8_t* __restrict__ scale, MxScaleLayout lay) {
     const int64_t r = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
     if (r >= rows) return;
-    mx_row(x + r * cols, cols, q + r * cols, scale + r * (cols / 32));
+    mx_row(x + r * cols, cols, q + r * cols, scale, lay, r);
 }
 
 // Same, written in the permuted row order of the grouped GEMMs (row p < T*k
@@ -481,13 +501,23 @@ __global__ void __launch_bounds__(256)
     if (p >= rows) return;
     const int64_t Tk = (int64_t)T * k;
     const int64_t tok = p < Tk ? (int64_t)(perm[p] / k) : p - Tk;
-    mx_row(x + tok * cols, cols, q + p * cols, scale + p * (cols / 32));
+    mx_row(x + tok * cols, cols, q + p * cols, scale, MxScaleLayout{rows, cols, false}, p);
 }
 
 cudaError_t launch_quant_mx_rows(const uint16_t* x, int64_t rows, int cols, uint8_t* q,
                                  uint8_t* scale, cudaStream_t s) {
     if (rows == 0) return cudaSuccess;
-    k_quant_mx_rows<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(x, rows, cols, q, scale);
+    k_quant_mx_rows<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(x, rows, cols, q, scale,
+                                                               MxScaleLayout{rows, cols, false});
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quant_mx_weights(const uint16_t* W, int64_t batch, int rows, int cols,
+                                    uint8_t* q, uint8_t* scale, cudaStream_t s) {
+    const int64_t n = batch * rows;
+    if (n == 0) return cudaSuccess;
+    k_quant_mx_rows<<<(unsigned)((n + 7) / 8), 256, 0, s>>>(W, n, cols, q, scale,
+                                                            MxScaleLayout{rows, cols, true});
     return cudaGetLastError();
 }
 

@@ -83,7 +83,9 @@ typedef struct moe_shape {
  *   w_gu  [E][2I][d]   bf16 (wdtype 0) or e4m3 (wdtype 1, 2)
  *   w_d   [E][d][I]
  *   wdtype 1: w_gu_scale float [E][2I/128][d/128], w_d_scale float [E][d/128][I/128]
- *   wdtype 2: w_gu_scale uint8 E8M0 [E][2I][d/32], w_d_scale uint8 [E][d][I/32]
+ *   wdtype 2: w_gu_scale, w_d_scale uint8 E8M0, one per 1x32 block along K, in
+ *             the per-matrix image of moe_quantize_weights_mxfp8 (E matrices of
+ *             2I x d, resp. d x I)
  *   ws_gu [2I][d], ws_d [d][I], ws_*_scale likewise  (when I_shared > 0)
  *   router_hi, router_lo [E][d] bf16 from moe_router_split; router_bias [E]
  *   or NULL (added to the logits, so it steers both selection and weights). */
@@ -136,17 +138,23 @@ moe_status moe_quantize_act_fp8(const uint16_t* x, int64_t rows, int32_t cols,
  * each row of `batch` bf16 matrices [rows][cols] (cols % 128 == 0; K = cols)
  * in blocks of 32: b = E8M0 byte of floor(log2 amax) - 8 (clamped to
  * [0, 254], 0 for an all-zero block), q = e4m3_rne_satfinite(W * 2^(127-b)).
- * q [batch][rows][cols], scale uint8 [batch][rows][cols/32]. */
+ * rows % 128 == 0.  q [batch][rows][cols].  scale: batch*rows*cols/32 bytes in
+ * the image the grouped GEMMs copy into TMEM: for matrix m, row r, block j
+ * (K-block kb = j / 4 of 128 columns), at
+ *   m*rows*cols/32 + (kb*(rows/128) + r/128)*512 + (r%32)*16 + ((r%128)/32)*4 + j%4
+ * (each 512-byte piece is one k-block of 128 rows, fetched with one bulk copy). */
 moe_status moe_quantize_weights_mxfp8(const uint16_t* W, int64_t batch, int32_t rows,
                                       int32_t cols, uint8_t* q, uint8_t* scale, void* stream);
 
 /* [MX] The same quantisation of activation rows: x [rows][cols] bf16 ->
- * q [rows][cols] e4m3, scale [rows][cols/32] E8M0. */
+ * q [rows][cols] e4m3, scale E8M0 k-block-major [cols/128][rows][4] (byte j%4
+ * of row r's record for K-block j/4), so a GEMM's gather of one k-block's
+ * rows reads contiguous memory. */
 moe_status moe_quantize_act_mxfp8(const uint16_t* x, int64_t rows, int32_t cols, uint8_t* q,
                                   uint8_t* scale, void* stream);
 
 /* [MX] The same, in the permuted row order of the grouped GEMMs (as
- * moe_quantize_act_fp8_permuted): q [R][d], scale [R][d/32]. */
+ * moe_quantize_act_fp8_permuted): q [R][d], scale [d/128][R][4]. */
 moe_status moe_quantize_act_mxfp8_permuted(const uint16_t* x, const int32_t* perm, int32_t T,
                                            int32_t k, int32_t with_shared, int32_t d,
                                            uint8_t* q, uint8_t* scale, void* stream);
@@ -216,8 +224,8 @@ moe_status moe_permute_noalloc(const int32_t* ids, int32_t T, int32_t E, int32_t
  *           [R][d/128] (moe_quantize_act_fp8_permuted; perm is then not read
  *           and may be NULL); h [R][I] e4m3 with h_scale float [R][I/128]
  *           (1x128 quantisation of the FP32 h in the epilogue).
- * wdtype 2: the same with MXFP8: x_scale uint8 E8M0 [R][d/32]
- *           (moe_quantize_act_mxfp8_permuted), h_scale uint8 [R][I/32] (each
+ * wdtype 2: the same with MXFP8: x_scale uint8 E8M0 [d/128][R][4]
+ *           (moe_quantize_act_mxfp8_permuted), h_scale uint8 [I/128][R][4] (each
  *           1x32 block of the FP32 h quantised in the epilogue).
  * R = T*k + (I_shared ? T : 0).  ws: at least 256 bytes (the status word and
  * the tile counter). */

@@ -35,6 +35,18 @@ def _e8m0(b):
     return np.ldexp(1.0, b.astype(np.int64) - 127)
 
 
+def _kbm_to_rows(s, rows, cols):
+    """Activation scales, k-block-major [cols/128][rows][4] -> [rows][cols/32]."""
+    return s.reshape(cols // 128, rows, 4).transpose(1, 0, 2).reshape(rows, cols // 32)
+
+
+def _image_to_rows(s, batch, rows, cols):
+    """Weight scales in the block-scaled MMA's copy image -> [batch][rows][cols/32]:
+    per matrix, [k-block][128-row block][row % 32][row / 32 % 4][4]."""
+    a = s.reshape(batch, cols // 128, rows // 128, 32, 4, 4)      # b, kb, rb, l, g, kk
+    return a.transpose(0, 2, 4, 3, 1, 5).reshape(batch, rows, cols // 32)
+
+
 def _gpu_permute(ids_dev, E):
     T, k = ids_dev.shape
     counts = torch.empty(E, dtype=torch.int32, device=DEV)
@@ -56,18 +68,19 @@ def test_quantize_act_mxfp8_bit_exact(rows, cols):
     s = torch.empty((rows, cols // 32), dtype=torch.uint8, device=DEV)
     M.quantize_act_mxfp8(_u16(x.to(DEV)), q, s)
     oq, os_ = oracle.quant_mx_rows(x.float().numpy())
-    assert np.array_equal(s.cpu().numpy(), os_)
+    assert np.array_equal(_kbm_to_rows(s.cpu().numpy(), rows, cols), os_)
     assert np.array_equal(q.cpu().numpy(), oq)
 
 
-@pytest.mark.parametrize("batch,rows,cols", [(1, 1, 128), (3, 256, 384), (2, 2048, 1024)])
+@pytest.mark.parametrize("batch,rows,cols", [(1, 128, 128), (3, 256, 384), (2, 2048, 1024)])
 def test_quantize_weights_mxfp8_bit_exact(batch, rows, cols):
     W = random_bf16((batch, rows, cols), seed=rows + cols, idx=7, std=0.02)
     q = torch.empty(W.shape, dtype=torch.uint8, device=DEV)
     s = torch.empty((batch, rows, cols // 32), dtype=torch.uint8, device=DEV)
     M.quantize_weights_mxfp8(_u16(W.to(DEV)), q, s)
     oq, os_ = oracle.quant_mx_bf16(bits(W))
-    assert np.array_equal(s.cpu().numpy(), os_) and np.array_equal(q.cpu().numpy(), oq)
+    assert np.array_equal(_image_to_rows(s.cpu().numpy(), batch, rows, cols), os_)
+    assert np.array_equal(q.cpu().numpy(), oq)
 
 
 def _permuted_quant(x_dev, perm, cfg):
@@ -87,7 +100,8 @@ def test_quantize_act_mxfp8_permuted_bit_exact(cfg):
     _, _, operm, _ = oracle.permute(ids.numpy(), cfg.E)
     tok = np.concatenate([operm // cfg.k, np.arange(cfg.T) if cfg.Is else np.zeros(0, np.int64)])
     oq, os_ = oracle.quant_mx_rows(x.float().numpy()[tok])
-    assert np.array_equal(q.cpu().numpy(), oq) and np.array_equal(s.cpu().numpy(), os_)
+    assert np.array_equal(q.cpu().numpy(), oq)
+    assert np.array_equal(_kbm_to_rows(s.cpu().numpy(), cfg.rows(), cfg.d), os_)
 
 
 @pytest.mark.parametrize("cfg", MX, ids=MX_IDS)
@@ -96,7 +110,7 @@ def test_weights_mxfp8_match_oracle_quantisation(cfg):
     layer = M.MoELayer(cfg, inp)
     q, s = oracle.quant_mx_bf16(bits(inp["w_d"]))
     assert np.array_equal(layer.mats["w_d"].cpu().numpy(), q)
-    assert np.array_equal(layer.scales["w_d"].cpu().numpy(), s)
+    assert np.array_equal(_image_to_rows(layer.scales["w_d"].cpu().numpy(), cfg.E, cfg.d, cfg.I), s)
 
 
 @pytest.mark.parametrize("cfg", MX, ids=MX_IDS)
@@ -113,7 +127,7 @@ def test_gemm_gateup_mx(cfg):
     assert M.read_device_status(layer.ws) == M.OK
     _, ooff, operm, _ = oracle.permute(ids.numpy(), cfg.E)
     ref = oracle.gateup(oracle_layer(cfg, inp), bits(inp["x"]), operm, ooff)  # FP64 h, pre-quantisation
-    gq, gs = hq.cpu().numpy(), hs.cpu().numpy()
+    gq, gs = hq.cpu().numpy(), _kbm_to_rows(hs.cpu().numpy(), R, cfg.I)
     X = np.repeat(_e8m0(gs), 32, axis=1)
     deq = oracle.e4m3_decode(gq) * X
     # one e4m3 rounding of the block (relative 2^-4, or 2^-10 X near zero) plus
