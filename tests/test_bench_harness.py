@@ -66,6 +66,9 @@ def test_algorithmic_work_of_the_gemms():
     assert b == 201 * 2 * 1536 * 4096 * 2 + 64 * 4096 * 2 + R * 1536 * 2
     f8, b8 = bench.gateup_algorithmic(CONFIGS["fp8"], 4096, n_active=256)
     assert b8 == 257 * 2 * 2048 * 6144 + 4096 * 6144 + (4096 * 9) * 2048
+    # MXFP8 adds one scale byte per 32 elements of weights, x and h
+    fm, bm = bench.gateup_algorithmic(CONFIGS["mxfp8"], 4096, n_active=256)
+    assert fm == f8 and bm == b8 + (257 * 2 * 2048 * 6144 + 4096 * 6144 + (4096 * 9) * 2048) // 32
     fd, bd = bench.down_algorithmic(cfg, cfg.T, n_active=200)
     assert fd == 2.0 * R * 1536 * 4096
     assert CONFIGS["prefill"].flops() == pytest.approx(2.82e12, rel=0.01)
