@@ -330,6 +330,20 @@ def run_ours(args, cfg: MoEConfig):
     if layer.device_status() != M.OK:
         raise RuntimeError("device status after warm-up: " + M.status_string(layer.device_status()))
 
+    # the timed steps: one moe_forward per step, replayed from a CUDA graph (the
+    # library's launches are capturable), so host launch gaps do not count
+    graph = None
+    if not args.no_graph:
+        y_ref = y.clone()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            M.forward(shape, layer.weights, x.view(torch.uint16), y.view(torch.uint16), layer.ws)
+        graph.replay()
+        torch.cuda.synchronize()
+        if not torch.equal(y, y_ref) or layer.device_status() != M.OK:
+            raise RuntimeError("graph replay does not reproduce the eager forward")
+        stream = torch.cuda.current_stream()
+
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clocks:
@@ -337,13 +351,22 @@ def run_ours(args, cfg: MoEConfig):
         torch.cuda.synchronize()
         t_start.record(stream)
         for i in range(args.steps):
-            M.forward_profiled(shape, layer.weights, x.view(torch.uint16), y.view(torch.uint16),
-                               layer.ws, events[i])
+            if graph is not None:
+                graph.replay()
+            else:
+                M.forward_profiled(shape, layer.weights, x.view(torch.uint16), y.view(torch.uint16),
+                                   layer.ws, events[i])
         t_end.record(stream)
         torch.cuda.synchronize()
         barrier()
     ms_total = t_start.elapsed_time(t_end)
     ms_total = max_over_ranks(ms_total, dev)
+    if graph is not None:
+        # per-stage times: the same steps again, eagerly, with the library's stage events
+        for i in range(args.steps):
+            M.forward_profiled(shape, layer.weights, x.view(torch.uint16), y.view(torch.uint16),
+                               layer.ws, events[i])
+        torch.cuda.synchronize()
     ms_step = ms_total / args.steps
     value = world * cfg.T * args.steps / (ms_total / 1e3)
 
@@ -423,7 +446,9 @@ def run_ours(args, cfg: MoEConfig):
                        "active_experts": n_active,
                        "l2": "no flush: the expert weights read each step "
                              f"({(gu_bytes + dn_bytes) / 1e9:.1f} GB) exceed the 126 MB L2",
-                       "parallelism": f"{world} independent replicas (tokens sharded, no collective)"},
+                       "parallelism": f"{world} independent replicas (tokens sharded, no collective)",
+                       "launch": ("one CUDA graph replay of moe_forward per step" if graph is not None
+                                  else "eager moe_forward_profiled launches")},
             "roofline": roof,
             "cpu_baseline": cpu,
             "e2e": e2e,
@@ -445,6 +470,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--config", default="decode", choices=sorted(CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-graph", action="store_true",
+                    help="time eager launches with stage events instead of CUDA graph replays")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--tokens", type=int, default=None,
                     help="override T (a smaller case of the same layer, e.g. for profiling)")
