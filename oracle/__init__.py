@@ -45,7 +45,8 @@ class _Layer(ctypes.Structure):
                 ("wdtype", ctypes.c_int), ("renorm", ctypes.c_int),
                 ("w_gu", ctypes.c_void_p), ("w_d", ctypes.c_void_p),
                 ("ws_gu", ctypes.c_void_p), ("ws_d", ctypes.c_void_p),
-                ("router_w", ctypes.c_void_p), ("router_bias", ctypes.c_void_p)]
+                ("router_w", ctypes.c_void_p), ("router_bias", ctypes.c_void_p),
+                ("act_sx", ctypes.c_float), ("act_sh", ctypes.c_float)]
 
 
 class _Out(ctypes.Structure):
@@ -80,6 +81,8 @@ def lib():
         L.orc_mx_scale_byte.argtypes = [ctypes.c_float]
         L.orc_quant_mx_rows.argtypes = [vp, i64, i32, vp, vp]
         L.orc_quant_mx_bf16.argtypes = [vp, i64, i32, i32, vp, vp]
+        L.orc_quant_fp8_tensor.argtypes = [vp, i64, i32, i32, vp, vp]
+        L.orc_quant_fp8_static.argtypes = [vp, i64, ctypes.c_float, vp]
         L.orc_gateup.argtypes = [ctypes.POINTER(_Layer), vp, vp, vp, vp]
         L.orc_down.argtypes = [ctypes.POINTER(_Layer), vp, vp, vp]
         L.orc_combine.argtypes = [ctypes.POINTER(_Layer), vp, vp, vp, vp]
@@ -188,6 +191,25 @@ def quant_fp8_rows(v: np.ndarray):
     return q, s
 
 
+def quant_fp8_tensor(W: np.ndarray):
+    """W: bf16 bits [..., rows, cols] -> (q uint8, s float32 [...]): one scale per matrix."""
+    W = _c(W, np.uint16)
+    rows, cols = W.shape[-2:]
+    batch = int(np.prod(W.shape[:-2])) if W.ndim > 2 else 1
+    q = np.empty(W.shape, np.uint8)
+    s = np.empty(W.shape[:-2] if W.ndim > 2 else (1,), np.float32)
+    lib().orc_quant_fp8_tensor(_p(W), batch, rows, cols, _p(q), _p(s))
+    return q, s
+
+
+def quant_fp8_static(v: np.ndarray, s: float) -> np.ndarray:
+    """v: float32 array, static scale s -> e4m3 codes of fp32(v / s), saturating."""
+    v = _c(v, np.float32)
+    q = np.empty(v.shape, np.uint8)
+    lib().orc_quant_fp8_static(_p(v), v.size, float(s), _p(q))
+    return q
+
+
 def e8m0_decode(b: int) -> float:
     return lib().orc_e8m0_decode(int(b))
 
@@ -232,7 +254,10 @@ class Layer:
     ws_gu: Optional[np.ndarray] = None   # bf16 bits [2Is, d]
     ws_d: Optional[np.ndarray] = None    # bf16 bits [d, Is]
     router_bias: Optional[np.ndarray] = None
-    wdtype: int = 0             # 0 bf16, 1 fp8 e4m3 with 128x128 block scales, 2 mxfp8
+    wdtype: int = 0             # 0 bf16, 1 fp8 e4m3 with 128x128 block scales, 2 mxfp8,
+                                # 3 fp8 per tensor (static activation scales act_sx, act_sh)
+    act_sx: float = 1.0
+    act_sh: float = 1.0
     renorm: bool = True
 
     def _struct(self, T: Optional[int] = None):
@@ -244,7 +269,8 @@ class Layer:
         k = self._keep
         return _Layer(self.T if T is None else T, self.d, self.E, self.k, self.I,
                       self.Is, self.wdtype, int(self.renorm),
-                      _p(k[0]), _p(k[1]), _p(k[2]), _p(k[3]), _p(k[4]), _p(k[5]))
+                      _p(k[0]), _p(k[1]), _p(k[2]), _p(k[3]), _p(k[4]), _p(k[5]),
+                      float(self.act_sx), float(self.act_sh))
 
     def rows(self, T: Optional[int] = None) -> int:
         T = self.T if T is None else T

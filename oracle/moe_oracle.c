@@ -117,6 +117,29 @@ static float quant_group(const float* v, int n, int64_t stride, uint8_t* q, int6
 }
 
 /* ---------------------------------------------------------------------------
+ * Per-tensor FP8: one scale per weight matrix; static activation scales
+ * ------------------------------------------------------------------------- */
+
+void orc_quant_fp8_tensor(const uint16_t* W, int64_t batch, int rows, int cols, uint8_t* q,
+                          float* s) {
+    int64_t n = (int64_t)rows * cols;
+    #pragma omp parallel for schedule(static)
+    for (int64_t b = 0; b < batch; ++b) {
+        float* f = (float*)malloc(sizeof(float) * (size_t)n);
+        for (int64_t i = 0; i < n; ++i) f[i] = (float)orc_bf16_decode(W[b * n + i]);
+        s[b] = quant_group(f, (int)n, 1, q + b * n, 1);
+        free(f);
+    }
+}
+
+void orc_quant_fp8_static(const float* v, int64_t n, float s, uint8_t* q) {
+    for (int64_t i = 0; i < n; ++i) {
+        volatile float t = v[i] / s;
+        q[i] = orc_e4m3_round((double)t);
+    }
+}
+
+/* ---------------------------------------------------------------------------
  * [MX] MXFP8: E8M0 shared scale per block of 32, e4m3 elements
  * ------------------------------------------------------------------------- */
 
@@ -303,6 +326,14 @@ static double* group_weights(const orc_layer* L, const uint16_t* W, int rows, in
         for (int64_t i = 0; i < n; ++i) out[i] = orc_bf16_decode(W[i]);
         return out;
     }
+    if (L->wdtype == 3) {
+        uint8_t* q = (uint8_t*)malloc((size_t)n);
+        float sw;
+        orc_quant_fp8_tensor(W, 1, rows, cols, q, &sw);
+        for (int64_t i = 0; i < n; ++i) out[i] = orc_e4m3_decode(q[i]) * (double)sw;
+        free(q);
+        return out;
+    }
     if (L->wdtype == 2) {
         uint8_t* q = (uint8_t*)malloc((size_t)n);
         uint8_t* sb = (uint8_t*)malloc((size_t)(n / 32 + 1));
@@ -327,7 +358,8 @@ static double* group_weights(const orc_layer* L, const uint16_t* W, int rows, in
 
 /* An activation row as the GEMM consumes it: BF16 values as they are, or for
  * FP8 layers the dequantised 1x128-group quantisation of the FP32 row. */
-static void activation_row(const orc_layer* L, const double* v, int n, double* out) {
+static void activation_row(const orc_layer* L, const double* v, int n, double* out,
+                           float static_scale) {
     if (L->wdtype == 0) {
         for (int i = 0; i < n; ++i) out[i] = v[i];
         return;
@@ -335,6 +367,13 @@ static void activation_row(const orc_layer* L, const double* v, int n, double* o
     float* f = (float*)malloc(sizeof(float) * (size_t)n);
     uint8_t* q = (uint8_t*)malloc((size_t)n);
     for (int i = 0; i < n; ++i) f[i] = (float)v[i];
+    if (L->wdtype == 3) {
+        orc_quant_fp8_static(f, n, static_scale, q);
+        for (int i = 0; i < n; ++i) out[i] = orc_e4m3_decode(q[i]) * (double)static_scale;
+        free(f);
+        free(q);
+        return;
+    }
     if (L->wdtype == 2) {
         uint8_t* sb = (uint8_t*)malloc((size_t)(n / 32 + 1));
         orc_quant_mx_rows(f, 1, n, q, sb);
@@ -374,7 +413,7 @@ void orc_gateup(const orc_layer* L, const uint16_t* x, const int32_t* perm,
         for (int64_t p = p0; p < p1; ++p) {
             int64_t t = g < L->E ? perm[p] / L->k : p - Tk;
             for (int i = 0; i < d; ++i) xr[i] = orc_bf16_decode(x[t * d + i]);
-            activation_row(L, xr, d, xa);
+            activation_row(L, xr, d, xa, L->act_sx);
             for (int n = 0; n < I; ++n) {
                 double gs = 0.0, us = 0.0;
                 const double* wg = W + (int64_t)n * d;
@@ -406,7 +445,7 @@ void orc_down(const orc_layer* L, const double* h, const int32_t* offsets, doubl
         double* W = group_weights(L, Wsrc, d, I);
         double* ha = (double*)malloc(sizeof(double) * (size_t)I);
         for (int64_t p = p0; p < p1; ++p) {
-            activation_row(L, h + p * hs, I, ha);
+            activation_row(L, h + p * hs, I, ha, L->act_sh);
             for (int n = 0; n < d; ++n) {
                 double acc = 0.0;
                 const double* w = W + (int64_t)n * I;

@@ -101,10 +101,22 @@ void orc_quant_mx_rows(const float* v, int64_t rows, int cols, uint8_t* q, uint8
 void orc_quant_mx_bf16(const uint16_t* W, int64_t batch, int rows, int cols, uint8_t* q,
                        uint8_t* s);
 
+/* [G8][HY] Per-tensor FP8 ("HPC-Ops ...", section HPC-Ops的主要功能, GroupGEMM FP8:
+ * per-tensor and block-wise FP8; "腾讯混元大模型：从多场景适配到高效部署的全栈技术解析",
+ * section 量化压缩技术实践 / FP8量化方案: static FP8 quantisation of weights and
+ * activations with scales precomputed from calibration data).  Weights: one
+ * scale per matrix, s = fp32(amax) / 448 (amax == 0 -> 1), q = e4m3(fp32(W/s));
+ * activations: a given static scale s, q = e4m3_rne_satfinite(fp32(v / s)). */
+void orc_quant_fp8_tensor(const uint16_t* W, int64_t batch, int rows, int cols, uint8_t* q,
+                          float* s);
+void orc_quant_fp8_static(const float* v, int64_t n, float s, uint8_t* q);
+
 typedef struct {
     int T, d, E, k, I, Is;     /* Is = 0: no shared expert                     */
     int wdtype;                /* 0: BF16 weights; 1: FP8 e4m3, 128x128 blocks;
-                                  2: MXFP8 (e4m3, E8M0 scale per 1x32 along K)
+                                  2: MXFP8 (e4m3, E8M0 scale per 1x32 along K);
+                                  3: FP8 per tensor (one scale per weight matrix,
+                                  static activation scales act_sx, act_sh)
                                   (the oracle quantises the BF16 weights itself) */
     int renorm;
     const uint16_t* w_gu;      /* bf16 [E][2I][d]: gate rows 0..I-1, up I..2I-1 */
@@ -113,6 +125,7 @@ typedef struct {
     const uint16_t* ws_d;      /* bf16 [d][Is] or NULL                          */
     const float* router_w;     /* f32 [E][d]; the oracle splits it itself       */
     const float* router_bias;  /* f32 [E] or NULL                               */
+    float act_sx, act_sh;      /* wdtype 3: static scales of x and of h         */
 } orc_layer;
 
 /* [FM][FP] Gate-Up stage over the permuted rows.  Rows p < T*k belong to the
