@@ -1,6 +1,6 @@
 """Benchmark of the fused MoE layer forward (one JSON line on rank 0).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config decode|prefill|fp8|mxfp8|skew|tiny]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config decode|prefill|fp8|mxfp8|fp8t|skew|tiny]
                     [--impl ours|reference] [--no-cpu-baseline]
 
 A step is one moe_forward over one batch of the workload's T tokens (router
@@ -45,7 +45,7 @@ from expert_layer_dual_b200.inputs import make_layer  # noqa: E402
 METRIC = "fused MoE layer tokens/s"
 UNIT = "tokens/s"
 # oracle token sample per step of the CPU baseline / reference arm
-CPU_SAMPLE = {"tiny": 16, "decode": 64, "prefill": 16, "fp8": 8, "mxfp8": 8, "skew": 16}
+CPU_SAMPLE = {"tiny": 16, "decode": 64, "prefill": 16, "fp8": 8, "mxfp8": 8, "fp8t": 8, "skew": 16}
 
 
 def cpu_sample(cfg: MoEConfig) -> int:
@@ -56,7 +56,8 @@ def describe(cfg: MoEConfig) -> str:
     s = f"{cfg.name}: T={cfg.T} d={cfg.d} E={cfg.E} top-{cfg.k}"
     s += f" + shared I={cfg.I}" if cfg.Is else f" I={cfg.I}"
     s += {0: ", BF16 weights", 1: ", FP8 e4m3 128x128 block-scaled weights",
-          2: ", MXFP8 (e4m3, E8M0 scale per 1x32) weights and activations"}[cfg.wdtype]
+          2: ", MXFP8 (e4m3, E8M0 scale per 1x32) weights and activations",
+          3: ", FP8 e4m3 per-tensor weight scales, static calibrated activation scales"}[cfg.wdtype]
     if cfg.zipf_bias:
         s += ", Zipf(1.2)-biased routing"
     return s
@@ -169,6 +170,7 @@ KERNEL_SOURCES = {
     "k_gateup_bf16": ["csrc/gemm_bf16.cu", "csrc/common.cuh", "csrc/grouped_common.cuh"],
     "k_gateup_fp8": ["csrc/gemm_fp8.cu", "csrc/common.cuh", "csrc/grouped_common.cuh"],
     "k_gateup_mx": ["csrc/gemm_mx.cu", "csrc/common.cuh", "csrc/grouped_common.cuh"],
+    "k_gateup_f8t": ["csrc/gemm_f8t.cu", "csrc/common.cuh", "csrc/grouped_common.cuh"],
 }
 
 
@@ -226,7 +228,21 @@ def _bits(t):
     return t.detach().contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
 
 
-def oracle_sample(cfg: MoEConfig, inp: dict, n_tokens: int):
+def oracle_static_scales(cfg: MoEConfig, inp: dict, n_tokens: int = 8):
+    """Static activation scales of a per-tensor FP8 layer for the oracle runs
+    without a GPU: amax(x) / 448 and amax(h) / 448 over the first n_tokens, h
+    from the oracle's own BF16 stages (the GPU layer calibrates the same way on
+    64 tokens with its BF16 kernels)."""
+    import oracle
+    L, xs = oracle_sample(MoEConfig(**{**cfg.__dict__, "wdtype": 0}), inp, n_tokens)
+    out = oracle.forward(L, xs)
+    h = oracle.gateup(L, xs, out["perm"], out["offsets"])
+    amax_x = float(np.abs(oracle.bf16_decode(xs)).max())
+    amax_h = float(np.abs(h).max())
+    return (amax_x / 448.0 if amax_x > 0 else 1.0, amax_h / 448.0 if amax_h > 0 else 1.0)
+
+
+def oracle_sample(cfg: MoEConfig, inp: dict, n_tokens: int, act=(1.0, 1.0)):
     """Host inputs of the oracle for the first n_tokens of the workload: x rows,
     the router weight and the experts the oracle's own routing selects."""
     import oracle
@@ -246,7 +262,8 @@ def oracle_sample(cfg: MoEConfig, inp: dict, n_tokens: int):
     L = oracle.Layer(T=n, d=cfg.d, E=cfg.E, k=cfg.k, I=cfg.I, Is=cfg.Is, w_gu=w_gu, w_d=w_d,
                      ws_gu=None if inp.get("ws_gu") is None else _bits(inp["ws_gu"]),
                      ws_d=None if inp.get("ws_d") is None else _bits(inp["ws_d"]),
-                     router_w=rw, router_bias=bias, wdtype=cfg.wdtype, renorm=cfg.renorm)
+                     router_w=rw, router_bias=bias, wdtype=cfg.wdtype, renorm=cfg.renorm,
+                     act_sx=act[0], act_sh=act[1])
     return L, xs
 
 
@@ -272,7 +289,8 @@ def run_reference(args, cfg: MoEConfig):
     t1 = oracle_times(L1, x1, 1)
     budget = 150.0 / (args.warmup + args.steps)
     n = int(max(1, min(cpu_sample(cfg), budget / max(t1[0], 1e-3))))
-    L, xs = oracle_sample(cfg, inp, n)
+    act = oracle_static_scales(cfg, inp) if cfg.wdtype == 3 else (1.0, 1.0)
+    L, xs = oracle_sample(cfg, inp, n, act)
     n = xs.shape[0]
     times, cores = oracle_times(L, xs, args.warmup + args.steps), oracle.num_threads()
     timed = times[args.warmup:]
@@ -392,7 +410,7 @@ def run_ours(args, cfg: MoEConfig):
         roof = {"bound": "tensor", "achieved": gu_flops / (gu_ms / 1e3) / 1e12, "peak": peak,
                 "unit": "TFLOP/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["kernel"] = "k_gateup_" + {0: "bf16", 1: "fp8", 2: "mx"}[cfg.wdtype]
+    roof["kernel"] = "k_gateup_" + {0: "bf16", 1: "fp8", 2: "mx", 3: "f8t"}[cfg.wdtype]
     roof["peak_source"] = (f"{peak_kind} MEASURED_PEAKS.json "
                            + ("hbm_gbs" if roof["bound"] == "hbm" else "bf16_tflops (burst: the timed loop is well under a second)"
                               + (" x2 (e4m3 nominal ratio)" if cfg.wdtype else "")))
@@ -424,7 +442,7 @@ def run_ours(args, cfg: MoEConfig):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
-        L, xs = oracle_sample(cfg, inp, cpu_sample(cfg))
+        L, xs = oracle_sample(cfg, inp, cpu_sample(cfg), layer.act_scales)
         n, cores = xs.shape[0], oracle.num_threads()
         times = oracle_times(L, xs, 1)
         # repeat up to about 10 s of CPU work (at most 30 s)
@@ -440,7 +458,7 @@ def run_ours(args, cfg: MoEConfig):
         out = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": {0: "bf16", 1: "f8e4m3", 2: "mxf8e4m3"}[cfg.wdtype],
+            "scaling": "weak", "vs_baseline": None, "dtype": {0: "bf16", 1: "f8e4m3", 2: "mxf8e4m3", 3: "f8e4m3"}[cfg.wdtype],
             "data": "synthetic",
             "config": {"workload": describe(cfg), "tokens_per_gpu": cfg.T,
                        "active_experts": n_active,

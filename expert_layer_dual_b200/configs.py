@@ -21,7 +21,8 @@ class MoEConfig:
     k: int
     I: int
     Is: int = 0
-    wdtype: int = 0          # 0 bf16 weights, 1 fp8 e4m3 with 128x128 block scales, 2 MXFP8
+    wdtype: int = 0          # 0 bf16 weights, 1 fp8 e4m3 with 128x128 block scales, 2 MXFP8,
+                             # 3 FP8 per tensor with static (calibrated) activation scales
     zipf_bias: bool = False  # skewed routing: per-expert Zipf(s=1.2) logit bias
     seed: int = 0
     renorm: bool = True
@@ -54,6 +55,10 @@ CONFIGS = {
     # the FP8 layer in MXFP8: e4m3 weights and activations, E8M0 scale per 1x32
     # (the MXFP8 weight format of the same page, section 实现拆解 item 4)
     "mxfp8": MoEConfig("mxfp8", T=4096, d=6144, E=256, k=8, I=2048, Is=2048, wdtype=2, seed=3),
+    # the FP8 layer with per-tensor scales: one scale per weight matrix, static
+    # activation scales ("HPC-Ops" GroupGEMM FP8 per-tensor; the Hunyuan page's
+    # static FP8 scheme)
+    "fp8t": MoEConfig("fp8t", T=4096, d=6144, E=256, k=8, I=2048, Is=2048, wdtype=3, seed=3),
     # skewed routing: 16384 tokens, Zipf-biased router logits
     "skew": MoEConfig("skew", T=16384, d=4096, E=256, k=8, I=1536, Is=1536,
                       zipf_bias=True, seed=4),

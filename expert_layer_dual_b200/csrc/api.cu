@@ -104,6 +104,10 @@ WsLayout ws_layout(const moe_shape& s) {
         L.xs = take(R * (d / 128) * 4);
         L.h = take(R * I);
         L.hs = take(R * (I / 128) * 4);
+    } else if (s.wdtype == MOE_WDTYPE_FP8_TENSOR) {
+        L.xq = take(R * d);                               // e4m3 x, permuted rows
+        L.xs = L.hs = 0;                                  // static scales
+        L.h = take(R * I);
     } else if (s.wdtype == MOE_WDTYPE_MXFP8) {
         L.xq = take(R * d);                               // e4m3 x, permuted rows
         L.xs = take(R * (d / 32));                        // E8M0 byte per 1x32 block
@@ -133,7 +137,7 @@ moe_status check_shape(const moe_shape* s) {
         return MOE_ERR_UNSUPPORTED;
     if (s->I_shared != 0 && s->I_shared != s->I) return MOE_ERR_UNSUPPORTED;
     if (s->wdtype != MOE_WDTYPE_BF16 && s->wdtype != MOE_WDTYPE_FP8_BLOCK128 &&
-        s->wdtype != MOE_WDTYPE_MXFP8)
+        s->wdtype != MOE_WDTYPE_MXFP8 && s->wdtype != MOE_WDTYPE_FP8_TENSOR)
         return MOE_ERR_UNSUPPORTED;
     if ((int64_t)s->T * s->k + s->T >= (int64_t)1 << 31) return MOE_ERR_UNSUPPORTED;
     if ((int64_t)s->E * 2 * s->I >= (int64_t)1 << 31 || (int64_t)s->E * s->d >= (int64_t)1 << 31)
@@ -153,6 +157,10 @@ moe_status check_weights(const moe_shape* s, const moe_weights* w, bool need_gat
                       (sh && (w->ws_d == nullptr || (fp8 && w->ws_d_scale == nullptr)))))
         return MOE_ERR_INVALID_ARG;
     if (need_router && (w->router_hi == nullptr || w->router_lo == nullptr))
+        return MOE_ERR_INVALID_ARG;
+    if (s->wdtype == MOE_WDTYPE_FP8_TENSOR &&
+        (!(w->act_scale_x > 0.0f) || !(w->act_scale_h > 0.0f) || !isfinite(w->act_scale_x) ||
+         !isfinite(w->act_scale_h)))
         return MOE_ERR_INVALID_ARG;
     return MOE_OK;
 }
@@ -200,6 +208,12 @@ moe_status run_gateup(const moe_shape* s, const moe_weights* w, const void* x, c
                                               static_cast<const uint16_t*>(w->w_gu),
                                               static_cast<const uint16_t*>(w->ws_gu),
                                               static_cast<uint16_t*>(h), st));
+    if (s->wdtype == MOE_WDTYPE_FP8_TENSOR)
+        return cuda_status(launch_gateup_f8t(
+            a, static_cast<const uint8_t*>(x), w->act_scale_x, w->act_scale_h,
+            static_cast<const uint8_t*>(w->w_gu), static_cast<const float*>(w->w_gu_scale),
+            static_cast<const uint8_t*>(w->ws_gu), static_cast<const float*>(w->ws_gu_scale),
+            static_cast<uint8_t*>(h), st));
     if (s->wdtype == MOE_WDTYPE_MXFP8)
         return cuda_status(launch_gateup_mx(
             a, static_cast<const uint8_t*>(x), static_cast<const uint8_t*>(xs),
@@ -221,6 +235,11 @@ moe_status run_down(const moe_shape* s, const moe_weights* w, const void* h, con
                                                              : launch_down_bf16)(
             a, static_cast<const uint16_t*>(h), static_cast<const uint16_t*>(w->w_d),
             static_cast<const uint16_t*>(w->ws_d), o, st));
+    if (s->wdtype == MOE_WDTYPE_FP8_TENSOR)
+        return cuda_status(launch_down_f8t(
+            a, static_cast<const uint8_t*>(h), w->act_scale_h, static_cast<const uint8_t*>(w->w_d),
+            static_cast<const float*>(w->w_d_scale), static_cast<const uint8_t*>(w->ws_d),
+            static_cast<const float*>(w->ws_d_scale), o, st));
     if (s->wdtype == MOE_WDTYPE_MXFP8)
         return cuda_status(launch_down_mx(
             a, static_cast<const uint8_t*>(h), static_cast<const uint8_t*>(hs),
@@ -253,6 +272,7 @@ moe_status forward_device(const moe_shape* s, const moe_weights* w, const uint16
     int32_t* seg = at<int32_t>(ws, L.seg);
     const bool fp8 = s->wdtype == MOE_WDTYPE_FP8_BLOCK128;
     const bool mx = s->wdtype == MOE_WDTYPE_MXFP8;
+    const bool f8t = s->wdtype == MOE_WDTYPE_FP8_TENSOR;
     moe_status r;
     if (cudaMemsetAsync(status, 0, sizeof(int32_t), st) != cudaSuccess) return MOE_ERR_CUDA;
     if (!mark(0)) return MOE_ERR_CUDA;
@@ -284,6 +304,14 @@ moe_status forward_device(const moe_shape* s, const moe_weights* w, const uint16
     if (!mark(3)) return MOE_ERR_CUDA;
     const void* a_in = x;
     const void* a_scale = nullptr;
+    if (f8t) {
+        const int64_t R = (int64_t)s->T * s->k + (s->I_shared > 0 ? s->T : 0);
+        if ((r = cuda_status(launch_quant_act_fp8_static(x, perm, s->T, s->k, R, s->d,
+                                                         w->act_scale_x, at<uint8_t>(ws, L.xq),
+                                                         st))) != MOE_OK)
+            return r;
+        a_in = at<uint8_t>(ws, L.xq);
+    }
     if (mx) {
         if ((r = cuda_status(launch_quant_mx_permuted(x, perm, s->T, s->k, s->I_shared > 0 ? 1 : 0,
                                                       s->d, at<uint8_t>(ws, L.xq),
@@ -367,6 +395,40 @@ moe_status moe_quantize_act_fp8(const uint16_t* x, int64_t rows, int32_t cols, u
     if (x == nullptr || q == nullptr || scale == nullptr) return MOE_ERR_INVALID_ARG;
     if (!device_ok()) return MOE_ERR_UNSUPPORTED;
     return cuda_status(launch_quant_act_fp8(x, rows, cols, q, scale, as_stream(stream)));
+}
+
+moe_status moe_quantize_weights_fp8_tensor(const uint16_t* W, int64_t batch, int32_t rows,
+                                           int32_t cols, uint8_t* q, float* scale, void* stream) {
+    if (batch < 0 || rows < 0 || cols < 0) return MOE_ERR_INVALID_ARG;
+    if (cols % 8 != 0) return MOE_ERR_UNSUPPORTED;
+    if (batch * rows * (int64_t)cols == 0) return MOE_OK;
+    if (W == nullptr || q == nullptr || scale == nullptr) return MOE_ERR_INVALID_ARG;
+    if (batch >= 65536) return MOE_ERR_UNSUPPORTED;
+    if (!device_ok()) return MOE_ERR_UNSUPPORTED;
+    return cuda_status(launch_quant_weights_fp8_tensor(W, batch, rows, cols, q, scale, as_stream(stream)));
+}
+
+moe_status moe_quantize_act_fp8_static(const uint16_t* x, int64_t rows, int32_t cols, float scale,
+                                       uint8_t* q, void* stream) {
+    if (rows < 0 || cols <= 0 || !(scale > 0.0f) || !isfinite(scale)) return MOE_ERR_INVALID_ARG;
+    if (cols % 8 != 0) return MOE_ERR_UNSUPPORTED;
+    if (rows == 0) return MOE_OK;
+    if (x == nullptr || q == nullptr) return MOE_ERR_INVALID_ARG;
+    if (!device_ok()) return MOE_ERR_UNSUPPORTED;
+    return cuda_status(launch_quant_act_fp8_static(x, nullptr, 0, 1, rows, cols, scale, q,
+                                                   as_stream(stream)));
+}
+
+moe_status moe_quantize_act_fp8_static_permuted(const uint16_t* x, const int32_t* perm, int32_t T,
+                                                int32_t k, int32_t with_shared, int32_t d,
+                                                float scale, uint8_t* q, void* stream) {
+    if (T < 0 || k <= 0 || d <= 0 || !(scale > 0.0f) || !isfinite(scale)) return MOE_ERR_INVALID_ARG;
+    if (d % 8 != 0 || (int64_t)T * k + T >= ((int64_t)1 << 31)) return MOE_ERR_UNSUPPORTED;
+    if (T == 0) return MOE_OK;
+    if (x == nullptr || perm == nullptr || q == nullptr) return MOE_ERR_INVALID_ARG;
+    if (!device_ok()) return MOE_ERR_UNSUPPORTED;
+    const int64_t R = (int64_t)T * k + (with_shared ? T : 0);
+    return cuda_status(launch_quant_act_fp8_static(x, perm, T, k, R, d, scale, q, as_stream(stream)));
 }
 
 moe_status moe_quantize_weights_mxfp8(const uint16_t* W, int64_t batch, int32_t rows, int32_t cols,
@@ -459,9 +521,10 @@ moe_status moe_gemm_gateup(const moe_shape* shape, const moe_weights* weights, c
     if (r != MOE_OK) return r;
     if ((r = check_weights(shape, weights, true, false, false)) != MOE_OK) return r;
     if (shape->T == 0) return MOE_OK;
-    const bool fp8 = shape->wdtype != MOE_WDTYPE_BF16;  // FP8 or MXFP8: permuted e4m3 rows
+    const bool fp8 = shape->wdtype != MOE_WDTYPE_BF16;  // permuted e4m3 rows
+    const bool scaled = fp8 && shape->wdtype != MOE_WDTYPE_FP8_TENSOR;  // per-row scales
     if (x == nullptr || offsets == nullptr || h == nullptr || (!fp8 && perm == nullptr) ||
-        (fp8 && (x_scale == nullptr || h_scale == nullptr)))
+        (scaled && (x_scale == nullptr || h_scale == nullptr)))
         return MOE_ERR_INVALID_ARG;
     if ((r = check_ws(ws, ws_bytes, kWsHeader)) != MOE_OK) return r;
     if (!device_ok()) return MOE_ERR_UNSUPPORTED;
@@ -478,8 +541,8 @@ moe_status moe_gemm_down(const moe_shape* shape, const moe_weights* weights, con
     if (r != MOE_OK) return r;
     if ((r = check_weights(shape, weights, false, true, false)) != MOE_OK) return r;
     if (shape->T == 0) return MOE_OK;
-    const bool fp8 = shape->wdtype != MOE_WDTYPE_BF16;
-    if (h == nullptr || offsets == nullptr || o == nullptr || (fp8 && h_scale == nullptr))
+    const bool scaled = shape->wdtype == MOE_WDTYPE_FP8_BLOCK128 || shape->wdtype == MOE_WDTYPE_MXFP8;
+    if (h == nullptr || offsets == nullptr || o == nullptr || (scaled && h_scale == nullptr))
         return MOE_ERR_INVALID_ARG;
     if ((r = check_ws(ws, ws_bytes, kWsHeader)) != MOE_OK) return r;
     if (!device_ok()) return MOE_ERR_UNSUPPORTED;

@@ -55,6 +55,14 @@ cudaError_t launch_quant_mx_weights(const uint16_t* W, int64_t batch, int rows, 
 cudaError_t launch_quant_mx_permuted(const uint16_t* x, const int32_t* perm, int T, int k,
                                      int has_shared, int cols, uint8_t* q, uint8_t* scale,
                                      cudaStream_t s);
+// Per-tensor FP8: weights with one scale per matrix (scale [batch]);
+// activations with a static scale, rows as they are (perm NULL) or in the
+// permuted order of the grouped GEMMs (rows = T*k + shared T).
+cudaError_t launch_quant_weights_fp8_tensor(const uint16_t* W, int64_t batch, int rows, int cols,
+                                            uint8_t* q, float* scale, cudaStream_t s);
+cudaError_t launch_quant_act_fp8_static(const uint16_t* x, const int32_t* perm, int T, int k,
+                                        int64_t rows, int cols, float scale, uint8_t* q,
+                                        cudaStream_t s);
 cudaError_t launch_selftest_timeout(int32_t* status, uint64_t limit_ns, cudaStream_t s);
 
 // ---- router.cu (tcgen05 dual-BF16 GEMM)
@@ -105,6 +113,14 @@ cudaError_t launch_gateup_mx(const GroupedGemmArgs& a, const uint8_t* xq, const 
 cudaError_t launch_down_mx(const GroupedGemmArgs& a, const uint8_t* hq, const uint8_t* hs,
                            const uint8_t* w_d, const uint8_t* w_d_s, const uint8_t* ws_d,
                            const uint8_t* ws_d_s, float* o, cudaStream_t s);
+
+// ---- gemm_f8t.cu (tcgen05 grouped GEMMs, per-tensor FP8, static activation scales)
+cudaError_t launch_gateup_f8t(const GroupedGemmArgs& a, const uint8_t* xq, float sx, float sh,
+                              const uint8_t* w_gu, const float* w_gu_s, const uint8_t* ws_gu,
+                              const float* ws_gu_s, uint8_t* hq, cudaStream_t s);
+cudaError_t launch_down_f8t(const GroupedGemmArgs& a, const uint8_t* hq, float sh,
+                            const uint8_t* w_d, const float* w_d_s, const uint8_t* ws_d,
+                            const float* ws_d_s, float* o, cudaStream_t s);
 
 // ---- tensor maps (api.cu)
 // 2-D row-major tensor [rows][cols] of `elem_bytes`-sized elements, box

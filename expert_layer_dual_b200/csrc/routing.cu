@@ -531,6 +531,96 @@ cudaError_t launch_quant_mx_permuted(const uint16_t* x, const int32_t* perm, int
     return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------------------
+// Per-tensor FP8.  Weights: one scale per matrix, s = fp32(amax) / 448
+// (amax == 0 -> 1), q = e4m3(fp32(W / s)); computed in three stream-ordered
+// passes -- the matrix amax (an atomicMax on the FP32 bits, which order like
+// the values for non-negative floats) into `scale`, the codes, then `scale`
+// rewritten from amax to s.  Activations: a static scale s given by the
+// caller, q = e4m3(fp32(v / s)), saturating.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+    k_amax_matrices(const uint16_t* __restrict__ W, int64_t per, uint32_t* __restrict__ amax_bits) {
+    const int64_t m = blockIdx.y;
+    const uint16_t* src = W + m * per;
+    float amax = 0.0f;
+    for (int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 8; i < per;
+         i += (int64_t)gridDim.x * blockDim.x * 8) {
+        float f[8];
+        bf16x8_to_f32(*reinterpret_cast<const uint4*>(src + i), f);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(f[j]));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    if ((threadIdx.x & 31) == 0) atomicMax(amax_bits + m, __float_as_uint(amax));
+}
+
+__global__ void __launch_bounds__(256)
+    k_quant_matrices(const uint16_t* __restrict__ W, int64_t per, const uint32_t* __restrict__ amax_bits,
+                     uint8_t* __restrict__ q) {
+    const int64_t m = blockIdx.y;
+    const float s = group_scale(__uint_as_float(amax_bits[m]));
+    for (int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 8; i < per;
+         i += (int64_t)gridDim.x * blockDim.x * 8) {
+        float f[8];
+        bf16x8_to_f32(*reinterpret_cast<const uint4*>(W + m * per + i), f);
+        uint2 o;
+        o.x = quant4_e4m3(f[0], f[1], f[2], f[3], s);
+        o.y = quant4_e4m3(f[4], f[5], f[6], f[7], s);
+        *reinterpret_cast<uint2*>(q + m * per + i) = o;
+    }
+}
+
+__global__ void k_scale_from_amax(float* __restrict__ scale, int64_t batch) {
+    const int64_t m = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    if (m < batch) scale[m] = group_scale(scale[m]);
+}
+
+cudaError_t launch_quant_weights_fp8_tensor(const uint16_t* W, int64_t batch, int rows, int cols,
+                                            uint8_t* q, float* scale, cudaStream_t s) {
+    const int64_t per = (int64_t)rows * cols;
+    if (batch == 0 || per == 0) return cudaSuccess;
+    cudaError_t e = cudaMemsetAsync(scale, 0, sizeof(float) * (size_t)batch, s);
+    if (e != cudaSuccess) return e;
+    const int64_t want = (per / 8 + 255) / 256;
+    const unsigned bx = (unsigned)(want < 1024 ? want : 1024);
+    const dim3 grid(bx, (unsigned)batch);
+    k_amax_matrices<<<grid, 256, 0, s>>>(W, per, reinterpret_cast<uint32_t*>(scale));
+    k_quant_matrices<<<grid, 256, 0, s>>>(W, per, reinterpret_cast<const uint32_t*>(scale), q);
+    k_scale_from_amax<<<(unsigned)((batch + 255) / 256), 256, 0, s>>>(scale, batch);
+    return cudaGetLastError();
+}
+
+// One warp per row, 8 values (16 bytes in, 8 bytes out) per lane per step.
+__global__ void __launch_bounds__(256)
+    k_quant_static(const uint16_t* __restrict__ x, const int32_t* __restrict__ perm, int T, int k,
+                   int64_t rows, int cols, float s, uint8_t* __restrict__ q) {
+    const int64_t p = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+    if (p >= rows) return;
+    const int lane = threadIdx.x & 31;
+    const int64_t Tk = (int64_t)T * k;
+    const int64_t src_row = perm == nullptr ? p : (p < Tk ? (int64_t)(perm[p] / k) : p - Tk);
+    const uint16_t* src = x + src_row * cols;
+    uint8_t* dst = q + p * cols;
+    for (int c = lane * 8; c < cols; c += 256) {
+        float f[8];
+        bf16x8_to_f32(*reinterpret_cast<const uint4*>(src + c), f);
+        uint2 o;
+        o.x = quant4_e4m3(f[0], f[1], f[2], f[3], s);
+        o.y = quant4_e4m3(f[4], f[5], f[6], f[7], s);
+        *reinterpret_cast<uint2*>(dst + c) = o;
+    }
+}
+
+cudaError_t launch_quant_act_fp8_static(const uint16_t* x, const int32_t* perm, int T, int k,
+                                        int64_t rows, int cols, float scale, uint8_t* q,
+                                        cudaStream_t s) {
+    if (rows == 0) return cudaSuccess;
+    k_quant_static<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(x, perm, T, k, rows, cols, scale, q);
+    return cudaGetLastError();
+}
+
 // one block of 256 threads per 128x128 block; thread = half a row (64 values)
 __global__ void __launch_bounds__(256)
     k_quant_w(const uint16_t* __restrict__ W, int rows, int cols, uint8_t* __restrict__ q,

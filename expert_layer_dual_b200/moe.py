@@ -28,12 +28,13 @@ if not os.path.exists(LIB_PATH):
 _lib = ctypes.CDLL(LIB_PATH)
 
 OK, INVALID_ARG, UNSUPPORTED, CUDA_ERROR, WORKSPACE_TOO_SMALL, DEVICE_TIMEOUT, DEVICE_BAD_INDEX = range(7)
-WDTYPE_BF16, WDTYPE_FP8_BLOCK128, WDTYPE_MXFP8 = 0, 1, 2
+WDTYPE_BF16, WDTYPE_FP8_BLOCK128, WDTYPE_MXFP8, WDTYPE_FP8_TENSOR = 0, 1, 2, 3
 
 EXPORTS = ["moe_status_string", "moe_workspace_bytes", "moe_permute_workspace_bytes",
            "moe_router_split", "moe_quantize_weights_fp8", "moe_quantize_act_fp8",
            "moe_quantize_act_fp8_permuted", "moe_quantize_weights_mxfp8", "moe_quantize_act_mxfp8",
-           "moe_quantize_act_mxfp8_permuted",
+           "moe_quantize_act_mxfp8_permuted", "moe_quantize_weights_fp8_tensor",
+           "moe_quantize_act_fp8_static", "moe_quantize_act_fp8_static_permuted",
            "moe_router_logits", "moe_route_topk", "moe_permute", "moe_permute_noalloc",
            "moe_gemm_gateup",
            "moe_gemm_down", "moe_combine", "moe_forward", "moe_forward_profiled", "moe_forward_host",
@@ -49,7 +50,8 @@ class moe_shape(ctypes.Structure):
 class moe_weights(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
                 ("w_gu", "w_d", "w_gu_scale", "w_d_scale", "ws_gu", "ws_d", "ws_gu_scale",
-                 "ws_d_scale", "router_hi", "router_lo", "router_bias")]
+                 "ws_d_scale", "router_hi", "router_lo", "router_bias")] + \
+               [("act_scale_x", ctypes.c_float), ("act_scale_h", ctypes.c_float)]
 
 
 _vp, _i32, _i64, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
@@ -63,6 +65,10 @@ _sig = {
     "moe_quantize_act_fp8": (_i32, [_vp, _i64, _i32, _vp, _vp, _vp]),
     "moe_quantize_act_fp8_permuted": (_i32, [_vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
     "moe_quantize_weights_mxfp8": (_i32, [_vp, _i64, _i32, _i32, _vp, _vp, _vp]),
+    "moe_quantize_weights_fp8_tensor": (_i32, [_vp, _i64, _i32, _i32, _vp, _vp, _vp]),
+    "moe_quantize_act_fp8_static": (_i32, [_vp, _i64, _i32, ctypes.c_float, _vp, _vp]),
+    "moe_quantize_act_fp8_static_permuted": (_i32, [_vp, _vp, _i32, _i32, _i32, _i32, ctypes.c_float,
+                                                    _vp, _vp]),
     "moe_quantize_act_mxfp8": (_i32, [_vp, _i64, _i32, _vp, _vp, _vp]),
     "moe_quantize_act_mxfp8_permuted": (_i32, [_vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
     "moe_router_logits": (_i32, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _vp]),
@@ -149,6 +155,27 @@ def quantize_weights_mxfp8(W, q, scale, stream=None):
     batch = W.numel() // (rows * cols)
     _check(_lib.moe_quantize_weights_mxfp8(_p(W), batch, rows, cols, _p(q), _p(scale), _stream(stream)),
            "moe_quantize_weights_mxfp8")
+
+
+def quantize_weights_fp8_tensor(W, q, scale, stream=None):
+    """W bf16 bits [..., rows, cols] -> q e4m3 (same shape), scale float32 [...] (one per matrix)."""
+    rows, cols = W.shape[-2:]
+    batch = W.numel() // (rows * cols)
+    _check(_lib.moe_quantize_weights_fp8_tensor(_p(W), batch, rows, cols, _p(q), _p(scale),
+                                                _stream(stream)), "moe_quantize_weights_fp8_tensor")
+
+
+def quantize_act_fp8_static(x, scale, q, stream=None):
+    rows, cols = x.shape
+    _check(_lib.moe_quantize_act_fp8_static(_p(x), rows, cols, float(scale), _p(q), _stream(stream)),
+           "moe_quantize_act_fp8_static")
+
+
+def quantize_act_fp8_static_permuted(x, perm, k, with_shared, scale, q, stream=None):
+    T, d = x.shape
+    _check(_lib.moe_quantize_act_fp8_static_permuted(_p(x), _p(perm), T, k, int(with_shared), d,
+                                                     float(scale), _p(q), _stream(stream)),
+           "moe_quantize_act_fp8_static_permuted")
 
 
 def quantize_act_mxfp8(x, q, scale, stream=None):
@@ -281,6 +308,11 @@ class MoELayer:
                                 dtype=torch.float32, device=dev)
                 quantize_weights_fp8(t.view(torch.uint16), q, s)
                 self.mats[name], self.scales[name] = q, s
+            elif cfg.wdtype == WDTYPE_FP8_TENSOR:
+                q = torch.empty(t.shape, dtype=torch.uint8, device=dev)
+                s = torch.empty(t.shape[:-2] if t.dim() > 2 else (1,), dtype=torch.float32, device=dev)
+                quantize_weights_fp8_tensor(t.view(torch.uint16), q, s)
+                self.mats[name], self.scales[name] = q, s
             elif cfg.wdtype == WDTYPE_MXFP8:
                 q = torch.empty(t.shape, dtype=torch.uint8, device=dev)
                 s = torch.empty(t.shape[:-1] + (t.shape[-1] // 32,), dtype=torch.uint8, device=dev)
@@ -288,14 +320,54 @@ class MoELayer:
                 self.mats[name], self.scales[name] = q, s
             else:
                 self.mats[name], self.scales[name] = t.view(torch.uint16), None
+        self.act_scales = (1.0, 1.0)
+        if cfg.wdtype == WDTYPE_FP8_TENSOR:
+            self.act_scales = self._calibrate_static_scales(cfg, inputs, dev)
         self.weights = moe_weights(*[_p(v) for v in (
             self.mats["w_gu"], self.mats["w_d"], self.scales["w_gu"], self.scales["w_d"],
             self.mats["ws_gu"], self.mats["ws_d"], self.scales["ws_gu"], self.scales["ws_d"],
-            self.router_hi, self.router_lo, self.router_bias)])
+            self.router_hi, self.router_lo, self.router_bias)], *self.act_scales)
         nbytes = workspace_bytes(shape_of(cfg, self.max_tokens))
         if nbytes == 0:
             raise MoEError(UNSUPPORTED, "moe_workspace_bytes")
         self.ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+
+    CALIBRATION_TOKENS = 64
+
+    def _calibrate_static_scales(self, cfg: MoEConfig, inputs: dict, dev):
+        """Static activation scales of the per-tensor FP8 layer, calibrated on the
+        first CALIBRATION_TOKENS tokens of the input: amax(x) / 448 and amax(h) / 448,
+        h the gate-up output of those tokens computed with the BF16 weights by this
+        library's own stages (router, top-k, permute, BF16 gate-up)."""
+        x = inputs["x"][: self.CALIBRATION_TOKENS].to(dev, torch.bfloat16).contiguous()
+        T, E, k = x.shape[0], cfg.E, cfg.k
+        amax_x = float(x.float().abs().max().item())
+        bf = {n: (None if inputs.get(n) is None else inputs[n].to(dev, torch.bfloat16).contiguous())
+              for n in ("w_gu", "w_d", "ws_gu", "ws_d")}
+        w16 = moe_weights(_p(bf["w_gu"]), _p(bf["w_d"]), None, None, _p(bf["ws_gu"]), _p(bf["ws_d"]),
+                          None, None, _p(self.router_hi), _p(self.router_lo), _p(self.router_bias),
+                          1.0, 1.0)
+        shape16 = moe_shape(T, cfg.d, E, k, cfg.I, cfg.Is, WDTYPE_BF16, int(cfg.renorm))
+        logits = torch.empty((T, E), dtype=torch.float32, device=dev)
+        router_logits(x.view(torch.uint16), self.router_hi, self.router_lo, self.router_bias, logits)
+        ids = torch.empty((T, k), dtype=torch.int32, device=dev)
+        wts = torch.empty((T, k), dtype=torch.float32, device=dev)
+        route_topk(logits, k, int(cfg.renorm), ids, wts)
+        counts = torch.empty(E, dtype=torch.int32, device=dev)
+        offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+        perm = torch.empty(T * k, dtype=torch.int32, device=dev)
+        inv = torch.empty(T * k, dtype=torch.int32, device=dev)
+        pws = torch.empty(permute_workspace_bytes(T, E, k), dtype=torch.uint8, device=dev)
+        permute(ids, E, counts, offsets, perm, inv, pws)
+        R = T * k + (T if cfg.Is else 0)
+        h = torch.empty((R, cfg.I), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(4096, dtype=torch.uint8, device=dev)
+        gemm_gateup(shape16, w16, x.view(torch.uint16), None, perm, offsets, h.view(torch.uint16),
+                    None, ws)
+        amax_h = float(h.float().abs().max().item())
+        sx = amax_x / 448.0 if amax_x > 0 else 1.0
+        sh = amax_h / 448.0 if amax_h > 0 else 1.0
+        return (sx, sh)
 
     def shape(self, T: int) -> moe_shape:
         if T > self.max_tokens:

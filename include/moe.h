@@ -70,6 +70,9 @@ typedef int32_t moe_status;
 #define MOE_WDTYPE_MXFP8 2          /* MXFP8: weights and activations e4m3 with one
                                        E8M0 (power-of-two) scale byte per 1x32
                                        block along K; native block-scaled MMA      */
+#define MOE_WDTYPE_FP8_TENSOR 3     /* FP8 per tensor: e4m3 weights with one f32
+                                       scale per matrix; activations e4m3 with
+                                       static (calibrated) scales act_scale_x/h    */
 
 /* Layer shape.  T tokens of hidden size d; E routed experts of intermediate
  * size I, top-k routing; I_shared = 0 (no shared expert) or I. */
@@ -86,6 +89,9 @@ typedef struct moe_shape {
  *   wdtype 2: w_gu_scale, w_d_scale uint8 E8M0, one per 1x32 block along K, in
  *             the per-matrix image of moe_quantize_weights_mxfp8 (E matrices of
  *             2I x d, resp. d x I)
+ *   wdtype 3: w_gu_scale, w_d_scale float [E] (one per matrix), ws_*_scale float
+ *             [1]; act_scale_x, act_scale_h the static scales of x and of h
+ *             (finite, > 0; q = e4m3_rne_satfinite(fp32(v / s)))
  *   ws_gu [2I][d], ws_d [d][I], ws_*_scale likewise  (when I_shared > 0)
  *   router_hi, router_lo [E][d] bf16 from moe_router_split; router_bias [E]
  *   or NULL (added to the logits, so it steers both selection and weights). */
@@ -101,6 +107,8 @@ typedef struct moe_weights {
     const uint16_t* router_hi;
     const uint16_t* router_lo;
     const float* router_bias;
+    float act_scale_x;        /* wdtype 3 only */
+    float act_scale_h;        /* wdtype 3 only */
 } moe_weights;
 
 /* Human-readable name of a status code (static storage). */
@@ -158,6 +166,25 @@ moe_status moe_quantize_act_mxfp8(const uint16_t* x, int64_t rows, int32_t cols,
 moe_status moe_quantize_act_mxfp8_permuted(const uint16_t* x, const int32_t* perm, int32_t T,
                                            int32_t k, int32_t with_shared, int32_t d,
                                            uint8_t* q, uint8_t* scale, void* stream);
+
+/* [G8][HY] Offline per-tensor FP8 quantisation ("HPC-Ops ...", section
+ * HPC-Ops的主要功能, GroupGEMM FP8: per-tensor FP8; "腾讯混元大模型：从多场景适配到
+ * 高效部署的全栈技术解析", section 量化压缩技术实践 / FP8量化方案): each of `batch`
+ * bf16 matrices [rows][cols] (cols % 8 == 0) gets one scale s = fp32(amax)/448
+ * (amax == 0 -> 1), q = e4m3_rne_satfinite(fp32(W / s)).  q [batch][rows][cols],
+ * scale float [batch] (also used as scratch while it runs). */
+moe_status moe_quantize_weights_fp8_tensor(const uint16_t* W, int64_t batch, int32_t rows,
+                                           int32_t cols, uint8_t* q, float* scale, void* stream);
+
+/* [HY] Static activation quantisation with a calibrated scale (> 0):
+ * q = e4m3_rne_satfinite(fp32(x / scale)); x [rows][cols] bf16, cols % 8 == 0. */
+moe_status moe_quantize_act_fp8_static(const uint16_t* x, int64_t rows, int32_t cols, float scale,
+                                       uint8_t* q, void* stream);
+
+/* [HY] The same, in the permuted row order of the grouped GEMMs: q [R][d]. */
+moe_status moe_quantize_act_fp8_static_permuted(const uint16_t* x, const int32_t* perm, int32_t T,
+                                                int32_t k, int32_t with_shared, int32_t d,
+                                                float scale, uint8_t* q, void* stream);
 
 /* [FM] The same activation quantisation, written in the permuted row order
  * of the grouped GEMMs (the FP8 gate-up GEMM's A operand): row p < T*k holds
@@ -224,6 +251,9 @@ moe_status moe_permute_noalloc(const int32_t* ids, int32_t T, int32_t E, int32_t
  *           [R][d/128] (moe_quantize_act_fp8_permuted; perm is then not read
  *           and may be NULL); h [R][I] e4m3 with h_scale float [R][I/128]
  *           (1x128 quantisation of the FP32 h in the epilogue).
+ * wdtype 3: x [R][d] e4m3 (moe_quantize_act_fp8_static_permuted with
+ *           weights->act_scale_x), h [R][I] e4m3 quantised with act_scale_h;
+ *           x_scale and h_scale are not read (may be NULL).
  * wdtype 2: the same with MXFP8: x_scale uint8 E8M0 [d/128][R][4]
  *           (moe_quantize_act_mxfp8_permuted), h_scale uint8 [I/128][R][4] (each
  *           1x32 block of the FP32 h quantised in the epilogue).

@@ -26,7 +26,9 @@ def bf16_to_f64(t: torch.Tensor) -> np.ndarray:
     return t.detach().float().cpu().double().numpy()
 
 
-def oracle_layer(cfg: MoEConfig, inp: dict, T: int = None) -> oracle.Layer:
+def oracle_layer(cfg: MoEConfig, inp: dict, T: int = None, act=(1.0, 1.0)) -> oracle.Layer:
+    """`act`: the static activation scales of a per-tensor FP8 layer (the GPU
+    layer's calibrated MoELayer.act_scales)."""
     def host(name):
         t = inp.get(name)
         return None if t is None else bits(t)
@@ -35,7 +37,7 @@ def oracle_layer(cfg: MoEConfig, inp: dict, T: int = None) -> oracle.Layer:
         w_gu=host("w_gu"), w_d=host("w_d"), ws_gu=host("ws_gu"), ws_d=host("ws_d"),
         router_w=inp["router_w"].detach().cpu().numpy(),
         router_bias=None if inp.get("router_bias") is None else inp["router_bias"].cpu().numpy(),
-        wdtype=cfg.wdtype, renorm=cfg.renorm)
+        wdtype=cfg.wdtype, renorm=cfg.renorm, act_sx=act[0], act_sh=act[1])
 
 
 def rms(a: np.ndarray) -> float:

@@ -35,6 +35,8 @@ SMALL = [
     MoEConfig("fp8odd", T=77, d=384, E=8, k=2, I=128, Is=0, wdtype=1, seed=32),
     MoEConfig("mxsmall", T=200, d=512, E=16, k=4, I=256, Is=256, wdtype=2, seed=33),
     MoEConfig("mxodd", T=77, d=384, E=8, k=2, I=128, Is=0, wdtype=2, seed=34),
+    MoEConfig("f8tsmall", T=200, d=512, E=16, k=4, I=256, Is=256, wdtype=3, seed=35),
+    MoEConfig("f8todd", T=77, d=384, E=8, k=2, I=128, Is=0, wdtype=3, seed=36),
 ]
 
 
@@ -108,7 +110,7 @@ def test_forward_small(cfg):
     st = _stage_outputs(layer, cfg, x)
     _check_routing_validity(st, cfg, cfg.T)
     st_np = {k: v.cpu().numpy() for k, v in st.items()}
-    ref = oracle.forward(oracle_layer(cfg, inp), bits(inp["x"]))
+    ref = oracle.forward(oracle_layer(cfg, inp, act=layer.act_scales), bits(inp["x"]))
     rel, namb = _compare_tokens(cfg, bf16_to_f64(y), st_np, ref, 6e-2 if cfg.wdtype else 2e-2)
     # the logits feeding the routing are FP32-accurate
     assert logit_rel_error(st_np["logits"], ref["logits"]).max() <= 1e-5
