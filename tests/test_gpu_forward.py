@@ -203,7 +203,8 @@ def _full_size_case(name, n_sample):
         w_d[e] = bits(inp["w_d"][int(e)])
     L = oracle.Layer(T=len(sample), d=cfg.d, E=cfg.E, k=cfg.k, I=cfg.I, Is=cfg.Is, w_gu=w_gu, w_d=w_d,
                      ws_gu=bits(inp["ws_gu"]), ws_d=bits(inp["ws_d"]), router_w=rw, router_bias=bias,
-                     wdtype=cfg.wdtype, renorm=cfg.renorm)
+                     wdtype=cfg.wdtype, renorm=cfg.renorm, act_sx=layer.act_scales[0],
+                     act_sh=layer.act_scales[1])
     ref = oracle.forward(L, xs)
     st_np = {k: v.cpu().numpy()[sample] for k, v in st.items() if k in ("logits", "ids", "w")}
     tol = 6e-2 if cfg.wdtype else 2e-2
@@ -212,7 +213,8 @@ def _full_size_case(name, n_sample):
     return cfg, st
 
 
-@pytest.mark.parametrize("name,n", [("decode", 64), ("prefill", 12), ("fp8", 4)])
+@pytest.mark.parametrize("name,n", [("decode", 64), ("prefill", 12), ("fp8", 4), ("mxfp8", 4),
+                                    ("fp8t", 4)])
 def test_forward_full_size(name, n):
     _full_size_case(name, n)
 
