@@ -154,13 +154,22 @@ def parse_clock_samples(lines):
 
 
 # ------------------------------------------------------------------ roofline
-def load_peaks():
+def load_peaks(sustained: bool = False):
+    """(HBM GB/s, dense BF16 TFLOP/s, source).  The BF16 figure is the burst one
+    for a short timed region, the sustained (power-capped) one for a long region."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
         with open(path) as f:
             p = json.load(f)
-        return p.get("hbm_gbs", 6650.0), p.get("bf16_tflops", 1590.0), "measured"
-    return 6650.0, 1590.0, "fallback"
+        tf = p.get("bf16_tflops_sustained", 1400.0) if sustained else p.get("bf16_tflops", 1590.0)
+        return p.get("hbm_gbs", 6650.0), tf, "measured"
+    return 6650.0, (1400.0 if sustained else 1590.0), "fallback"
+
+
+def power_capped(clocks: dict, ms_total: float) -> bool:
+    """Whether the timed region ran in the sustained regime: the power cap was
+    seen while it ran, or it was long enough to reach it (0.3 s)."""
+    return "sw_power_cap" in (clocks.get("reasons") or []) or ms_total > 300.0
 
 
 # DRAM traffic of the dominant kernel, from an ncu capture (dram__bytes_read.sum +
@@ -396,7 +405,8 @@ def run_ours(args, cfg: MoEConfig):
         raise RuntimeError("device status after timing: " + M.status_string(layer.device_status()))
 
     # roofline of the dominant kernel (the gate-up GEMM)
-    hbm_peak, tflops_peak, peak_kind = load_peaks()
+    sustained = power_capped(clocks.summary(), ms_total)
+    hbm_peak, tflops_peak, peak_kind = load_peaks(sustained)
     gu_ms = stage_ms["gemm_gateup"]
     gu_flops, gu_bytes = gateup_algorithmic(cfg, cfg.T, n_active)
     dn_flops, dn_bytes = down_algorithmic(cfg, cfg.T, n_active)
@@ -411,33 +421,50 @@ def run_ours(args, cfg: MoEConfig):
                 "unit": "TFLOP/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["kernel"] = "k_gateup_" + {0: "bf16", 1: "fp8", 2: "mx", 3: "f8t"}[cfg.wdtype]
+    tf_key = ("bf16_tflops_sustained (the timed region ran power-capped)" if sustained
+              else "bf16_tflops (burst: a short, unthrottled timed region)")
     roof["peak_source"] = (f"{peak_kind} MEASURED_PEAKS.json "
-                           + ("hbm_gbs" if roof["bound"] == "hbm" else "bf16_tflops (burst: the timed loop is well under a second)"
-                              + (" x2 (e4m3 nominal ratio)" if cfg.wdtype else "")))
+                           + ("hbm_gbs" if roof["bound"] == "hbm"
+                              else tf_key + (" x2 (e4m3 nominal ratio)" if cfg.wdtype else "")))
     roof["traffic"], roof["traffic_source"] = recorded_traffic(roof["kernel"], cfg.name)
     roof["algorithmic_bytes"] = gu_bytes
     roof["algorithmic_flops"] = gu_flops
     roof["launch_ms"] = gu_ms
 
-    # end to end through host buffers: copy x in, forward, copy y out, every step
-    xh = x.cpu().pin_memory()
-    yh = torch.empty_like(xh).pin_memory()
-    for _ in range(max(1, args.warmup)):
-        layer.forward_host(xh, yh)
+    # end to end through host buffers: every step copies its x in from pinned host
+    # memory, runs the forward and copies y out (moe_forward_host_async), the
+    # steps pipelined over two streams with one workspace each, so one step's
+    # copies overlap the other's kernels
+    xh = [x.cpu().pin_memory() for _ in range(2)]
+    yh = [torch.empty_like(xh[0]).pin_memory() for _ in range(2)]
+    wss = [layer.ws, torch.empty_like(layer.ws)]
+    streams = [torch.cuda.Stream(device=dev) for _ in range(2)]
+    for i in range(max(2, args.warmup)):
+        layer.forward_host_async(xh[i % 2], yh[i % 2], streams[i % 2], wss[i % 2])
+    torch.cuda.synchronize()
+    if not torch.equal(yh[0].to(dev), y) or layer.device_status() != M.OK:
+        raise RuntimeError("the host-buffer forward does not reproduce the device forward")
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
+    done = [torch.cuda.Event() for _ in range(2)]
     barrier()
     torch.cuda.synchronize()
     e0.record(stream)
-    for _ in range(args.steps):
-        layer.forward_host(xh, yh)
+    for st in streams:
+        st.wait_event(e0)
+    for i in range(args.steps):
+        layer.forward_host_async(xh[i % 2], yh[i % 2], streams[i % 2], wss[i % 2])
+    for j, st in enumerate(streams):
+        done[j].record(st)
+        stream.wait_event(done[j])
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
     e2e = {"value": world * cfg.T * args.steps / (e2e_ms / 1e3), "unit": UNIT,
-           "h2d_bytes_per_step": xh.numel() * xh.element_size(),
-           "d2h_bytes_per_step": yh.numel() * yh.element_size()}
+           "h2d_bytes_per_step": xh[0].numel() * xh[0].element_size(),
+           "d2h_bytes_per_step": yh[0].numel() * yh[0].element_size(),
+           "pipeline": "moe_forward_host_async, steps alternating over 2 streams (one workspace each)"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -591,6 +591,29 @@ moe_status moe_forward_profiled(const moe_shape* shape, const moe_weights* weigh
     return forward_device(shape, weights, x, y, ws, as_stream(stream), events);
 }
 
+moe_status moe_forward_host_async(const moe_shape* shape, const moe_weights* weights,
+                                  const uint16_t* x_host, uint16_t* y_host, void* ws,
+                                  size_t ws_bytes, void* stream) {
+    moe_status r = check_shape(shape);
+    if (r != MOE_OK) return r;
+    if ((r = check_weights(shape, weights, true, true, true)) != MOE_OK) return r;
+    if (shape->T == 0) return MOE_OK;
+    if (x_host == nullptr || y_host == nullptr) return MOE_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(*shape);
+    if ((r = check_ws(ws, ws_bytes, L.total)) != MOE_OK) return r;
+    if (!device_ok()) return MOE_ERR_UNSUPPORTED;
+    cudaStream_t st = as_stream(stream);
+    const size_t bytes = (size_t)shape->T * shape->d * 2;
+    uint16_t* xin = at<uint16_t>(ws, L.xin);
+    uint16_t* yout = at<uint16_t>(ws, L.yout);
+    if (cudaMemcpyAsync(xin, x_host, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if ((r = forward_device(shape, weights, xin, yout, ws, st)) != MOE_OK) return r;
+    if (cudaMemcpyAsync(y_host, yout, bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
 moe_status moe_forward_host(const moe_shape* shape, const moe_weights* weights,
                             const uint16_t* x_host, uint16_t* y_host, void* ws, size_t ws_bytes,
                             void* stream) {

@@ -38,6 +38,7 @@ EXPORTS = ["moe_status_string", "moe_workspace_bytes", "moe_permute_workspace_by
            "moe_router_logits", "moe_route_topk", "moe_permute", "moe_permute_noalloc",
            "moe_gemm_gateup",
            "moe_gemm_down", "moe_combine", "moe_forward", "moe_forward_profiled", "moe_forward_host",
+           "moe_forward_host_async",
            "moe_read_device_status", "moe_selftest_timeout"]
 
 
@@ -81,6 +82,7 @@ _sig = {
     "moe_forward": (_i32, [_S, _W, _vp, _vp, _vp, _sz, _vp]),
     "moe_forward_profiled": (_i32, [_S, _W, _vp, _vp, _vp, _sz, _vp, ctypes.POINTER(_vp), _i32]),
     "moe_forward_host": (_i32, [_S, _W, _vp, _vp, _vp, _sz, _vp]),
+    "moe_forward_host_async": (_i32, [_S, _W, _vp, _vp, _vp, _sz, _vp]),
     "moe_read_device_status": (_i32, [_vp, _vp]),
     "moe_selftest_timeout": (_i32, [_vp, _i32, _vp]),
 }
@@ -264,6 +266,12 @@ def forward_host(shape, weights, x_host, y_host, ws, stream=None):
            "moe_forward_host")
 
 
+def forward_host_async(shape, weights, x_host, y_host, ws, stream=None):
+    _check(_lib.moe_forward_host_async(ctypes.byref(shape), ctypes.byref(weights), _p(x_host),
+                                       _p(y_host), _p(ws), ws.numel() * ws.element_size(),
+                                       _stream(stream)), "moe_forward_host_async")
+
+
 def read_device_status(ws, stream=None) -> int:
     return int(_lib.moe_read_device_status(_p(ws), _stream(stream)))
 
@@ -384,6 +392,14 @@ class MoELayer:
     def forward_host(self, x_host: torch.Tensor, y_host: torch.Tensor, stream=None) -> torch.Tensor:
         forward_host(self.shape(x_host.shape[0]), self.weights, x_host.view(torch.uint16),
                      y_host.view(torch.uint16), self.ws, stream)
+        return y_host
+
+    def forward_host_async(self, x_host: torch.Tensor, y_host: torch.Tensor, stream=None,
+                           ws: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """Enqueue only (no synchronisation); `ws`: a workspace of this layer's
+        size for a second stream in flight (default: the layer's own)."""
+        forward_host_async(self.shape(x_host.shape[0]), self.weights, x_host.view(torch.uint16),
+                           y_host.view(torch.uint16), self.ws if ws is None else ws, stream)
         return y_host
 
     def device_status(self, stream=None) -> int:

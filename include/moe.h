@@ -306,6 +306,18 @@ moe_status moe_forward_host(const moe_shape* shape, const moe_weights* weights,
                             const uint16_t* x_host, uint16_t* y_host, void* ws,
                             size_t ws_bytes, void* stream);
 
+/* The same without the final synchronisation: enqueues the copy of x_host in,
+ * the forward and the copy of y out on `stream` and returns.  For pipelining
+ * consecutive batches over several streams (the copies of one batch overlap
+ * the kernels of another; H2D and D2H run on separate copy engines): use one
+ * workspace per stream with work in flight, keep x_host unmodified and read
+ * y_host only after `stream` has been synchronised (both pinned, or the copies
+ * are not asynchronous).  Errors found on the device go to ws's status word
+ * as for moe_forward. */
+moe_status moe_forward_host_async(const moe_shape* shape, const moe_weights* weights,
+                                  const uint16_t* x_host, uint16_t* y_host, void* ws,
+                                  size_t ws_bytes, void* stream);
+
 /* Synchronises `stream` and returns the device status word of `ws`
  * (MOE_OK, MOE_ERR_DEVICE_TIMEOUT or MOE_ERR_DEVICE_BAD_INDEX). */
 moe_status moe_read_device_status(const void* ws, void* stream);

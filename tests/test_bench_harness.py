@@ -72,3 +72,12 @@ def test_algorithmic_work_of_the_gemms():
     fd, bd = bench.down_algorithmic(cfg, cfg.T, n_active=200)
     assert fd == 2.0 * R * 1536 * 4096
     assert CONFIGS["prefill"].flops() == pytest.approx(2.82e12, rel=0.01)
+
+
+def test_peak_regime_follows_the_power_cap_and_region_length():
+    assert bench.power_capped({"reasons": ["sw_power_cap"]}, 50.0)
+    assert not bench.power_capped({"reasons": []}, 50.0)
+    assert bench.power_capped({"reasons": []}, 800.0)
+    hbm, burst, _ = bench.load_peaks(False)
+    _, sustained, _ = bench.load_peaks(True)
+    assert sustained <= burst and hbm > 0
