@@ -130,6 +130,27 @@ def test_forward_host_matches_device():
     assert torch.equal(yh, y_dev.cpu())
 
 
+def test_forward_host_async_pipelined_over_two_streams():
+    # batches alternate over two streams with one workspace each; every result
+    # equals the device forward of its own batch
+    cfg = SMALL[1]
+    inp = make_layer(cfg)
+    layer = M.MoELayer(cfg, inp)
+    xs = [inp["x"], torch.flip(inp["x"], dims=[0]).contiguous(), inp["x"] * 0.5]
+    refs = [layer.forward(x.to(DEV)).cpu() for x in xs]
+    torch.cuda.synchronize()
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    wss = [layer.ws, torch.empty_like(layer.ws)]
+    xh = [x.clone().pin_memory() for x in xs]
+    yh = [torch.empty_like(x).pin_memory() for x in xh]
+    for i in range(len(xs)):
+        layer.forward_host_async(xh[i], yh[i], streams[i % 2], wss[i % 2])
+    torch.cuda.synchronize()
+    for i in range(len(xs)):
+        assert torch.equal(yh[i], refs[i])
+    assert M.read_device_status(wss[0]) == M.OK and M.read_device_status(wss[1]) == M.OK
+
+
 def test_token_count_below_capacity_and_zero():
     cfg = SMALL[1]
     inp = make_layer(cfg)
