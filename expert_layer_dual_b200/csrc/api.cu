@@ -117,7 +117,7 @@ WsLayout ws_layout(const moe_shape& s) {
         L.xq = L.xs = L.hs = 0;
         L.h = take(R * I * 2);
     }
-    L.o = take(R * d * 4);                                // FP32 rows of the down GEMM
+    L.o = take(R * d * 2);                                // FP16 rows of the down GEMM
     L.xin = take(T * d * 2);
     L.yout = take(T * d * 2);
     L.total = off;
@@ -228,7 +228,7 @@ moe_status run_gateup(const moe_shape* s, const moe_weights* w, const void* x, c
 }
 
 moe_status run_down(const moe_shape* s, const moe_weights* w, const void* h, const void* hs,
-                    const int32_t* offsets, float* o, int32_t* status, cudaStream_t st) {
+                    const int32_t* offsets, __half* o, int32_t* status, cudaStream_t st) {
     const GroupedGemmArgs a = gemm_args(s, offsets, nullptr, status);
     if (s->wdtype == MOE_WDTYPE_BF16)
         return cuda_status((use_pair_tiles(s->T, s->E, s->k) ? launch_down_bf16_2sm
@@ -331,7 +331,7 @@ moe_status forward_device(const moe_shape* s, const moe_weights* w, const uint16
     if (!mark(4)) return MOE_ERR_CUDA;
     void* h = at<uint8_t>(ws, L.h);
     void* hs = (fp8 || mx) ? at<uint8_t>(ws, L.hs) : nullptr;
-    float* o = at<float>(ws, L.o);
+    __half* o = at<__half>(ws, L.o);
     if ((r = run_gateup(s, w, a_in, a_scale, perm, offsets, h, hs, status, st)) != MOE_OK) return r;
     if (!mark(5)) return MOE_ERR_CUDA;
     if ((r = run_down(s, w, h, hs, offsets, o, status, st)) != MOE_OK) return r;
@@ -535,7 +535,7 @@ moe_status moe_gemm_gateup(const moe_shape* shape, const moe_weights* weights, c
 }
 
 moe_status moe_gemm_down(const moe_shape* shape, const moe_weights* weights, const void* h,
-                         const void* h_scale, const int32_t* offsets, float* o, void* ws,
+                         const void* h_scale, const int32_t* offsets, void* o, void* ws,
                          size_t ws_bytes, void* stream) {
     moe_status r = check_shape(shape);
     if (r != MOE_OK) return r;
@@ -549,18 +549,18 @@ moe_status moe_gemm_down(const moe_shape* shape, const moe_weights* weights, con
     cudaStream_t st = as_stream(stream);
     int32_t* status = at<int32_t>(ws, 0);
     if (cudaMemsetAsync(status, 0, sizeof(int32_t), st) != cudaSuccess) return MOE_ERR_CUDA;
-    return run_down(shape, weights, h, h_scale, offsets, o, status, st);
+    return run_down(shape, weights, h, h_scale, offsets, static_cast<__half*>(o), status, st);
 }
 
-moe_status moe_combine(const moe_shape* shape, const float* o, const int32_t* inv,
+moe_status moe_combine(const moe_shape* shape, const void* o, const int32_t* inv,
                        const float* w, uint16_t* y, void* stream) {
     moe_status r = check_shape(shape);
     if (r != MOE_OK) return r;
     if (shape->T == 0) return MOE_OK;
     if (o == nullptr || inv == nullptr || w == nullptr || y == nullptr) return MOE_ERR_INVALID_ARG;
     if (!device_ok()) return MOE_ERR_UNSUPPORTED;
-    return cuda_status(launch_combine(o, inv, w, y, shape->T, shape->d, shape->k,
-                                      shape->I_shared > 0 ? 1 : 0, as_stream(stream)));
+    return cuda_status(launch_combine(static_cast<const __half*>(o), inv, w, y, shape->T, shape->d,
+                                      shape->k, shape->I_shared > 0 ? 1 : 0, as_stream(stream)));
 }
 
 moe_status moe_forward(const moe_shape* shape, const moe_weights* weights, const uint16_t* x,

@@ -10,6 +10,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -509,6 +510,25 @@ __device__ __forceinline__ void st_global_v4(void* p, uint32_t a, uint32_t b, ui
     asm volatile("st.global.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(a), "r"(b), "r"(c),
                  "r"(d)
                  : "memory");
+}
+
+// Two FP32 values as an FP16 pair (lo in the low half): round to nearest
+// even, saturating (finite values beyond +-65504 become +-65504; NaN stays NaN).
+__device__ __forceinline__ uint32_t pack_f16x2_sat(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// 32 consecutive FP32 values, each times f, stored as FP16: 64 bytes at a
+// 16-byte aligned address (the expert-output rows o of the down GEMMs).
+__device__ __forceinline__ void st_f16x32(__half* dst, const float* v, float f = 1.0f) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+        st_global_v4(dst + 8 * q, pack_f16x2_sat(v[8 * q] * f, v[8 * q + 1] * f),
+                     pack_f16x2_sat(v[8 * q + 2] * f, v[8 * q + 3] * f),
+                     pack_f16x2_sat(v[8 * q + 4] * f, v[8 * q + 5] * f),
+                     pack_f16x2_sat(v[8 * q + 6] * f, v[8 * q + 7] * f));
 }
 
 }  // namespace moe

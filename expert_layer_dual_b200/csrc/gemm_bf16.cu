@@ -23,7 +23,7 @@
 //  - one thread issues tcgen05.mma into one of two 256-column TMEM
 //    accumulators, so the epilogue of a tile overlaps the next tile's MMAs;
 //  - 4 epilogue warps read TMEM (tcgen05.ld), apply SiLU*mul (gate-up) and
-//    store rows (h in bf16, the MMA operand of the down GEMM; o in FP32);
+//    store rows (h in bf16, the MMA operand of the down GEMM; o in FP16);
 // Every wait is bounded; a timeout sets the device status word and all roles
 // stop, drain their copies in flight and free TMEM.
 #include "common.cuh"
@@ -331,11 +331,12 @@ __global__ void __launch_bounds__(GATEUP_THREADS, 1)
 // ---------------------------------------------------------------------------
 // Down: o[p][n0 + j] = h[p] . Wd[n0 + j]
 // ---------------------------------------------------------------------------
-// o stays FP32 [R][d]: rounding it to bf16 before the weighted combine would
-// add a second rounding of every term to the layer output's own.
+// o is stored FP16 [R][d] (saturating): its rounding (2^-11 relative) adds
+// little to the layer output's own bf16 rounding, where a bf16 o would add a
+// second rounding of the same size to every term of the weighted combine.
 __global__ void __launch_bounds__(DOWN_THREADS, 1)
     k_down_bf16(const __grid_constant__ CUtensorMap tm_h, const __grid_constant__ CUtensorMap tm_w,
-                const __grid_constant__ CUtensorMap tm_ws, GroupedGemmArgs a, float* __restrict__ o) {
+                const __grid_constant__ CUtensorMap tm_ws, GroupedGemmArgs a, __half* __restrict__ o) {
     extern __shared__ uint8_t smem_raw[];
     Smem sm = carve_smem(smem_raw);
     Bars* b = sm.bars;
@@ -405,19 +406,13 @@ __global__ void __launch_bounds__(DOWN_THREADS, 1)
             tc_fence_after_sync();
             const uint32_t taddr = tmem + (static_cast<uint32_t>(warp * 32) << 16) + buf * BN;
             const int ncols = min(BN, a.d - t.n * BN);
-            float* dst = o + (int64_t)(t.row0 + row) * a.d + t.n * BN;
+            __half* dst = o + (int64_t)(t.row0 + row) * a.d + t.n * BN;
 #pragma unroll 1
             for (int c = 0; c < BN / 32; ++c) {
                 if (c * 32 >= ncols) break;  // uniform across the warp
                 float v[32];
                 tmem_load32(taddr + c * 32, v);
-                if (row < t.nrows) {
-#pragma unroll
-                    for (int q = 0; q < 8; ++q)
-                        st_global_v4(dst + c * 32 + q * 4, __float_as_uint(v[4 * q]),
-                                     __float_as_uint(v[4 * q + 1]), __float_as_uint(v[4 * q + 2]),
-                                     __float_as_uint(v[4 * q + 3]));
-                }
+                if (row < t.nrows) st_f16x32(dst + c * 32, v);
             }
             tc_fence_before_sync();
             warp_arrive(&b->tempty[buf]);
@@ -455,7 +450,7 @@ cudaError_t launch_gateup_bf16(const GroupedGemmArgs& a, const uint16_t* x, cons
 }
 
 cudaError_t launch_down_bf16(const GroupedGemmArgs& a, const uint16_t* h, const uint16_t* w_d,
-                             const uint16_t* ws_d, float* o, cudaStream_t s) {
+                             const uint16_t* ws_d, __half* o, cudaStream_t s) {
     if (a.T == 0) return cudaSuccess;
     const uint64_t R = (uint64_t)a.T * a.k + (a.has_shared ? a.T : 0);
     CUtensorMap th, tw, tws;

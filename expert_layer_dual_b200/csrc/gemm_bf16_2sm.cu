@@ -167,7 +167,7 @@ __device__ __forceinline__ void mma_role(Smem& sm, const GroupedGemmArgs& a, uin
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DOWN_THREADS, 1)
     k_down_bf16_2sm(const __grid_constant__ CUtensorMap tm_h, const __grid_constant__ CUtensorMap tm_w,
                     const __grid_constant__ CUtensorMap tm_ws, GroupedGemmArgs a,
-                    float* __restrict__ o) {
+                    __half* __restrict__ o) {
     extern __shared__ uint8_t smem_raw[];
     Smem sm = carve(smem_raw);
     Bars* b = sm.bars;
@@ -228,19 +228,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DOWN_THREADS, 1)
             tc_fence_after_sync();
             const uint32_t taddr = tmem + (static_cast<uint32_t>(warp * 32) << 16) + buf * BN;
             const int ncols = min(BN, a.d - p.t.n * BN);
-            float* dst = o + (int64_t)(p.row0 + row) * a.d + p.t.n * BN;
+            __half* dst = o + (int64_t)(p.row0 + row) * a.d + p.t.n * BN;
 #pragma unroll 1
             for (int c = 0; c < BN / 32; ++c) {
                 if (c * 32 >= ncols) break;  // uniform across the warp
                 float v[32];
                 tmem_load32(taddr + c * 32, v);
-                if (row < p.nrows) {
-#pragma unroll
-                    for (int q = 0; q < 8; ++q)
-                        st_global_v4(dst + c * 32 + q * 4, __float_as_uint(v[4 * q]),
-                                     __float_as_uint(v[4 * q + 1]), __float_as_uint(v[4 * q + 2]),
-                                     __float_as_uint(v[4 * q + 3]));
-                }
+                if (row < p.nrows) st_f16x32(dst + c * 32, v);
             }
             tc_fence_before_sync();
             warp_arrive_leader(&b->tempty[buf]);
@@ -264,7 +258,7 @@ int pair_grid() { return (current_device_info().num_sms / 2) * 2; }
 }  // namespace
 
 cudaError_t launch_down_bf16_2sm(const GroupedGemmArgs& a, const uint16_t* h, const uint16_t* w_d,
-                                 const uint16_t* ws_d, float* o, cudaStream_t s) {
+                                 const uint16_t* ws_d, __half* o, cudaStream_t s) {
     if (a.T == 0) return cudaSuccess;
     const uint64_t R = (uint64_t)a.T * a.k + (a.has_shared ? a.T : 0);
     CUtensorMap th, tw, tws;

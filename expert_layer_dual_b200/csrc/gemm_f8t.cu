@@ -273,7 +273,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 __global__ void __launch_bounds__(THREADS, 1)
     k_down_f8t(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_w,
                const __grid_constant__ CUtensorMap tm_ws, GroupedGemmArgs a, float sh,
-               const float* __restrict__ wsc, const float* __restrict__ wssc, float* __restrict__ o) {
+               const float* __restrict__ wsc, const float* __restrict__ wssc, __half* __restrict__ o) {
     extern __shared__ uint8_t smem_raw[];
     Smem sm = carve(smem_raw);
     Bars* b = sm.bars;
@@ -315,19 +315,13 @@ __global__ void __launch_bounds__(THREADS, 1)
             const float f = sh * (t.g >= a.E ? wssc[0] : wsc[t.g]);
             const uint32_t taddr = tmem + (static_cast<uint32_t>(warp * 32) << 16) + buf * BN;
             const int ncols = min(BN, a.d - t.n * BN);
-            float* dst = o + (int64_t)(t.row0 + row) * a.d + t.n * BN;
+            __half* dst = o + (int64_t)(t.row0 + row) * a.d + t.n * BN;
 #pragma unroll 1
             for (int c = 0; c < BN / 32; ++c) {
                 if (c * 32 >= ncols) break;  // uniform across the warp
                 float v[32];
                 tmem_load32(taddr + c * 32, v);
-                if (row < t.nrows) {
-#pragma unroll
-                    for (int q = 0; q < 8; ++q)
-                        st_global_v4(dst + c * 32 + q * 4, __float_as_uint(v[4 * q] * f),
-                                     __float_as_uint(v[4 * q + 1] * f), __float_as_uint(v[4 * q + 2] * f),
-                                     __float_as_uint(v[4 * q + 3] * f));
-                }
+                if (row < t.nrows) st_f16x32(dst + c * 32, v, f);
             }
             tc_fence_before_sync();
             warp_arrive(&b->tempty[buf]);
@@ -371,7 +365,7 @@ cudaError_t launch_gateup_f8t(const GroupedGemmArgs& a, const uint8_t* xq, float
 
 cudaError_t launch_down_f8t(const GroupedGemmArgs& a, const uint8_t* hq, float sh,
                             const uint8_t* w_d, const float* w_d_s, const uint8_t* ws_d,
-                            const float* ws_d_s, float* o, cudaStream_t s) {
+                            const float* ws_d_s, __half* o, cudaStream_t s) {
     if (a.T == 0) return cudaSuccess;
     const uint64_t R = (uint64_t)a.T * a.k + (a.has_shared ? a.T : 0);
     CUtensorMap ta, tw, tws;

@@ -472,7 +472,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     k_down_fp8(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_w,
                const __grid_constant__ CUtensorMap tm_ws, GroupedGemmArgs a,
                const float* __restrict__ hs, const float* __restrict__ wsc,
-               const float* __restrict__ wssc, float* __restrict__ o) {
+               const float* __restrict__ wssc, __half* __restrict__ o) {
     extern __shared__ uint8_t smem_raw[];
     Smem sm = carve(smem_raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -546,11 +546,9 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (valid && live) {
                 float acc[64];
                 unpack_acc(acc2, acc);
-                float* dst = o + (int64_t)(t.row0 + row) * a.d + t.n * BN + qtr * 64;
-#pragma unroll
-                for (int q = 0; q < 16; ++q)
-                    st_global_v4(dst + 4 * q, __float_as_uint(acc[4 * q]), __float_as_uint(acc[4 * q + 1]),
-                                 __float_as_uint(acc[4 * q + 2]), __float_as_uint(acc[4 * q + 3]));
+                __half* dst = o + (int64_t)(t.row0 + row) * a.d + t.n * BN + qtr * 64;
+                st_f16x32(dst, acc);
+                st_f16x32(dst + 32, acc + 32);
             }
         }
     }
@@ -590,7 +588,7 @@ cudaError_t launch_gateup_fp8(const GroupedGemmArgs& a, const uint8_t* xq, const
 
 cudaError_t launch_down_fp8(const GroupedGemmArgs& a, const uint8_t* hq, const float* hs,
                             const uint8_t* w_d, const float* w_d_s, const uint8_t* ws_d,
-                            const float* ws_d_s, float* o, cudaStream_t s) {
+                            const float* ws_d_s, __half* o, cudaStream_t s) {
     if (a.T == 0) return cudaSuccess;
     const uint64_t R = (uint64_t)a.T * a.k + (a.has_shared ? a.T : 0);
     CUtensorMap ta, tw, tws;

@@ -375,7 +375,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     k_down_mx(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_w,
               const __grid_constant__ CUtensorMap tm_ws, GroupedGemmArgs a,
               const uint8_t* __restrict__ hs, const uint8_t* __restrict__ wsc,
-              const uint8_t* __restrict__ wssc, float* __restrict__ o) {
+              const uint8_t* __restrict__ wssc, __half* __restrict__ o) {
     extern __shared__ uint8_t smem_raw[];
     Smem sm = carve(smem_raw);
     Bars* b = sm.bars;
@@ -427,11 +427,9 @@ __global__ void __launch_bounds__(THREADS, 1)
             warp_arrive(&b->tempty);
             const int col = t.n * BN + qtr * 64;
             if (row < t.nrows && col < a.d) {
-                float* dst = o + (int64_t)(t.row0 + row) * a.d + col;
-#pragma unroll
-                for (int q = 0; q < 16; ++q)
-                    st_global_v4(dst + 4 * q, __float_as_uint(v[4 * q]), __float_as_uint(v[4 * q + 1]),
-                                 __float_as_uint(v[4 * q + 2]), __float_as_uint(v[4 * q + 3]));
+                __half* dst = o + (int64_t)(t.row0 + row) * a.d + col;
+                st_f16x32(dst, v);
+                st_f16x32(dst + 32, v + 32);
             }
         }
     }
@@ -473,7 +471,7 @@ cudaError_t launch_gateup_mx(const GroupedGemmArgs& a, const uint8_t* xq, const 
 
 cudaError_t launch_down_mx(const GroupedGemmArgs& a, const uint8_t* hq, const uint8_t* hs,
                            const uint8_t* w_d, const uint8_t* w_d_s, const uint8_t* ws_d,
-                           const uint8_t* ws_d_s, float* o, cudaStream_t s) {
+                           const uint8_t* ws_d_s, __half* o, cudaStream_t s) {
     if (a.T == 0) return cudaSuccess;
     const uint64_t R = (uint64_t)a.T * a.k + (a.has_shared ? a.T : 0);
     CUtensorMap ta, tw, tws;

@@ -4,6 +4,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -35,7 +36,7 @@ cudaError_t launch_permute(const int32_t* ids, int T, int E, int k, int32_t* cou
                            int32_t* offsets, int32_t* perm, int32_t* inv, int32_t* seg_hist,
                            int32_t* status, cudaStream_t s);
 // o [R][d] f32: routed rows then (has_shared) the shared expert's rows
-cudaError_t launch_combine(const float* o, const int32_t* inv, const float* w, uint16_t* y, int T,
+cudaError_t launch_combine(const __half* o, const int32_t* inv, const float* w, uint16_t* y, int T,
                            int d, int k, int has_shared, cudaStream_t s);
 cudaError_t launch_quant_act_fp8(const uint16_t* x, int64_t rows, int cols, uint8_t* q,
                                  float* scale, cudaStream_t s);
@@ -89,11 +90,11 @@ struct GroupedGemmArgs {
 cudaError_t launch_gateup_bf16(const GroupedGemmArgs& a, const uint16_t* x, const uint16_t* w_gu,
                                const uint16_t* ws_gu, uint16_t* h, cudaStream_t s);
 cudaError_t launch_down_bf16(const GroupedGemmArgs& a, const uint16_t* h, const uint16_t* w_d,
-                             const uint16_t* ws_d, float* o, cudaStream_t s);
+                             const uint16_t* ws_d, __half* o, cudaStream_t s);
 
 // ---- gemm_bf16_2sm.cu (down GEMM on CTA-pair tiles of 256 rows)
 cudaError_t launch_down_bf16_2sm(const GroupedGemmArgs& a, const uint16_t* h, const uint16_t* w_d,
-                                 const uint16_t* ws_d, float* o, cudaStream_t s);
+                                 const uint16_t* ws_d, __half* o, cudaStream_t s);
 // Whether the CTA-pair down kernel serves this shape (>= 512 rows per expert on average).
 inline bool use_pair_tiles(int T, int E, int k) { return (int64_t)T * k >= (int64_t)512 * E; }
 
@@ -103,7 +104,7 @@ cudaError_t launch_gateup_fp8(const GroupedGemmArgs& a, const uint8_t* xq, const
                               const float* ws_gu_s, uint8_t* hq, float* hs, cudaStream_t s);
 cudaError_t launch_down_fp8(const GroupedGemmArgs& a, const uint8_t* hq, const float* hs,
                             const uint8_t* w_d, const float* w_d_s, const uint8_t* ws_d,
-                            const float* ws_d_s, float* o, cudaStream_t s);
+                            const float* ws_d_s, __half* o, cudaStream_t s);
 
 // ---- gemm_mx.cu (tcgen05 block-scaled grouped GEMMs, MXFP8: e4m3 + E8M0 per 1x32)
 // Scales are bytes [rows][K/32]; h / o as in the FP8 path.
@@ -112,7 +113,7 @@ cudaError_t launch_gateup_mx(const GroupedGemmArgs& a, const uint8_t* xq, const 
                              const uint8_t* ws_gu_s, uint8_t* hq, uint8_t* hs, cudaStream_t s);
 cudaError_t launch_down_mx(const GroupedGemmArgs& a, const uint8_t* hq, const uint8_t* hs,
                            const uint8_t* w_d, const uint8_t* w_d_s, const uint8_t* ws_d,
-                           const uint8_t* ws_d_s, float* o, cudaStream_t s);
+                           const uint8_t* ws_d_s, __half* o, cudaStream_t s);
 
 // ---- gemm_f8t.cu (tcgen05 grouped GEMMs, per-tensor FP8, static activation scales)
 cudaError_t launch_gateup_f8t(const GroupedGemmArgs& a, const uint8_t* xq, float sx, float sh,
@@ -120,7 +121,7 @@ cudaError_t launch_gateup_f8t(const GroupedGemmArgs& a, const uint8_t* xq, float
                               const float* ws_gu_s, uint8_t* hq, cudaStream_t s);
 cudaError_t launch_down_f8t(const GroupedGemmArgs& a, const uint8_t* hq, float sh,
                             const uint8_t* w_d, const float* w_d_s, const uint8_t* ws_d,
-                            const float* ws_d_s, float* o, cudaStream_t s);
+                            const float* ws_d_s, __half* o, cudaStream_t s);
 
 // ---- tensor maps (api.cu)
 // 2-D row-major tensor [rows][cols] of `elem_bytes`-sized elements, box

@@ -272,9 +272,9 @@ cudaError_t launch_permute(const int32_t* ids, int T, int E, int k, int32_t* cou
 }
 
 // ---------------------------------------------------------------------------
-// Combine: y[t] = sum_j w[t][j] * o[inv[t*k+j]] + o[T*k+t], FP32 rows from
-// the down GEMM, FP32 sum in the order j = 0..k-1 then the shared row, one
-// bf16 rounding.  One block per token, 16-byte loads along d.
+// Combine: y[t] = sum_j w[t][j] * o[inv[t*k+j]] + o[T*k+t], FP16 rows from
+// the down GEMM (widened exactly), FP32 sum in the order j = 0..k-1 then the
+// shared row, one bf16 rounding.  One block per token, 16-byte loads along d.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float* f) {
     const uint32_t r[4] = {u.x, u.y, u.z, u.w};
@@ -285,17 +285,20 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float* f) {
     }
 }
 
-__device__ __forceinline__ void add8(float* acc, const float* row, float wj) {
-    const float4 a = __ldg(reinterpret_cast<const float4*>(row));
-    const float4 b = __ldg(reinterpret_cast<const float4*>(row) + 1);
-    acc[0] = fmaf(wj, a.x, acc[0]); acc[1] = fmaf(wj, a.y, acc[1]);
-    acc[2] = fmaf(wj, a.z, acc[2]); acc[3] = fmaf(wj, a.w, acc[3]);
-    acc[4] = fmaf(wj, b.x, acc[4]); acc[5] = fmaf(wj, b.y, acc[5]);
-    acc[6] = fmaf(wj, b.z, acc[6]); acc[7] = fmaf(wj, b.w, acc[7]);
+// acc[i] += wj * row[i] for the 8 FP16 values of one 16-byte load.
+__device__ __forceinline__ void add8(float* acc, const __half* row, float wj) {
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(row));
+    const uint32_t r[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&r[i]));
+        acc[2 * i] = fmaf(wj, f.x, acc[2 * i]);
+        acc[2 * i + 1] = fmaf(wj, f.y, acc[2 * i + 1]);
+    }
 }
 
 __global__ void __launch_bounds__(128)
-    k_combine(const float* __restrict__ o, const int32_t* __restrict__ inv,
+    k_combine(const __half* __restrict__ o, const int32_t* __restrict__ inv,
               const float* __restrict__ w, uint16_t* __restrict__ y, int T, int d, int k,
               int has_shared) {
     __shared__ int32_t rows[8];
@@ -329,7 +332,7 @@ __global__ void __launch_bounds__(128)
     }
 }
 
-cudaError_t launch_combine(const float* o, const int32_t* inv, const float* w, uint16_t* y, int T,
+cudaError_t launch_combine(const __half* o, const int32_t* inv, const float* w, uint16_t* y, int T,
                            int d, int k, int has_shared, cudaStream_t s) {
     if (T == 0) return cudaSuccess;
     k_combine<<<T, 128, 0, s>>>(o, inv, w, y, T, d, k, has_shared);

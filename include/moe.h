@@ -265,18 +265,22 @@ moe_status moe_gemm_gateup(const moe_shape* shape, const moe_weights* weights,
                            void* ws, size_t ws_bytes, void* stream);
 
 /* [FM][G8] Grouped Down GEMM: o[p] = h[p] . Wd[e]^T with FP32 accumulation,
- * same row grouping as moe_gemm_gateup, stored FP32: o [R][d] f32.  (The
- * rows stay FP32 until the weighted combine so the layer output is rounded
- * to bf16 once.)  ws: at least 256 bytes (the status word). */
+ * same row grouping as moe_gemm_gateup, stored as IEEE FP16 (binary16 bit
+ * patterns): o [R][d] f16, rounded to nearest even and saturating (finite
+ * sums beyond +-65504 are stored as +-65504).  FP16 keeps 11 significant
+ * bits, so this rounding (at most 2^-11 relative) adds little to the bf16
+ * rounding of the layer output; bf16 rows would add a second rounding of
+ * the output's own size.  ws: at least 256 bytes (the status word). */
 moe_status moe_gemm_down(const moe_shape* shape, const moe_weights* weights,
                          const void* h, const void* h_scale, const int32_t* offsets,
-                         float* o, void* ws, size_t ws_bytes, void* stream);
+                         void* o, void* ws, size_t ws_bytes, void* stream);
 
 /* [FM] Top-K weighted aggregation plus the shared expert:
  *   y[t] = sum_j w[t][j] * o[inv[t*k+j]] + o[T*k+t]
- * FP32 sum in the order j = 0..k-1 then the shared term (only when
- * I_shared > 0), one bf16 rounding.  o [R][d] f32, y [T][d] bf16. */
-moe_status moe_combine(const moe_shape* shape, const float* o, const int32_t* inv,
+ * o widened exactly to FP32, FP32 sum in the order j = 0..k-1 then the
+ * shared term (only when I_shared > 0), one bf16 rounding.
+ * o [R][d] f16 (as moe_gemm_down writes it), y [T][d] bf16. */
+moe_status moe_combine(const moe_shape* shape, const void* o, const int32_t* inv,
                        const float* w, uint16_t* y, void* stream);
 
 /* The whole layer in one call: router logits -> top-k -> permute ->

@@ -44,6 +44,11 @@ def rms(a: np.ndarray) -> float:
     return float(np.sqrt(np.mean(np.square(a, dtype=np.float64))))
 
 
+# Expert-output rows o are stored FP16 (round to nearest even): one rounding
+# of at most 2^-11 relative on top of the FP32 accumulation (1e-4).
+O_RTOL = 2.0 ** -11 + 1e-4
+
+
 def assert_close_rel(got, ref, rtol, atol, what=""):
     """|got - ref| <= atol + rtol * |ref| elementwise, with a useful message."""
     got = np.asarray(got, np.float64)

@@ -11,7 +11,7 @@ import torch
 import oracle
 from expert_layer_dual_b200.configs import MoEConfig
 from expert_layer_dual_b200.inputs import make_layer, random_bf16, random_ids
-from gpu_util import assert_close_rel, bf16_to_f64, bits, oracle_layer, rms
+from gpu_util import O_RTOL, assert_close_rel, bf16_to_f64, bits, oracle_layer, rms
 
 pytestmark = pytest.mark.gpu
 
@@ -119,9 +119,9 @@ def test_gemm_down_f8t(cfg):
     hin = random_bf16((R, cfg.I), seed=cfg.seed, idx=11, std=0.5)
     hq = torch.empty((R, cfg.I), dtype=torch.uint8, device=DEV)
     M.quantize_act_fp8_static(_u16(hin.to(DEV)), sh, hq)
-    o = torch.empty((R, cfg.d), dtype=torch.float32, device=DEV)
+    o = torch.empty((R, cfg.d), dtype=torch.float16, device=DEV)
     M.gemm_down(layer.shape(cfg.T), layer.weights, hq, None, offsets, o, layer.ws)
     assert M.read_device_status(layer.ws) == M.OK
     _, ooff, _, _ = oracle.permute(ids.numpy(), cfg.E)
     ref = oracle.down(oracle_layer(cfg, inp, act=(sx, sh)), bf16_to_f64(hin), ooff, cfg.T)
-    assert_close_rel(o.cpu().double().numpy(), ref, rtol=1e-4, atol=1e-4 * rms(ref), what="o")
+    assert_close_rel(o.cpu().double().numpy(), ref, rtol=O_RTOL, atol=1e-4 * rms(ref), what="o")

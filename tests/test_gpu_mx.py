@@ -10,7 +10,7 @@ import torch
 import oracle
 from expert_layer_dual_b200.configs import MoEConfig
 from expert_layer_dual_b200.inputs import make_layer, random_bf16, random_ids
-from gpu_util import assert_close_rel, bf16_to_f64, bits, oracle_layer, rms
+from gpu_util import O_RTOL, assert_close_rel, bf16_to_f64, bits, oracle_layer, rms
 
 pytestmark = pytest.mark.gpu
 
@@ -151,9 +151,9 @@ def test_gemm_down_mx(cfg):
     hq = torch.empty((R, cfg.I), dtype=torch.uint8, device=DEV)
     hs = torch.empty((R, cfg.I // 32), dtype=torch.uint8, device=DEV)
     M.quantize_act_mxfp8(_u16(hin.to(DEV)), hq, hs)
-    o = torch.empty((R, cfg.d), dtype=torch.float32, device=DEV)
+    o = torch.empty((R, cfg.d), dtype=torch.float16, device=DEV)
     M.gemm_down(layer.shape(cfg.T), layer.weights, hq, hs, offsets, o, layer.ws)
     assert M.read_device_status(layer.ws) == M.OK
     _, ooff, _, _ = oracle.permute(ids.numpy(), cfg.E)
     ref = oracle.down(oracle_layer(cfg, inp), bf16_to_f64(hin), ooff, cfg.T)
-    assert_close_rel(o.cpu().double().numpy(), ref, rtol=1e-4, atol=1e-4 * rms(ref), what="o")
+    assert_close_rel(o.cpu().double().numpy(), ref, rtol=O_RTOL, atol=1e-4 * rms(ref), what="o")

@@ -18,7 +18,7 @@ import oracle
 from expert_layer_dual_b200.configs import MoEConfig
 from expert_layer_dual_b200.inputs import (make_layer, random_bf16, random_ids, random_logits,
                                            random_weights)
-from gpu_util import assert_close_rel, bf16_to_f64, bits, logit_rel_error, oracle_layer, rms
+from gpu_util import O_RTOL, assert_close_rel, bf16_to_f64, bits, logit_rel_error, oracle_layer, rms
 
 pytestmark = pytest.mark.gpu
 
@@ -158,13 +158,36 @@ def test_gemm_down_bf16(cfg):
     _, offsets, _, _ = _gpu_permute(ids.to(DEV), cfg.E)
     R = cfg.rows()
     hin = random_bf16((R, cfg.I), seed=cfg.seed, idx=1, std=0.5)
-    o = torch.empty((R, cfg.d), dtype=torch.float32, device=DEV)
+    o = torch.empty((R, cfg.d), dtype=torch.float16, device=DEV)
     M.gemm_down(layer.shape(cfg.T), layer.weights, _u16(hin.to(DEV)), None, offsets, o, layer.ws)
     assert M.read_device_status(layer.ws) == M.OK
     _, ooff, _, _ = oracle.permute(ids.numpy(), cfg.E)
     ref = oracle.down(oracle_layer(cfg, inp), bf16_to_f64(hin), ooff, cfg.T)
-    # FP32 rows: only the tensor core's FP32 accumulation over I terms
-    assert_close_rel(o.cpu().double().numpy(), ref, rtol=1e-4, atol=1e-4 * rms(ref), what="o")
+    # FP16 rows: the tensor core's FP32 accumulation over I terms, one FP16 rounding
+    assert_close_rel(o.cpu().double().numpy(), ref, rtol=O_RTOL, atol=1e-4 * rms(ref), what="o")
+
+
+def test_gemm_down_saturates_fp16_rows():
+    """Sums past the FP16 range are stored as +-65504 (never inf); the rest as usual."""
+    cfg = SMALL[0]
+    inp = make_layer(cfg)
+    layer = M.MoELayer(cfg, inp)
+    ids = random_ids(cfg.T, cfg.E, cfg.k, seed=cfg.seed + 210)
+    _, offsets, _, _ = _gpu_permute(ids.to(DEV), cfg.E)
+    R = cfg.rows()
+    hin = random_bf16((R, cfg.I), seed=cfg.seed, idx=12, std=2.0e6)
+    o = torch.empty((R, cfg.d), dtype=torch.float16, device=DEV)
+    M.gemm_down(layer.shape(cfg.T), layer.weights, _u16(hin.to(DEV)), None, offsets, o, layer.ws)
+    assert M.read_device_status(layer.ws) == M.OK
+    _, ooff, _, _ = oracle.permute(ids.numpy(), cfg.E)
+    ref = oracle.down(oracle_layer(cfg, inp), bf16_to_f64(hin), ooff, cfg.T)
+    got = o.cpu().double().numpy()
+    assert np.all(np.isfinite(got))
+    big = np.abs(ref) > 65504.0 * (1 + 1e-3)
+    assert big.mean() > 0.1 and (~big).mean() > 0.01          # both regimes are exercised
+    assert np.array_equal(got[big], np.sign(ref[big]) * 65504.0)
+    small = np.abs(ref) < 65504.0 * (1 - 1e-3)
+    assert_close_rel(got[small], ref[small], rtol=O_RTOL, atol=1e-4 * rms(ref), what="o")
 
 
 @pytest.mark.parametrize("cfg", SMALL, ids=IDS)
@@ -172,7 +195,7 @@ def test_combine(cfg):
     ids = random_ids(cfg.T, cfg.E, cfg.k, seed=cfg.seed + 300)
     _, _, _, inv = _gpu_permute(ids.to(DEV), cfg.E)
     R = cfg.rows()
-    o = torch.randn((R, cfg.d), generator=torch.Generator().manual_seed(cfg.seed))
+    o = torch.randn((R, cfg.d), generator=torch.Generator().manual_seed(cfg.seed)).half()
     w = random_weights(cfg.T, cfg.k, seed=cfg.seed)
     y = torch.empty((cfg.T, cfg.d), dtype=torch.bfloat16, device=DEV)
     M.combine(M.shape_of(cfg), o.to(DEV), inv, w.to(DEV), _u16(y))
@@ -278,9 +301,9 @@ def test_gemm_down_fp8(cfg):
     hq = torch.empty((R, cfg.I), dtype=torch.uint8, device=DEV)
     hs = torch.empty((R, cfg.I // 128), dtype=torch.float32, device=DEV)
     M.quantize_act_fp8(_u16(hin.to(DEV)), hq, hs)
-    o = torch.empty((R, cfg.d), dtype=torch.float32, device=DEV)
+    o = torch.empty((R, cfg.d), dtype=torch.float16, device=DEV)
     M.gemm_down(layer.shape(cfg.T), layer.weights, hq, hs, offsets, o, layer.ws)
     assert M.read_device_status(layer.ws) == M.OK
     _, ooff, _, _ = oracle.permute(ids.numpy(), cfg.E)
     ref = oracle.down(oracle_layer(cfg, inp), bf16_to_f64(hin), ooff, cfg.T)
-    assert_close_rel(o.cpu().double().numpy(), ref, rtol=1e-4, atol=1e-4 * rms(ref), what="o")
+    assert_close_rel(o.cpu().double().numpy(), ref, rtol=O_RTOL, atol=1e-4 * rms(ref), what="o")
