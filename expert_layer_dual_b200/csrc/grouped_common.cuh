@@ -4,10 +4,13 @@
 // owns rows offsets[g] .. offsets[g+1]-1 (the contiguous per-expert interval
 // of the routing stage), the shared expert owns rows T*k .. T*k+T-1.  A group
 // of n rows has ceil(n / 128) m-tiles; every group has the same number of
-// n-tiles.  Tiles are numbered group by group, and inside a group n-tile by
-// n-tile with the m-tiles innermost, so tiles with neighbouring numbers share
-// weight tiles.  The host never learns the counts: each CTA rebuilds the
-// m-tile prefix from `offsets` in its prologue.
+// n-tiles.  Tiles are numbered group by group; inside a group, the m-tiles
+// are taken in blocks of kMBlock, and each block runs n-tile by n-tile with
+// its m-tiles innermost.  Tiles with neighbouring numbers therefore share a
+// weight tile, and the rows of one block (a few MB) stay in L2 while they are
+// read once per n-tile; a group of at most kMBlock m-tiles is one block.
+// The host never learns the counts: each CTA rebuilds the m-tile prefix from
+// `offsets` in its prologue.
 //
 // Tiles are handed out dynamically: the producer of each CTA takes the next
 // number from a global counter when it is ready for a new tile and publishes
@@ -23,6 +26,7 @@
 namespace moe {
 
 constexpr int kMaxGroups = 257;  // 256 routed + 1 shared
+constexpr int kMBlock = 8;       // m-tiles per block of a large group
 
 struct TileTable {
     int32_t goff[kMaxGroups + 1];     // first row of each group, goff[G] = end
@@ -74,8 +78,11 @@ __device__ __forceinline__ Tile decode_tile(const TileTable* tt, int G, int n_ti
     t.g = lo;
     const int mt = tt->mstart[lo + 1] - tt->mstart[lo];
     const int local = tile - tt->mstart[lo] * n_tiles;
-    t.n = local / mt;
-    const int m = local - t.n * mt;
+    const int blk = local / (kMBlock * n_tiles);      // block of m-tiles
+    const int mb = min(kMBlock, mt - blk * kMBlock);  // m-tiles in this block
+    const int r = local - blk * kMBlock * n_tiles;
+    t.n = r / mb;
+    const int m = blk * kMBlock + (r - t.n * mb);
     t.row0 = tt->goff[lo] + m * BM;
     const int rows = tt->goff[lo + 1] - tt->goff[lo];
     t.nrows = min(BM, rows - m * BM);
