@@ -151,6 +151,34 @@ def test_forward_host_async_pipelined_over_two_streams():
     assert M.read_device_status(wss[0]) == M.OK and M.read_device_status(wss[1]) == M.OK
 
 
+@pytest.mark.parametrize("cfg", [SMALL[1], SMALL[6], SMALL[8], SMALL[10]],
+                         ids=lambda c: c.name)
+def test_forward_cuda_graph_replay_equals_eager(cfg):
+    # moe_forward captured once in a CUDA graph (as bench.py times it): a replay
+    # reads the input buffer as it is at replay time and writes the eager result
+    inp = make_layer(cfg)
+    layer = M.MoELayer(cfg, inp)
+    xa = inp["x"].to(DEV)
+    xb = torch.flip(inp["x"], dims=[0]).contiguous().to(DEV)
+    ref_a, ref_b = layer.forward(xa).clone(), layer.forward(xb).clone()
+    x = xa.clone()
+    y = torch.empty_like(x)
+    shape = layer.shape(cfg.T)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        M.forward(shape, layer.weights, x.view(torch.uint16), y.view(torch.uint16), layer.ws)
+    graph.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(y, ref_a)
+    x.copy_(xb)
+    graph.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(y, ref_b)
+    assert layer.device_status() == M.OK
+    del graph
+
+
 def test_token_count_below_capacity_and_zero():
     cfg = SMALL[1]
     inp = make_layer(cfg)
