@@ -74,10 +74,14 @@ def test_algorithmic_work_of_the_gemms():
     assert CONFIGS["prefill"].flops() == pytest.approx(2.82e12, rel=0.01)
 
 
-def test_peak_regime_follows_the_power_cap_and_region_length():
-    assert bench.power_capped({"reasons": ["sw_power_cap"]}, 50.0)
-    assert not bench.power_capped({"reasons": []}, 50.0)
-    assert bench.power_capped({"reasons": []}, 800.0)
+def test_peak_regime_follows_the_clock_under_load():
+    capped = {"sm_mhz": 1342.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]}
+    flagged_full_clock = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]}
+    assert bench.power_capped(capped, 50.0)
+    assert not bench.power_capped(flagged_full_clock, 800.0)
+    # without clock samples, the length of the timed region decides
+    assert not bench.power_capped({"sm_mhz": None, "sm_max_mhz": None, "reasons": []}, 50.0)
+    assert bench.power_capped({"sm_mhz": None, "sm_max_mhz": None, "reasons": []}, 800.0)
     hbm, burst, _ = bench.load_peaks(False)
     _, sustained, _ = bench.load_peaks(True)
     assert sustained <= burst and hbm > 0
