@@ -17,9 +17,10 @@
 //    of both CTAs; the epilogue warps of the other CTA signal the leader's
 //    accumulator barrier through cluster-mapped addresses.
 // Measured on B200: +15% over the one-CTA kernel on a dense 16384-row problem,
-// +8% on the skewed workload (~512 rows per expert), but -10% at ~256 rows
-// per expert, where 256-row tiles pad more; so it serves >= 512 rows per
-// expert on average.  Every wait is bounded, as in the one-CTA kernels.
+// +8% on the skewed workload, +3% at ~256 rows per expert (prefill; with FP16
+// expert outputs -- it was -10% with FP32 rows, where 256-row tiles pad more)
+// and much slower at a few rows per expert (decode); so it serves >= 256 rows
+// per expert on average.  Every wait is bounded, as in the one-CTA kernels.
 #include "common.cuh"
 #include "grouped_common.cuh"
 #include "launch.h"

@@ -95,8 +95,8 @@ cudaError_t launch_down_bf16(const GroupedGemmArgs& a, const uint16_t* h, const 
 // ---- gemm_bf16_2sm.cu (down GEMM on CTA-pair tiles of 256 rows)
 cudaError_t launch_down_bf16_2sm(const GroupedGemmArgs& a, const uint16_t* h, const uint16_t* w_d,
                                  const uint16_t* ws_d, __half* o, cudaStream_t s);
-// Whether the CTA-pair down kernel serves this shape (>= 512 rows per expert on average).
-inline bool use_pair_tiles(int T, int E, int k) { return (int64_t)T * k >= (int64_t)512 * E; }
+// Whether the CTA-pair down kernel serves this shape (>= 256 rows per expert on average).
+inline bool use_pair_tiles(int T, int E, int k) { return (int64_t)T * k >= (int64_t)256 * E; }
 
 // ---- gemm_fp8.cu (tcgen05 grouped GEMMs, e4m3 with 128x128 block scales)
 cudaError_t launch_gateup_fp8(const GroupedGemmArgs& a, const uint8_t* xq, const float* xs,

@@ -32,7 +32,7 @@ SMALL = [
     MoEConfig("ragged", T=300, d=512, E=16, k=4, I=256, Is=256, seed=21),
     MoEConfig("odd", T=203, d=384, E=40, k=8, I=128, Is=128, seed=22),
     MoEConfig("wide", T=130, d=256, E=256, k=8, I=128, Is=128, seed=23),
-    # >= 512 rows per expert on average: the down GEMM runs on CTA pairs
+    # >= 256 rows per expert on average: the down GEMM runs on CTA pairs
     MoEConfig("pair", T=1100, d=512, E=8, k=4, I=256, Is=256, seed=27),
     MoEConfig("pairodd", T=1100, d=384, E=6, k=3, I=128, Is=128, seed=28),
 ]
