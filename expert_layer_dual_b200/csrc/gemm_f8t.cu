@@ -16,7 +16,7 @@
 // MMAs, and 4 epilogue warps:
 //  - gate-up: h = silu(s g) * (s u), s = s_x * s_w[e], quantised with the
 //    static scale of h (e4m3 of fp32(h / s_h), saturating);
-//  - down: o = s_h * s_w[e] * acc, FP32 rows.
+//  - down: o = s_h * s_w[e] * acc, stored as FP16 rows.
 // Every wait is bounded, as in the other kernels.
 #include "common.cuh"
 #include "grouped_common.cuh"
@@ -268,7 +268,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 }
 
 // ---------------------------------------------------------------------------
-// Down: o = s_h * s_w[e] * (hq . Wq), FP32 rows.
+// Down: o = s_h * s_w[e] * (hq . Wq), stored as FP16 rows.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(THREADS, 1)
     k_down_f8t(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_w,

@@ -37,7 +37,7 @@
 // computes h = silu(g) * u, the group's amax (combining the four column
 // quarters through shared memory) and writes e4m3 h with its scale.  Down's
 // tile is 128 rows x 256 output columns (two weight scale blocks) and writes
-// FP32 o.  Every wait is bounded, as in the BF16 kernels.
+// o in FP16.  Every wait is bounded, as in the BF16 kernels.
 #include "common.cuh"
 #include "grouped_common.cuh"
 #include "launch.h"

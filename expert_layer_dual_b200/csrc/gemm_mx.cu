@@ -32,7 +32,7 @@
 //  - 16 epilogue warps drain the accumulator: gate-up computes
 //    h = silu(g) * u for 32 columns per thread -- exactly one MX block -- and
 //    writes e4m3 h with its E8M0 scale (no cross-thread amax); down writes
-//    FP32 o.  The accumulator is handed back as soon as it has been read.
+//    o in FP16.  The accumulator is handed back as soon as it has been read.
 // Every wait is bounded, as in the other kernels.
 #include "common.cuh"
 #include "grouped_common.cuh"
@@ -369,7 +369,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 }
 
 // ---------------------------------------------------------------------------
-// Down: o[p][n0 + j] = (MX h)[p] . (MX Wd)[n0 + j], FP32 rows.
+// Down: o[p][n0 + j] = (MX h)[p] . (MX Wd)[n0 + j], FP32 sums stored as FP16 rows.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(THREADS, 1)
     k_down_mx(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_w,

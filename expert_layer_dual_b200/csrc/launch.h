@@ -35,7 +35,7 @@ int permute_segments(int64_t n_assign);
 cudaError_t launch_permute(const int32_t* ids, int T, int E, int k, int32_t* counts,
                            int32_t* offsets, int32_t* perm, int32_t* inv, int32_t* seg_hist,
                            int32_t* status, cudaStream_t s);
-// o [R][d] f32: routed rows then (has_shared) the shared expert's rows
+// o [R][d] FP16: routed rows then (has_shared) the shared expert's rows
 cudaError_t launch_combine(const __half* o, const int32_t* inv, const float* w, uint16_t* y, int T,
                            int d, int k, int has_shared, cudaStream_t s);
 cudaError_t launch_quant_act_fp8(const uint16_t* x, int64_t rows, int cols, uint8_t* q,
