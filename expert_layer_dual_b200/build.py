@@ -19,7 +19,7 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libmoe_b200.so")
-SOURCES = ["api.cu", "routing.cu", "router.cu", "gemm_bf16.cu", "gemm_bf16_2sm.cu", "gemm_fp8.cu", "gemm_mx.cu", "gemm_f8t.cu",
+SOURCES = ["api.cu", "routing.cu", "router.cu", "gemm_bf16.cu", "gemm_bf16_wide.cu", "gemm_bf16_2sm.cu", "gemm_fp8.cu", "gemm_mx.cu", "gemm_f8t.cu",
            "noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-O2",

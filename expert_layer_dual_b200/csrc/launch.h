@@ -92,6 +92,14 @@ cudaError_t launch_gateup_bf16(const GroupedGemmArgs& a, const uint16_t* x, cons
 cudaError_t launch_down_bf16(const GroupedGemmArgs& a, const uint16_t* h, const uint16_t* w_d,
                              const uint16_t* ws_d, __half* o, cudaStream_t s);
 
+// ---- gemm_bf16_wide.cu (gate-up with 256-row tiles: two accumulators share each weight stage)
+cudaError_t launch_gateup_bf16_wide(const GroupedGemmArgs& a, const uint16_t* x,
+                                    const uint16_t* w_gu, const uint16_t* ws_gu, uint16_t* h,
+                                    cudaStream_t s);
+// Whether the 256-row gate-up serves this shape: >= 512 rows per expert on average and
+// at least ~20 waves of its tiles.
+bool use_wide_gateup(int T, int E, int k, int I, int has_shared);
+
 // ---- gemm_bf16_2sm.cu (down GEMM on CTA-pair tiles of 256 rows)
 cudaError_t launch_down_bf16_2sm(const GroupedGemmArgs& a, const uint16_t* h, const uint16_t* w_d,
                                  const uint16_t* ws_d, __half* o, cudaStream_t s);

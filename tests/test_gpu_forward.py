@@ -15,7 +15,8 @@ import torch
 import oracle
 from expert_layer_dual_b200.configs import CONFIGS, MoEConfig
 from expert_layer_dual_b200.inputs import make_layer
-from gpu_util import ambiguous_tokens, bf16_to_f64, bits, logit_rel_error, oracle_layer, row_scale, rms
+from gpu_util import (ambiguous_tokens, assert_close_rel, bf16_to_f64, bits, logit_rel_error,
+                      oracle_layer, row_scale, rms)
 
 pytestmark = pytest.mark.gpu
 
@@ -266,6 +267,49 @@ def _full_size_case(name, n_sample):
                                     ("fp8t", 4)])
 def test_forward_full_size(name, n):
     _full_size_case(name, n)
+
+
+def test_gemm_gateup_full_size_wide_tiles_on_sampled_rows():
+    # On the skewed workload (>= 512 rows per expert on average, many tiles) the BF16
+    # gate-up runs on 256-row tiles (two accumulators per tile).  Sampled rows of h,
+    # including rows 128-255 of a tile, rows of a tail tile of at most 128 rows and the
+    # shared expert's rows, against the oracle's gate-up of that one token with that
+    # one expert's weights.
+    cfg = CONFIGS["skew"]
+    inp = make_layer(cfg, device=DEV)
+    layer = M.MoELayer(cfg, inp)
+    x = inp["x"]
+    st = _stage_outputs(layer, cfg, x)
+    R = cfg.rows()
+    h = torch.empty((R, cfg.I), dtype=torch.bfloat16, device=DEV)
+    M.gemm_gateup(layer.shape(cfg.T), layer.weights, x.view(torch.uint16), None, st["perm"],
+                  st["offsets"], h.view(torch.uint16), None, layer.ws)
+    assert M.read_device_status(layer.ws) == M.OK
+    offsets = st["offsets"].cpu().numpy()
+    perm = st["perm"].cpu().numpy()
+    Tk = cfg.T * cfg.k
+    goff = np.concatenate([offsets, [R]])                   # the shared group last
+    rng = np.random.default_rng(5)
+    sizes = np.diff(goff)
+    rows = []
+    groups = {int(np.argmax(sizes[:cfg.E])), cfg.E}            # the largest expert, the shared one
+    groups |= set(rng.choice(np.nonzero(sizes[:cfg.E])[0], 5, replace=False).tolist())
+    for g in sorted(groups):
+        n = int(goff[g + 1] - goff[g])
+        for r in {0, min(n - 1, 127), min(n - 1, 128), min(n - 1, 255), n - 1}:
+            if 0 <= r < n:
+                rows.append((g, int(goff[g]) + r))
+    hb = bf16_to_f64(h[torch.as_tensor([p for _, p in rows], device=DEV)])
+    for i, (g, p) in enumerate(rows):
+        tok = perm[p] // cfg.k if p < Tk else p - Tk
+        w_gu = bits(inp["ws_gu"])[None] if g == cfg.E else bits(inp["w_gu"][g])[None]
+        L = oracle.Layer(T=1, d=cfg.d, E=1, k=1, I=cfg.I, Is=0, w_gu=w_gu,
+                         w_d=np.zeros((1, cfg.d, cfg.I), np.uint16), ws_gu=None, ws_d=None,
+                         router_w=np.zeros((1, cfg.d), np.float32), wdtype=0)
+        ref = oracle.gateup(L, bits(x[int(tok)])[None], np.zeros(1, np.int32),
+                            np.array([0, 1], np.int32))
+        assert_close_rel(hb[i][None], ref, rtol=2.0 ** -8, atol=1e-3 * rms(ref),
+                         what=f"h row {p} (group {g})")
 
 
 def test_forward_full_size_skew():
