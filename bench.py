@@ -182,6 +182,7 @@ def power_capped(clocks: dict, ms_total: float) -> bool:
 # hash of the kernel's sources; reported only while the sources still match.
 KERNEL_SOURCES = {
     "k_gateup_bf16": ["csrc/gemm_bf16.cu", "csrc/common.cuh", "csrc/grouped_common.cuh"],
+    "k_gateup_bf16_wide": ["csrc/gemm_bf16_wide.cu", "csrc/common.cuh", "csrc/grouped_common.cuh"],
     "k_gateup_fp8": ["csrc/gemm_fp8.cu", "csrc/common.cuh", "csrc/grouped_common.cuh"],
     "k_gateup_mx": ["csrc/gemm_mx.cu", "csrc/common.cuh", "csrc/grouped_common.cuh"],
     "k_gateup_f8t": ["csrc/gemm_f8t.cu", "csrc/common.cuh", "csrc/grouped_common.cuh"],
@@ -210,6 +211,16 @@ def recorded_traffic(kernel: str, workload: str):
                 return None, "kernel changed since the capture"
             return int(parts[2]), "ncu capture, profiles/dram_traffic.txt"
     return None, "no capture for this workload"
+
+
+def gateup_kernel(cfg: MoEConfig, T: int, num_sms: int) -> str:
+    """Name of the gate-up kernel moe_forward launches for this shape: the
+    library's dispatch rule (use_wide_gateup in gemm_bf16_wide.cu) for BF16."""
+    if cfg.wdtype != 0:
+        return "k_gateup_" + {1: "fp8", 2: "mx", 3: "f8t"}[cfg.wdtype]
+    rows = T * cfg.k + (T if cfg.Is > 0 else 0)
+    wide = T * cfg.k >= 512 * cfg.E and rows // 256 * (cfg.I // 128) >= 20 * num_sms
+    return "k_gateup_bf16_wide" if wide else "k_gateup_bf16"
 
 
 def gateup_algorithmic(cfg: MoEConfig, T: int, n_active: int):
@@ -425,7 +436,7 @@ def run_ours(args, cfg: MoEConfig):
         roof = {"bound": "tensor", "achieved": gu_flops / (gu_ms / 1e3) / 1e12, "peak": peak,
                 "unit": "TFLOP/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["kernel"] = "k_gateup_" + {0: "bf16", 1: "fp8", 2: "mx", 3: "f8t"}[cfg.wdtype]
+    roof["kernel"] = gateup_kernel(cfg, cfg.T, torch.cuda.get_device_properties(dev).multi_processor_count)
     tf_key = ("bf16_tflops_sustained (the SM clock sat below 90% of its maximum)" if sustained
               else "bf16_tflops (burst: the SM clock stayed at its maximum)")
     roof["peak_source"] = (f"{peak_kind} MEASURED_PEAKS.json "
