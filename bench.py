@@ -215,12 +215,11 @@ def recorded_traffic(kernel: str, workload: str):
 
 def gateup_kernel(cfg: MoEConfig, T: int, num_sms: int) -> str:
     """Name of the gate-up kernel moe_forward launches for this shape: the
-    library's dispatch rule (use_wide_gateup in gemm_bf16_wide.cu) for BF16."""
+    library's dispatch rule (use_wide_gateup in launch.h) for BF16."""
+    del num_sms
     if cfg.wdtype != 0:
         return "k_gateup_" + {1: "fp8", 2: "mx", 3: "f8t"}[cfg.wdtype]
-    rows = T * cfg.k + (T if cfg.Is > 0 else 0)
-    wide = T * cfg.k >= 512 * cfg.E and rows // 256 * (cfg.I // 128) >= 20 * num_sms
-    return "k_gateup_bf16_wide" if wide else "k_gateup_bf16"
+    return "k_gateup_bf16_wide" if T * cfg.k >= 256 * cfg.E else "k_gateup_bf16"
 
 
 def gateup_algorithmic(cfg: MoEConfig, T: int, n_active: int):

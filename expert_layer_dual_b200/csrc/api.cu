@@ -204,9 +204,8 @@ moe_status run_gateup(const moe_shape* s, const moe_weights* w, const void* x, c
                       int32_t* status, cudaStream_t st) {
     const GroupedGemmArgs a = gemm_args(s, offsets, perm, status);
     if (s->wdtype == MOE_WDTYPE_BF16)
-        return cuda_status((use_wide_gateup(s->T, s->E, s->k, s->I, s->I_shared > 0 ? 1 : 0)
-                                ? launch_gateup_bf16_wide
-                                : launch_gateup_bf16)(
+        return cuda_status((use_wide_gateup(s->T, s->E, s->k) ? launch_gateup_bf16_wide
+                                                              : launch_gateup_bf16)(
             a, static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(w->w_gu),
             static_cast<const uint16_t*>(w->ws_gu), static_cast<uint16_t*>(h), st));
     if (s->wdtype == MOE_WDTYPE_FP8_TENSOR)

@@ -14,11 +14,10 @@
 // 1.5x fewer bytes per FLOP; the two accumulators fill TMEM, so a tile's
 // epilogue does not overlap the next tile's MMAs, and 256-row tiles leave
 // more of the last wave idle.  Measured on B200 with the bench's CUDA-graph
-// timing: 4% faster per step on the skewed workload (experts of up to 8209
-// rows), 0-4% slower at prefill (~256 rows per expert: the second tile of an
-// expert is mostly empty), equal on a dense 16384-row problem and 5% slower
-// with ~800 tiles in all; so it serves shapes with at least 512 rows per
-// expert on average and ~20 waves of tiles.
+// timing, against the 128-row kernel, both with the fast SiLU: 4-7% faster
+// per step at prefill (~256 rows per expert), 3% on the skewed workload,
+// 2-3% with ~512 rows per expert, 1-7% on a dense 16384-row problem; so it
+// serves shapes with at least 256 rows per expert on average.
 //  - persistent, one CTA per SM, tiles from the dynamic schedule of
 //    grouped_common.cuh;
 //  - three 64 KB stages: 256 rows gathered from x through the permutation by
@@ -296,13 +295,6 @@ __global__ void __launch_bounds__(THREADS, 1)
 bool g_smem_set[64] = {false};
 
 }  // namespace
-
-bool use_wide_gateup(int T, int E, int k, int I, int has_shared) {
-    const int64_t rows = (int64_t)T * k + (has_shared ? T : 0);
-    const int64_t min_tiles = rows / BM * (I / 128);  // without padding: a lower bound
-    return (int64_t)T * k >= (int64_t)512 * E &&
-           min_tiles >= (int64_t)20 * current_device_info().num_sms;
-}
 
 cudaError_t launch_gateup_bf16_wide(const GroupedGemmArgs& a, const uint16_t* x,
                                     const uint16_t* w_gu, const uint16_t* ws_gu, uint16_t* h,

@@ -96,9 +96,8 @@ cudaError_t launch_down_bf16(const GroupedGemmArgs& a, const uint16_t* h, const 
 cudaError_t launch_gateup_bf16_wide(const GroupedGemmArgs& a, const uint16_t* x,
                                     const uint16_t* w_gu, const uint16_t* ws_gu, uint16_t* h,
                                     cudaStream_t s);
-// Whether the 256-row gate-up serves this shape: >= 512 rows per expert on average and
-// at least ~20 waves of its tiles.
-bool use_wide_gateup(int T, int E, int k, int I, int has_shared);
+// Whether the 256-row gate-up serves this shape (>= 256 rows per expert on average).
+inline bool use_wide_gateup(int T, int E, int k) { return (int64_t)T * k >= (int64_t)256 * E; }
 
 // ---- gemm_bf16_2sm.cu (down GEMM on CTA-pair tiles of 256 rows)
 cudaError_t launch_down_bf16_2sm(const GroupedGemmArgs& a, const uint16_t* h, const uint16_t* w_d,

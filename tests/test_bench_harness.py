@@ -90,8 +90,8 @@ def test_peak_regime_follows_the_clock_under_load():
 def test_gateup_kernel_follows_the_library_dispatch():
     from expert_layer_dual_b200.configs import CONFIGS
     names = {n: bench.gateup_kernel(CONFIGS[n], CONFIGS[n].T, 148) for n in CONFIGS}
-    assert names["decode"] == names["prefill"] == "k_gateup_bf16"
-    assert names["skew"] == "k_gateup_bf16_wide"
+    assert names["decode"] == names["tiny"] == "k_gateup_bf16"
+    assert names["prefill"] == names["skew"] == "k_gateup_bf16_wide"
     assert names["fp8"] == "k_gateup_fp8" and names["mxfp8"] == "k_gateup_mx"
     assert names["fp8t"] == "k_gateup_f8t"
     assert set(names.values()) <= set(bench.KERNEL_SOURCES)
