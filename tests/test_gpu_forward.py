@@ -32,6 +32,10 @@ SMALL = [
     MoEConfig("wide", T=130, d=256, E=256, k=8, I=128, Is=128, seed=23),
     MoEConfig("skewbias", T=150, d=256, E=64, k=8, I=128, Is=128, zipf_bias=True, seed=25),
     MoEConfig("norenorm", T=64, d=256, E=32, k=4, I=128, Is=0, renorm=False, seed=26),
+    # >= 256 rows per expert on average: 256-row gate-up tiles and CTA-pair down tiles
+    MoEConfig("manyrows", T=600, d=384, E=8, k=4, I=256, Is=256, seed=28),
+    # 241..282 rows per expert: tiles whose second 128-row half is empty, and 3 N tiles
+    MoEConfig("manyedge", T=520, d=256, E=8, k=4, I=384, Is=0, seed=29),
     MoEConfig("fp8small", T=200, d=512, E=16, k=4, I=256, Is=256, wdtype=1, seed=31),
     MoEConfig("fp8odd", T=77, d=384, E=8, k=2, I=128, Is=0, wdtype=1, seed=32),
     MoEConfig("mxsmall", T=200, d=512, E=16, k=4, I=256, Is=256, wdtype=2, seed=33),
@@ -39,6 +43,7 @@ SMALL = [
     MoEConfig("f8tsmall", T=200, d=512, E=16, k=4, I=256, Is=256, wdtype=3, seed=35),
     MoEConfig("f8todd", T=77, d=384, E=8, k=2, I=128, Is=0, wdtype=3, seed=36),
 ]
+BY_NAME = {c.name: c for c in SMALL}
 
 
 def _stage_outputs(layer, cfg, x_dev):
@@ -121,7 +126,7 @@ def test_forward_small(cfg):
 
 
 def test_forward_host_matches_device():
-    cfg = SMALL[1]
+    cfg = BY_NAME["ragged"]
     inp = make_layer(cfg)
     layer = M.MoELayer(cfg, inp)
     y_dev = layer.forward(inp["x"].to(DEV))
@@ -134,7 +139,7 @@ def test_forward_host_matches_device():
 def test_forward_host_async_pipelined_over_two_streams():
     # batches alternate over two streams with one workspace each; every result
     # equals the device forward of its own batch
-    cfg = SMALL[1]
+    cfg = BY_NAME["ragged"]
     inp = make_layer(cfg)
     layer = M.MoELayer(cfg, inp)
     xs = [inp["x"], torch.flip(inp["x"], dims=[0]).contiguous(), inp["x"] * 0.5]
@@ -152,7 +157,8 @@ def test_forward_host_async_pipelined_over_two_streams():
     assert M.read_device_status(wss[0]) == M.OK and M.read_device_status(wss[1]) == M.OK
 
 
-@pytest.mark.parametrize("cfg", [SMALL[1], SMALL[6], SMALL[8], SMALL[10]],
+@pytest.mark.parametrize("cfg", [BY_NAME[n] for n in ("ragged", "manyrows", "fp8small",
+                                                      "mxsmall", "f8tsmall")],
                          ids=lambda c: c.name)
 def test_forward_cuda_graph_replay_equals_eager(cfg):
     # moe_forward captured once in a CUDA graph (as bench.py times it): a replay
@@ -181,7 +187,7 @@ def test_forward_cuda_graph_replay_equals_eager(cfg):
 
 
 def test_token_count_below_capacity_and_zero():
-    cfg = SMALL[1]
+    cfg = BY_NAME["ragged"]
     inp = make_layer(cfg)
     layer = M.MoELayer(cfg, inp)
     x = inp["x"].to(DEV)
@@ -194,7 +200,7 @@ def test_token_count_below_capacity_and_zero():
 
 
 def test_status_and_validation_paths():
-    cfg = SMALL[0]
+    cfg = BY_NAME["tiny"]
     inp = make_layer(cfg)
     layer = M.MoELayer(cfg, inp)
     # a bounded wait that nothing completes reports a timeout and leaves the context usable
