@@ -285,9 +285,8 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float* f) {
     }
 }
 
-// acc[i] += wj * row[i] for the 8 FP16 values of one 16-byte load.
-__device__ __forceinline__ void add8(float* acc, const __half* row, float wj) {
-    const uint4 u = __ldg(reinterpret_cast<const uint4*>(row));
+// acc[i] += wj * row[i] for the 8 FP16 values of one 16-byte load u.
+__device__ __forceinline__ void add8(float* acc, const uint4 u, float wj) {
     const uint32_t r[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -311,15 +310,23 @@ __global__ void __launch_bounds__(128)
     __syncthreads();
     const int64_t shared_row = (int64_t)T * k + t;
     for (int c = threadIdx.x * 8; c < d; c += blockDim.x * 8) {
+        // all k (+1) rows' loads first, so they are in flight together
+        uint4 u[9];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            if (j < k) u[j] = __ldg(reinterpret_cast<const uint4*>(o + (int64_t)rows[j] * d + c));
+        if (has_shared) u[8] = __ldg(reinterpret_cast<const uint4*>(o + shared_row * d + c));
         float acc[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
-        for (int j = 0; j < k; ++j) add8(acc, o + (int64_t)rows[j] * d + c, wts[j]);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            if (j < k) add8(acc, u[j], wts[j]);
         if (has_shared) {
             float sh[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) sh[i] = 0.0f;
-            add8(sh, o + shared_row * d + c, 1.0f);
+            add8(sh, u[8], 1.0f);
 #pragma unroll
             for (int i = 0; i < 8; ++i) acc[i] += sh[i];
         }
