@@ -48,11 +48,11 @@ cudaError_t launch_router_split(const float* W, uint16_t* hi, uint16_t* lo, int6
 }
 
 // ---------------------------------------------------------------------------
-// Top-k routing: one warp per token; lane l holds logits l, l+32, ... (E <=
-// 256).  k rounds of a warp arg-max over (value desc, id asc) -- a total
-// order, so every lane converges to the same winner -- select the experts in
-// descending order with ties to the lower id.  Weights: softmax over the
-// selected logits (or over all E when renorm == 0), in FP32.
+// Top-k routing: one warp selects for a token; lane l holds logits l, l+32,
+// ... (E <= 256).  k rounds of a warp arg-max over (value desc, id asc) -- a
+// total order, so every lane converges to the same winner -- select the
+// experts in descending order with ties to the lower id.  Weights: softmax
+// over the selected logits (or over all E when renorm == 0), in FP32.
 // ---------------------------------------------------------------------------
 constexpr int kTopkWarps = 8;
 
@@ -65,37 +65,11 @@ __device__ __forceinline__ float sum_partials(const float* p, int64_t stride, in
            ((p[4 * stride] + p[5 * stride]) + (p[6 * stride] + p[7 * stride]));
 }
 
-__global__ void __launch_bounds__(kTopkWarps * 32)
-    k_route_topk(const float* __restrict__ logits_in, const float* __restrict__ part_hi,
-                 const float* __restrict__ part_lo, int ksplit, const float* __restrict__ bias,
-                 float* __restrict__ logits_out, int T, int E, int k, int renorm,
-                 int32_t* __restrict__ ids, float* __restrict__ w) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int t = blockIdx.x * kTopkWarps + warp;
-    if (t >= T) return;
-    float v[8];
-    uint32_t taken = 0;
-    const int64_t pstride = (int64_t)T * E;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int e = lane + 32 * i;
-        if (e < E) {
-            if (part_hi != nullptr) {
-                // split-K router: hi sums + lo sums / 256 (one FMA) + bias
-                const int64_t off = (int64_t)t * E + e;
-                float x = fmaf(sum_partials(part_lo + off, pstride, ksplit), 0.00390625f,
-                               sum_partials(part_hi + off, pstride, ksplit));
-                if (bias != nullptr) x += bias[e];
-                logits_out[off] = x;
-                v[i] = x;
-            } else {
-                v[i] = logits_in[(int64_t)t * E + e];
-            }
-        } else {
-            v[i] = 0.0f;
-            taken |= 1u << i;
-        }
-    }
+// The warp's k selections from the logits v[i] of experts lane + 32 i (bits
+// of `taken` mark absent experts), then the routing weights of token t.
+__device__ __forceinline__ void select_topk(const float (&v)[8], uint32_t taken, int lane, int t,
+                                            int E, int k, int renorm, int32_t* __restrict__ ids,
+                                            float* __restrict__ w) {
     float my_v = 0.0f;
     int my_e = 0;
     for (int j = 0; j < k; ++j) {
@@ -145,6 +119,80 @@ __global__ void __launch_bounds__(kTopkWarps * 32)
     }
 }
 
+// A warp per token: the logits in memory (one router pass), or the sums of
+// the split-K router partials.
+__global__ void __launch_bounds__(kTopkWarps * 32)
+    k_route_topk(const float* __restrict__ logits_in, const float* __restrict__ part_hi,
+                 const float* __restrict__ part_lo, int ksplit, const float* __restrict__ bias,
+                 float* __restrict__ logits_out, int T, int E, int k, int renorm,
+                 int32_t* __restrict__ ids, float* __restrict__ w) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t = blockIdx.x * kTopkWarps + warp;
+    if (t >= T) return;
+    float v[8];
+    uint32_t taken = 0;
+    const int64_t pstride = (int64_t)T * E;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int e = lane + 32 * i;
+        if (e < E) {
+            if (part_hi != nullptr) {
+                // split-K router: hi sums + lo sums / 256 (one FMA) + bias
+                const int64_t off = (int64_t)t * E + e;
+                float x = fmaf(sum_partials(part_lo + off, pstride, ksplit), 0.00390625f,
+                               sum_partials(part_hi + off, pstride, ksplit));
+                if (bias != nullptr) x += bias[e];
+                logits_out[off] = x;
+                v[i] = x;
+            } else {
+                v[i] = logits_in[(int64_t)t * E + e];
+            }
+        } else {
+            v[i] = 0.0f;
+            taken |= 1u << i;
+        }
+    }
+    select_topk(v, taken, lane, t, E, k, renorm, ids, w);
+}
+
+// Split-K partials with few tokens: one block per token, one thread per
+// expert, so each logit's partial loads are all in flight at once; the
+// logits then go through shared memory to warp 0, which selects as above.
+__global__ void __launch_bounds__(256)
+    k_route_topk_sum(const float* __restrict__ part_hi, const float* __restrict__ part_lo,
+                     int ksplit, const float* __restrict__ bias, float* __restrict__ logits_out,
+                     int T, int E, int k, int renorm, int32_t* __restrict__ ids,
+                     float* __restrict__ w) {
+    __shared__ float lg[256];
+    const int t = blockIdx.x, e = threadIdx.x;
+    const int64_t pstride = (int64_t)T * E;
+    if (e < E) {
+        // hi sums + lo sums / 256 (one FMA) + bias
+        const int64_t off = (int64_t)t * E + e;
+        float x = fmaf(sum_partials(part_lo + off, pstride, ksplit), 0.00390625f,
+                       sum_partials(part_hi + off, pstride, ksplit));
+        if (bias != nullptr) x += bias[e];
+        logits_out[off] = x;
+        lg[e] = x;
+    }
+    __syncthreads();
+    if (threadIdx.x >= 32) return;
+    const int lane = threadIdx.x;
+    float v[8];
+    uint32_t taken = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int ei = lane + 32 * i;
+        if (ei < E) {
+            v[i] = lg[ei];
+        } else {
+            v[i] = 0.0f;
+            taken |= 1u << i;
+        }
+    }
+    select_topk(v, taken, lane, t, E, k, renorm, ids, w);
+}
+
 cudaError_t launch_route_topk(const float* logits, int T, int E, int k, int renorm, int32_t* ids,
                               float* w, cudaStream_t s) {
     if (T == 0) return cudaSuccess;
@@ -157,8 +205,13 @@ cudaError_t launch_route_topk_partials(const float* part_hi, const float* part_l
                                        const float* bias, float* logits, int T, int E, int k,
                                        int renorm, int32_t* ids, float* w, cudaStream_t s) {
     if (T == 0) return cudaSuccess;
-    k_route_topk<<<(T + kTopkWarps - 1) / kTopkWarps, kTopkWarps * 32, 0, s>>>(
-        nullptr, part_hi, part_lo, ksplit, bias, logits, T, E, k, renorm, ids, w);
+    // a block per token while a warp per token would leave most SMs idle
+    if (T <= 512)
+        k_route_topk_sum<<<T, 256, 0, s>>>(part_hi, part_lo, ksplit, bias, logits, T, E, k,
+                                           renorm, ids, w);
+    else
+        k_route_topk<<<(T + kTopkWarps - 1) / kTopkWarps, kTopkWarps * 32, 0, s>>>(
+            nullptr, part_hi, part_lo, ksplit, bias, logits, T, E, k, renorm, ids, w);
     return cudaGetLastError();
 }
 

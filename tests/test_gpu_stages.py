@@ -8,7 +8,9 @@ Tolerances (derived from the arithmetic):
     exact bf16 products against the FP64 sum);
   - top-k weights: 2e-6 absolute (FP32 exp and division of values <= 1);
   - bf16 outputs of one FP32-accumulated GEMM or sum: one bf16 rounding
-    (relative 2^-9) plus FP32 noise: rtol 2^-8, atol 1e-3 * rms(ref).
+    (8 significant bits: at most 2^-8 relative, reached just above a power of
+    two) plus FP32 noise (~1e-6 relative, inside the atol): rtol 2^-8,
+    atol 1e-3 * rms(ref).
 """
 import numpy as np
 import pytest
