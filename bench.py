@@ -222,6 +222,15 @@ def gateup_kernel(cfg: MoEConfig, T: int, num_sms: int) -> str:
     return "k_gateup_bf16_wide" if T * cfg.k >= 256 * cfg.E else "k_gateup_bf16"
 
 
+def kernels_per_step(cfg: MoEConfig, T: int) -> int:
+    """Kernels of this library one moe_forward launches, by its dispatch: the
+    router, the top-k, the permute (one kernel for at most 1024 assignments,
+    else count, scan and scatter), gate-up, down and combine, plus the
+    activation quantiser on the FP8 paths."""
+    permute = 1 if T * cfg.k <= 1024 else 3
+    return 5 + permute + (1 if cfg.wdtype else 0)
+
+
 def gateup_algorithmic(cfg: MoEConfig, T: int, n_active: int):
     """Algorithmic work of one gate-up launch: FLOPs, and bytes = the weights
     of every expert that received tokens (+ shared) read once, x read once,
@@ -495,7 +504,7 @@ def run_ours(args, cfg: MoEConfig):
                "sample": f"first {n} tokens of the {cfg.name} batch, whole layer in FP64, "
                          f"{len(times)} runs, {sum(times):.1f} s of CPU time"}
 
-    kernels_per_step = 8 + (1 if cfg.wdtype else 0)
+    launches_per_step = kernels_per_step(cfg, cfg.T)
     if rank == 0:
         out = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -512,7 +521,7 @@ def run_ours(args, cfg: MoEConfig):
             "roofline": roof,
             "cpu_baseline": cpu,
             "e2e": e2e,
-            "gpu_launches": kernels_per_step * args.steps,
+            "gpu_launches": launches_per_step * args.steps,
             "clocks": clocks.summary(),
             "stages_ms": stage_ms,
             "tflops": cfg.flops() / (ms_step / 1e3) / 1e12 * world,

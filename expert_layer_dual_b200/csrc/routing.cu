@@ -223,7 +223,8 @@ cudaError_t launch_route_topk_partials(const float* part_hi, const float* part_l
 // segment, the first output row of each expert; (3) each segment is placed
 // in order by one warp: __match_any_sync groups equal experts inside 32
 // consecutive assignments, the rank inside the group keeps the order stable.
-// No step depends on atomic ordering, so perm / inv are deterministic.
+// No step depends on atomic ordering, so perm / inv are deterministic.  A
+// single segment (at most kSeg assignments) runs all three in one block.
 // ---------------------------------------------------------------------------
 constexpr int kSeg = 1024;
 
@@ -309,18 +310,77 @@ __global__ void __launch_bounds__(32)
     }
 }
 
+// At most one segment (decode-sized batches): the three steps in one block --
+// the segment's histogram, the scan over experts, then warp 0 places the
+// assignments exactly as k_perm_scatter does, from the offsets.
+__global__ void __launch_bounds__(256)
+    k_perm_small(const int32_t* __restrict__ ids, int n, int E, int32_t* __restrict__ counts,
+                 int32_t* __restrict__ offsets, int32_t* __restrict__ perm,
+                 int32_t* __restrict__ inv, int32_t* status) {
+    __shared__ int32_t hist[256];
+    __shared__ int32_t buf[2][256];
+    const int e = threadIdx.x;
+    hist[e] = 0;
+    __syncthreads();
+    for (int a = threadIdx.x; a < n; a += blockDim.x) {
+        const int ea = ids[a];
+        if ((unsigned)ea < (unsigned)E)
+            atomicAdd(&hist[ea], 1);
+        else
+            report_status(status, MOE_ERR_DEVICE_BAD_INDEX);
+    }
+    __syncthreads();
+    const int32_t run = (e < E) ? hist[e] : 0;
+    if (e < E) counts[e] = run;
+    // inclusive Hillis-Steele scan of the totals over the 256 lanes
+    int cur = 0;
+    buf[0][e] = run;
+    __syncthreads();
+    for (int off = 1; off < 256; off <<= 1) {
+        const int32_t x = buf[cur][e] + (e >= off ? buf[cur][e - off] : 0);
+        buf[cur ^ 1][e] = x;
+        cur ^= 1;
+        __syncthreads();
+    }
+    const int32_t excl = buf[cur][e] - run;
+    if (e < E) {
+        offsets[e] = excl;
+        if (e == E - 1) offsets[E] = excl + run;
+    }
+    hist[e] = excl;  // every thread read its count above, before the scan's barriers
+    __syncthreads();
+    if (threadIdx.x >= 32) return;
+    const int lane = threadIdx.x;
+    for (int base = 0; base < n; base += 32) {
+        const int a = base + lane;
+        const int ea = (a < n) ? ids[a] : -1;
+        const bool ok = (unsigned)ea < (unsigned)E;
+        const unsigned peers = __match_any_sync(0xffffffffu, ok ? ea : -1 - lane);
+        int32_t start = 0;
+        if (ok) {
+            start = hist[ea];
+            const int32_t pos = start + __popc(peers & ((1u << lane) - 1u));
+            perm[pos] = a;
+            inv[a] = pos;
+        }
+        __syncwarp();
+        if (ok && lane == __ffs(peers) - 1) hist[ea] = start + __popc(peers);
+        __syncwarp();
+    }
+}
+
 cudaError_t launch_permute(const int32_t* ids, int T, int E, int k, int32_t* counts,
                            int32_t* offsets, int32_t* perm, int32_t* inv, int32_t* seg_hist,
                            int32_t* status, cudaStream_t s) {
     const int64_t n = (int64_t)T * k;
     const int nseg = permute_segments(n);
-    if (nseg > 0) {
-        k_perm_count<<<nseg, 256, 0, s>>>(ids, n, E, seg_hist, status);
+    if (nseg <= 1) {
+        k_perm_small<<<1, 256, 0, s>>>(ids, (int)n, E, counts, offsets, perm, inv, status);
+        return cudaGetLastError();
     }
+    k_perm_count<<<nseg, 256, 0, s>>>(ids, n, E, seg_hist, status);
     k_perm_scan<<<1, 256, 0, s>>>(seg_hist, nseg, E, counts, offsets);
-    if (nseg > 0) {
-        k_perm_scatter<<<nseg, 32, 0, s>>>(ids, n, E, seg_hist, perm, inv);
-    }
+    k_perm_scatter<<<nseg, 32, 0, s>>>(ids, n, E, seg_hist, perm, inv);
     return cudaGetLastError();
 }
 

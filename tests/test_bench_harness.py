@@ -95,3 +95,14 @@ def test_gateup_kernel_follows_the_library_dispatch():
     assert names["fp8"] == "k_gateup_fp8" and names["mxfp8"] == "k_gateup_mx"
     assert names["fp8t"] == "k_gateup_f8t"
     assert set(names.values()) <= set(bench.KERNEL_SOURCES)
+
+
+def test_launch_count_follows_the_library_dispatch():
+    from expert_layer_dual_b200.configs import CONFIGS
+    n = {k: bench.kernels_per_step(c, c.T) for k, c in CONFIGS.items()}
+    # router, top-k, the one-block permute (<= 1024 assignments), gate-up, down, combine
+    assert n["decode"] == n["tiny"] == 6
+    # the permute in three kernels (count, scan, scatter)
+    assert n["prefill"] == n["skew"] == 8
+    # + the activation quantiser
+    assert n["fp8"] == n["mxfp8"] == n["fp8t"] == 9
