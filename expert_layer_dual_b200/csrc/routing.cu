@@ -422,7 +422,8 @@ __global__ void __launch_bounds__(128)
     }
     __syncthreads();
     const int64_t shared_row = (int64_t)T * k + t;
-    for (int c = threadIdx.x * 8; c < d; c += blockDim.x * 8) {
+    // blockIdx.y splits the columns when there are few tokens
+    for (int c = (blockIdx.y * blockDim.x + threadIdx.x) * 8; c < d; c += gridDim.y * blockDim.x * 8) {
         // all k (+1) rows' loads first, so they are in flight together
         uint4 u[9];
 #pragma unroll
@@ -455,7 +456,12 @@ __global__ void __launch_bounds__(128)
 cudaError_t launch_combine(const __half* o, const int32_t* inv, const float* w, uint16_t* y, int T,
                            int d, int k, int has_shared, cudaStream_t s) {
     if (T == 0) return cudaSuccess;
-    k_combine<<<T, 128, 0, s>>>(o, inv, w, y, T, d, k, has_shared);
+    // with few tokens, several blocks per token (each a share of the 1024-column
+    // passes) so that about two blocks per SM have their loads in flight
+    const int passes = (d + 1023) / 1024;
+    const int want = (2 * current_device_info().num_sms + T - 1) / T;
+    const int ysplit = want < passes ? want : passes;
+    k_combine<<<dim3(T, ysplit > 1 ? ysplit : 1), 128, 0, s>>>(o, inv, w, y, T, d, k, has_shared);
     return cudaGetLastError();
 }
 
