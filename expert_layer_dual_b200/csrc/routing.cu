@@ -721,7 +721,36 @@ cudaError_t launch_quant_weights_fp8_tensor(const uint16_t* W, int64_t batch, in
     return cudaGetLastError();
 }
 
+// v / s rounded to nearest in FP32 -- the IEEE quotient -- for a divisor that
+// is the same for many values: with r the correctly rounded reciprocal of s,
+// the product v * r is corrected twice by its FMA residual (Markstein's
+// method).  It is used where every intermediate stays normal and finite:
+// 2^-100 <= |v| <= 2^100 and 2^-26 <= s <= 2^26, so the quotient lies within
+// [2^-126, 2^126]; elsewhere (and for NaN) the IEEE division itself.
+__device__ __forceinline__ float div_by_fixed(float v, float s, float r, bool s_in_range) {
+    const float a = fabsf(v);
+    if (!(s_in_range && a >= 0x1p-100f && a <= 0x1p100f)) return __fdiv_rn(v, s);
+    float q = v * r;
+    float e = fmaf(-q, s, v);
+    q = fmaf(e, r, q);
+    e = fmaf(-q, s, v);
+    return fmaf(e, r, q);
+}
+
+__device__ __forceinline__ uint32_t quant4_e4m3_fixed(float a, float b, float c, float d, float s,
+                                                      float r, bool s_in_range) {
+    const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(
+        make_float2(div_by_fixed(a, s, r, s_in_range), div_by_fixed(b, s, r, s_in_range)),
+        __NV_SATFINITE, __NV_E4M3);
+    const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(
+        make_float2(div_by_fixed(c, s, r, s_in_range), div_by_fixed(d, s, r, s_in_range)),
+        __NV_SATFINITE, __NV_E4M3);
+    return (uint32_t)lo | ((uint32_t)hi << 16);
+}
+
 // One warp per row, 8 values (16 bytes in, 8 bytes out) per lane per step.
+// The scale is the same for every value, so the division is done by its
+// reciprocal with the exact correction of div_by_fixed.
 __global__ void __launch_bounds__(256)
     k_quant_static(const uint16_t* __restrict__ x, const int32_t* __restrict__ perm, int T, int k,
                    int64_t rows, int cols, float s, uint8_t* __restrict__ q) {
@@ -732,12 +761,14 @@ __global__ void __launch_bounds__(256)
     const int64_t src_row = perm == nullptr ? p : (p < Tk ? (int64_t)(perm[p] / k) : p - Tk);
     const uint16_t* src = x + src_row * cols;
     uint8_t* dst = q + p * cols;
+    const float r = __frcp_rn(s);
+    const bool s_in_range = s >= 0x1p-26f && s <= 0x1p26f;
     for (int c = lane * 8; c < cols; c += 256) {
         float f[8];
         bf16x8_to_f32(*reinterpret_cast<const uint4*>(src + c), f);
         uint2 o;
-        o.x = quant4_e4m3(f[0], f[1], f[2], f[3], s);
-        o.y = quant4_e4m3(f[4], f[5], f[6], f[7], s);
+        o.x = quant4_e4m3_fixed(f[0], f[1], f[2], f[3], s, r, s_in_range);
+        o.y = quant4_e4m3_fixed(f[4], f[5], f[6], f[7], s, r, s_in_range);
         *reinterpret_cast<uint2*>(dst + c) = o;
     }
 }

@@ -62,6 +62,21 @@ def test_quantize_act_fp8_static_bit_exact(scale):
     assert np.array_equal(q.cpu().numpy(), oq)
 
 
+@pytest.mark.parametrize("scale", [2.0 ** -26, 3.1e-7, 1.7e-3, 0.0123, 5.1 / 448, 0.25, 1.0, 3.0,
+                                   777.7, 2.0 ** 26, 2.0 ** -27, 2.0 ** 27, 1.0e-30, 1.0e30])
+def test_quantize_act_fp8_static_every_bf16_value(scale):
+    # all 65536 bf16 bit patterns (zeros, subnormals, infinities and NaNs included):
+    # the static quantiser divides by its fixed scale through the reciprocal with two
+    # FMA corrections inside 2^-26 <= s <= 2^26 and 2^-100 <= |v| <= 2^100 (IEEE
+    # division elsewhere); its codes must equal the oracle's e4m3(fp32(v / s)) for all
+    bits16 = torch.arange(65536, dtype=torch.int32).to(torch.int16).view(torch.bfloat16)
+    x = bits16.reshape(512, 128).contiguous()
+    q = torch.empty((512, 128), dtype=torch.uint8, device=DEV)
+    M.quantize_act_fp8_static(_u16(x.to(DEV)), scale, q)
+    oq = oracle.quant_fp8_static(x.float().numpy(), np.float32(scale))
+    assert np.array_equal(q.cpu().numpy(), oq)
+
+
 @pytest.mark.parametrize("cfg", F8T, ids=IDS)
 def test_quantize_act_fp8_static_permuted_bit_exact(cfg):
     x = make_layer(cfg)["x"]
