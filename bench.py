@@ -92,24 +92,66 @@ def barrier():
 
 
 # ------------------------------------------------------------------ clocks
+def nvml_bus_id(dev) -> str:
+    """PCI bus id of a torch CUDA device in NVML's form (the index NVML and
+    nvidia-smi use need not be the CUDA index when CUDA_VISIBLE_DEVICES is set)."""
+    p = torch.cuda.get_device_properties(dev)
+    return f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+
+
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons while running."""
+    """SM clock, power and clock-event reasons of one GPU, sampled every
+    `period_s` by a thread reading NVML while the timed region runs (read
+    only: no setting of the GPU is touched).  Falls back to nvidia-smi's
+    100 ms loop when NVML is unavailable."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
+    def __init__(self, bus_id: str, period_s: float = 0.005):
+        self.bus_id = bus_id
+        self.period = period_s
+        self.lines = []
         self.proc = None
         self.path = None
+        self.thread = None
+        self.stop = False
+
+    def _nvml_loop(self, nv, h):
+        names = [("hw_slowdown", nv.nvmlClocksEventReasonHwSlowdown),
+                 ("hw_thermal_slowdown", nv.nvmlClocksEventReasonHwThermalSlowdown),
+                 ("sw_thermal_slowdown", nv.nvmlClocksEventReasonSwThermalSlowdown),
+                 ("sw_power_cap", nv.nvmlClocksEventReasonSwPowerCap)]
+        smax = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        while not self.stop:
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+            except nv.NVMLError:
+                break
+            flags = ["Active" if r & bit else "Not Active" for _, bit in names]
+            self.lines.append(", ".join(["0", str(sm), str(smax), f"{pw:.2f}", hex(r)] + flags))
+            time.sleep(self.period)
 
     def __enter__(self):
+        try:
+            import threading
+            import pynvml as nv
+            nv.nvmlInit()
+            h = nv.nvmlDeviceGetHandleByPciBusId(self.bus_id)
+            self.thread = threading.Thread(target=self._nvml_loop, args=(nv, h), daemon=True)
+            self.thread.start()
+            time.sleep(0.05)
+            return self
+        except Exception:  # noqa: BLE001 -- no NVML: sample with nvidia-smi instead
+            self.thread = None
         fd, self.path = tempfile.mkstemp(suffix=".csv")
         os.close(fd)
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-i", str(self.gpu), "-lms", "100"],
+                 "-i", self.bus_id, "-lms", "100"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
             time.sleep(0.3)
         except (OSError, FileNotFoundError):
@@ -117,6 +159,9 @@ class ClockSampler:
         return self
 
     def __exit__(self, *exc):
+        if self.thread is not None:
+            self.stop = True
+            self.thread.join(timeout=5)
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -125,9 +170,15 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self):
+        if self.thread is not None:
+            out = parse_clock_samples(self.lines)
+            out["source"] = f"NVML every {self.period * 1e3:.0f} ms"
+            return out
         if self.proc is None or not self.path or not os.path.exists(self.path):
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        return parse_clock_samples(open(self.path).read().splitlines())
+        out = parse_clock_samples(open(self.path).read().splitlines())
+        out["source"] = "nvidia-smi every 100 ms"
+        return out
 
 
 def parse_clock_samples(lines):
@@ -222,13 +273,24 @@ def gateup_kernel(cfg: MoEConfig, T: int, num_sms: int) -> str:
     return "k_gateup_bf16_wide" if T * cfg.k >= 256 * cfg.E else "k_gateup_bf16"
 
 
+def router_ksplit(T: int, d: int, E: int) -> int:
+    """The library's K split of the router GEMM (router_ksplit in router.cu)."""
+    tiles = -(-T // 128) * -(-E // 64)
+    nk, ks = d // 64, 1
+    while ks < 8 and tiles * ks * 2 <= 148 and nk // (ks * 2) >= 4:
+        ks *= 2
+    return ks
+
+
 def kernels_per_step(cfg: MoEConfig, T: int) -> int:
     """Kernels of this library one moe_forward launches, by its dispatch: the
-    router, the top-k, the permute (one kernel for at most 1024 assignments,
-    else count, scan and scatter), gate-up, down and combine, plus the
-    activation quantiser on the FP8 paths."""
+    router (with the top-k fused into it when one CTA covers a tile's whole K,
+    else followed by the top-k kernel), the permute (one kernel for at most
+    1024 assignments, else count, scan and scatter), gate-up, down and
+    combine, plus the activation quantiser on the FP8 paths."""
+    router = 1 if router_ksplit(T, cfg.d, cfg.E) == 1 else 2
     permute = 1 if T * cfg.k <= 1024 else 3
-    return 5 + permute + (1 if cfg.wdtype else 0)
+    return router + permute + 3 + (1 if cfg.wdtype else 0)
 
 
 def gateup_algorithmic(cfg: MoEConfig, T: int, n_active: int):
@@ -263,16 +325,18 @@ def _bits(t):
 
 def oracle_static_scales(cfg: MoEConfig, inp: dict, n_tokens: int = 8):
     """Static activation scales of a per-tensor FP8 layer for the oracle runs
-    without a GPU: amax(x) / 448 and amax(h) / 448 over the first n_tokens, h
-    from the oracle's own BF16 stages (the GPU layer calibrates the same way on
-    64 tokens with its BF16 kernels)."""
+    without a GPU, by the oracle's per-tensor rule s = fp32(amax) / 448: over
+    the first n_tokens of x, and over their gate-up output h from the
+    oracle's own BF16 stages, rounded to bf16 as the library's calibration
+    takes it (moe_calibrate_fp8_static does the same on the GPU with 64
+    tokens)."""
     import oracle
     L, xs = oracle_sample(MoEConfig(**{**cfg.__dict__, "wdtype": 0}), inp, n_tokens)
     out = oracle.forward(L, xs)
-    h = oracle.gateup(L, xs, out["perm"], out["offsets"])
-    amax_x = float(np.abs(oracle.bf16_decode(xs)).max())
-    amax_h = float(np.abs(h).max())
-    return (amax_x / 448.0 if amax_x > 0 else 1.0, amax_h / 448.0 if amax_h > 0 else 1.0)
+    h = oracle.gateup(L, xs, out["perm"], out["offsets"])[:, : cfg.I]
+    _, sx = oracle.quant_fp8_tensor(xs[None])
+    _, sh = oracle.quant_fp8_tensor(oracle.bf16_round(h)[None])
+    return (float(sx[0]), float(sh[0]))
 
 
 def oracle_sample(cfg: MoEConfig, inp: dict, n_tokens: int, act=(1.0, 1.0)):
@@ -381,30 +445,51 @@ def run_ours(args, cfg: MoEConfig):
     if layer.device_status() != M.OK:
         raise RuntimeError("device status after warm-up: " + M.status_string(layer.device_status()))
 
-    # the timed steps: one moe_forward per step, replayed from a CUDA graph (the
-    # library's launches are capturable), so host launch gaps do not count
+    # the timed steps: one moe_forward per step, all K of them captured in one
+    # CUDA graph (the library's launches are capturable) so host launch gaps do
+    # not count; each step records its stage events as event nodes of the graph,
+    # so the per-stage (roofline) times come from the timed replay itself
     graph = None
+    stage_source = "eager moe_forward_profiled launches (the timed steps)"
     if not args.no_graph:
         y_ref = y.clone()
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
+        one = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(one):
             M.forward(shape, layer.weights, x.view(torch.uint16), y.view(torch.uint16), layer.ws)
-        graph.replay()
+        one.replay()
         torch.cuda.synchronize()
         if not torch.equal(y, y_ref) or layer.device_status() != M.OK:
             raise RuntimeError("graph replay does not reproduce the eager forward")
+        del one
+        graph = torch.cuda.CUDAGraph()
+        try:
+            with torch.cuda.graph(graph):
+                for i in range(args.steps):
+                    M.forward_profiled(shape, layer.weights, x.view(torch.uint16), y.view(torch.uint16),
+                                       layer.ws, events[i])
+            stage_source = "event nodes inside the timed CUDA graph replay"
+        except Exception:  # noqa: BLE001 -- event nodes unavailable: time stages eagerly after
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                for i in range(args.steps):
+                    M.forward(shape, layer.weights, x.view(torch.uint16), y.view(torch.uint16), layer.ws)
+            stage_source = "eager moe_forward_profiled pass after the timed graph replay"
+        graph.replay()                                      # untimed: more warm-up steps
+        torch.cuda.synchronize()
+        if not torch.equal(y, y_ref) or layer.device_status() != M.OK:
+            raise RuntimeError("the K-step graph does not reproduce the eager forward")
         stream = torch.cuda.current_stream()
 
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local) as clocks:
+    with ClockSampler(nvml_bus_id(dev)) as clocks:
         barrier()
         torch.cuda.synchronize()
         t_start.record(stream)
-        for i in range(args.steps):
-            if graph is not None:
-                graph.replay()
-            else:
+        if graph is not None:
+            graph.replay()                                  # exactly K steps
+        else:
+            for i in range(args.steps):
                 M.forward_profiled(shape, layer.weights, x.view(torch.uint16), y.view(torch.uint16),
                                    layer.ws, events[i])
         t_end.record(stream)
@@ -412,8 +497,7 @@ def run_ours(args, cfg: MoEConfig):
         barrier()
     ms_total = t_start.elapsed_time(t_end)
     ms_total = max_over_ranks(ms_total, dev)
-    if graph is not None:
-        # per-stage times: the same steps again, eagerly, with the library's stage events
+    if graph is not None and stage_source.startswith("eager"):
         for i in range(args.steps):
             M.forward_profiled(shape, layer.weights, x.view(torch.uint16), y.view(torch.uint16),
                                layer.ws, events[i])
@@ -454,6 +538,7 @@ def run_ours(args, cfg: MoEConfig):
     roof["algorithmic_bytes"] = gu_bytes
     roof["algorithmic_flops"] = gu_flops
     roof["launch_ms"] = gu_ms
+    roof["launch_ms_source"] = stage_source
 
     # end to end through host buffers: every step copies its x in from pinned host
     # memory, runs the forward and copies y out (moe_forward_host_async), the
@@ -516,7 +601,8 @@ def run_ours(args, cfg: MoEConfig):
                        "l2": "no flush: the expert weights read each step "
                              f"({(gu_bytes + dn_bytes) / 1e9:.1f} GB) exceed the 126 MB L2",
                        "parallelism": f"{world} independent replicas (tokens sharded, no collective)",
-                       "launch": ("one CUDA graph replay of moe_forward per step" if graph is not None
+                       "launch": ("one CUDA graph holding the K steps' moe_forward launches, replayed once"
+                                  if graph is not None
                                   else "eager moe_forward_profiled launches")},
             "roofline": roof,
             "cpu_baseline": cpu,
@@ -537,7 +623,7 @@ def main(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", default="decode", choices=sorted(CONFIGS))
+    ap.add_argument("--config", default="skew", choices=sorted(CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-graph", action="store_true",
                     help="time eager launches with stage events instead of CUDA graph replays")

@@ -20,7 +20,7 @@ INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libmoe_b200.so")
 SOURCES = ["api.cu", "routing.cu", "router.cu", "gemm_bf16.cu", "gemm_bf16_wide.cu", "gemm_bf16_2sm.cu", "gemm_fp8.cu", "gemm_mx.cu", "gemm_f8t.cu",
-           "noalloc.cu"]
+           "ep.cu", "allreduce_norm.cu", "noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-O2",
          "--expt-relaxed-constexpr", "-I", INCLUDE]

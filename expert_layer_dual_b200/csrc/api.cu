@@ -2,6 +2,7 @@
 // carving, TMA descriptor creation and the stage sequence of moe_forward.
 // Host code only; every stage of the layer runs in the kernels of
 // routing.cu, router.cu, gemm_bf16.cu and gemm_fp8.cu.
+#include <cstring>
 #include <mutex>
 
 #include "common.cuh"
@@ -74,7 +75,7 @@ namespace {
 inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 struct WsLayout {
-    size_t logits, part, ids, w, counts, offsets, perm, inv, seg, xq, xs, h, hs, o, xin, yout, total;
+    size_t logits, part, rtk, ids, w, counts, offsets, perm, inv, seg, xq, xs, h, hs, o, xin, yout, total;
     int ksplit;
 };
 
@@ -92,6 +93,7 @@ WsLayout ws_layout(const moe_shape& s) {
     L.logits = take(T * E * 4);
     L.ksplit = router_ksplit(s.T, s.d, s.E);
     L.part = L.ksplit > 1 ? take(2 * (size_t)L.ksplit * T * E * 4) : 0;  // split-K router partials
+    L.rtk = L.ksplit == 1 ? take(router_topk_scratch_bytes(s.T, s.E)) : 0;  // fused top-k scratch
     L.ids = take(T * k * 4);
     L.w = take(T * k * 4);
     L.counts = take(E * 4);
@@ -177,8 +179,14 @@ moe_status check_ws(void* ws, size_t have, size_t need) {
     return MOE_OK;
 }
 
+// Tile counters of the grouped GEMMs' dynamic schedules, in the workspace
+// header after the status word: one per GEMM of a forward, so that the down
+// GEMM, launched while the gate-up drains, never shares one with it.
+constexpr int kGateupCounter = kWsTileCounter, kDownCounter = kWsTileCounter + 1;
+constexpr size_t kHeaderZeroBytes = (kDownCounter + 1) * sizeof(int32_t);
+
 GroupedGemmArgs gemm_args(const moe_shape* s, const int32_t* offsets, const int32_t* perm,
-                          int32_t* status) {
+                          int32_t* status, int counter, bool counter_zeroed) {
     GroupedGemmArgs a;
     a.T = s->T;
     a.d = s->d;
@@ -189,8 +197,9 @@ GroupedGemmArgs gemm_args(const moe_shape* s, const int32_t* offsets, const int3
     a.offsets = offsets;
     a.perm = perm;
     a.status = status;
-    a.tile_counter = status + kWsTileCounter;
+    a.tile_counter = status + counter;
     a.timeout_ns = kDefaultTimeoutNs;
+    a.counter_zeroed = counter_zeroed ? 1 : 0;
     return a;
 }
 
@@ -201,8 +210,8 @@ inline P* at(void* ws, size_t off) {
 
 moe_status run_gateup(const moe_shape* s, const moe_weights* w, const void* x, const void* xs,
                       const int32_t* perm, const int32_t* offsets, void* h, void* hs,
-                      int32_t* status, cudaStream_t st) {
-    const GroupedGemmArgs a = gemm_args(s, offsets, perm, status);
+                      int32_t* status, cudaStream_t st, bool counter_zeroed = false) {
+    const GroupedGemmArgs a = gemm_args(s, offsets, perm, status, kGateupCounter, counter_zeroed);
     if (s->wdtype == MOE_WDTYPE_BF16)
         return cuda_status((use_wide_gateup(s->T, s->E, s->k) ? launch_gateup_bf16_wide
                                                               : launch_gateup_bf16)(
@@ -228,8 +237,9 @@ moe_status run_gateup(const moe_shape* s, const moe_weights* w, const void* x, c
 }
 
 moe_status run_down(const moe_shape* s, const moe_weights* w, const void* h, const void* hs,
-                    const int32_t* offsets, __half* o, int32_t* status, cudaStream_t st) {
-    const GroupedGemmArgs a = gemm_args(s, offsets, nullptr, status);
+                    const int32_t* offsets, __half* o, int32_t* status, cudaStream_t st,
+                    bool counter_zeroed = false) {
+    const GroupedGemmArgs a = gemm_args(s, offsets, nullptr, status, kDownCounter, counter_zeroed);
     if (s->wdtype == MOE_WDTYPE_BF16)
         return cuda_status((use_pair_tiles(s->T, s->E, s->k) ? launch_down_bf16_2sm
                                                              : launch_down_bf16)(
@@ -251,39 +261,36 @@ moe_status run_down(const moe_shape* s, const moe_weights* w, const void* h, con
         static_cast<const uint8_t*>(w->ws_d), static_cast<const float*>(w->ws_d_scale), o, st));
 }
 
-// Records events[i] (when given) at the stage boundaries: 0 start, 1 router
-// logits, 2 top-k, 3 permute, 4 activation quantisation (FP8; else = 3),
-// 5 gate-up, 6 down, 7 combine.
-moe_status forward_device(const moe_shape* s, const moe_weights* w, const uint16_t* x, uint16_t* y,
-                          void* ws, cudaStream_t st, void* const* events = nullptr) {
-    auto mark = [&](int i) {
-        return events == nullptr ||
-               cudaEventRecord(static_cast<cudaEvent_t>(events[i]), st) == cudaSuccess;
-    };
-    const WsLayout L = ws_layout(*s);
+// Records events[i] (when given) on `st`; inside a stream capture the record
+// becomes an event node of the graph (timed on every replay).
+bool record_event(void* const* events, int i, cudaStream_t st) {
+    if (events == nullptr) return true;
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cap) != cudaSuccess) return false;
+    cudaEvent_t ev = static_cast<cudaEvent_t>(events[i]);
+    const cudaError_t e = cap == cudaStreamCaptureStatusActive
+                              ? cudaEventRecordWithFlags(ev, st, cudaEventRecordExternal)
+                              : cudaEventRecord(ev, st);
+    return e == cudaSuccess;
+}
+
+// The routing stages (router logits, top-k, permute) into the workspace
+// regions of L; events 1..3 as in forward_device.
+moe_status route_device(const moe_shape* s, const moe_weights* w, const uint16_t* x, void* ws,
+                        const WsLayout& L, cudaStream_t st, void* const* events) {
     int32_t* status = at<int32_t>(ws, 0);
     float* logits = at<float>(ws, L.logits);
     int32_t* ids = at<int32_t>(ws, L.ids);
     float* rw = at<float>(ws, L.w);
-    int32_t* counts = at<int32_t>(ws, L.counts);
-    int32_t* offsets = at<int32_t>(ws, L.offsets);
-    int32_t* perm = at<int32_t>(ws, L.perm);
-    int32_t* inv = at<int32_t>(ws, L.inv);
-    int32_t* seg = at<int32_t>(ws, L.seg);
-    const bool fp8 = s->wdtype == MOE_WDTYPE_FP8_BLOCK128;
-    const bool mx = s->wdtype == MOE_WDTYPE_MXFP8;
-    const bool f8t = s->wdtype == MOE_WDTYPE_FP8_TENSOR;
     moe_status r;
-    if (cudaMemsetAsync(status, 0, sizeof(int32_t), st) != cudaSuccess) return MOE_ERR_CUDA;
-    if (!mark(0)) return MOE_ERR_CUDA;
     if (L.ksplit == 1) {
-        if ((r = cuda_status(launch_router_logits(x, w->router_hi, w->router_lo, w->router_bias,
-                                                  logits, s->T, s->d, s->E, status, st))) != MOE_OK)
+        // router logits with the top-k fused into the same kernel
+        if ((r = cuda_status(launch_router_topk(x, w->router_hi, w->router_lo, w->router_bias,
+                                                logits, s->T, s->d, s->E, s->k, s->renormalize,
+                                                ids, rw, at<uint8_t>(ws, L.rtk), status, st))) !=
+            MOE_OK)
             return r;
-        if (!mark(1)) return MOE_ERR_CUDA;
-        if ((r = cuda_status(launch_route_topk(logits, s->T, s->E, s->k, s->renormalize, ids, rw,
-                                               st))) != MOE_OK)
-            return r;
+        if (!record_event(events, 1, st)) return MOE_ERR_CUDA;
     } else {
         // few tokens: K split across CTAs, partials combined inside the top-k kernel
         float* ph = at<float>(ws, L.part);
@@ -291,17 +298,42 @@ moe_status forward_device(const moe_shape* s, const moe_weights* w, const uint16
         if ((r = cuda_status(launch_router_partials(x, w->router_hi, w->router_lo, ph, pl, L.ksplit,
                                                     s->T, s->d, s->E, status, st))) != MOE_OK)
             return r;
-        if (!mark(1)) return MOE_ERR_CUDA;
+        if (!record_event(events, 1, st)) return MOE_ERR_CUDA;
         if ((r = cuda_status(launch_route_topk_partials(ph, pl, L.ksplit, w->router_bias, logits,
                                                         s->T, s->E, s->k, s->renormalize, ids, rw,
                                                         st))) != MOE_OK)
             return r;
     }
-    if (!mark(2)) return MOE_ERR_CUDA;
-    if ((r = cuda_status(launch_permute(ids, s->T, s->E, s->k, counts, offsets, perm, inv, seg,
-                                        status, st))) != MOE_OK)
+    if (!record_event(events, 2, st)) return MOE_ERR_CUDA;
+    if ((r = cuda_status(launch_permute(ids, s->T, s->E, s->k, at<int32_t>(ws, L.counts),
+                                        at<int32_t>(ws, L.offsets), at<int32_t>(ws, L.perm),
+                                        at<int32_t>(ws, L.inv), at<int32_t>(ws, L.seg), status,
+                                        st))) != MOE_OK)
         return r;
-    if (!mark(3)) return MOE_ERR_CUDA;
+    return record_event(events, 3, st) ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// Records events[i] (when given) at the stage boundaries: 0 start, 1 router
+// logits, 2 top-k, 3 permute, 4 activation quantisation (FP8; else = 3),
+// 5 gate-up, 6 down, 7 combine.
+moe_status forward_device(const moe_shape* s, const moe_weights* w, const uint16_t* x, uint16_t* y,
+                          void* ws, cudaStream_t st, void* const* events = nullptr) {
+    auto mark = [&](int i) { return record_event(events, i, st); };
+    const WsLayout L = ws_layout(*s);
+    int32_t* status = at<int32_t>(ws, 0);
+    float* rw = at<float>(ws, L.w);
+    int32_t* offsets = at<int32_t>(ws, L.offsets);
+    int32_t* perm = at<int32_t>(ws, L.perm);
+    int32_t* inv = at<int32_t>(ws, L.inv);
+    const bool fp8 = s->wdtype == MOE_WDTYPE_FP8_BLOCK128;
+    const bool mx = s->wdtype == MOE_WDTYPE_MXFP8;
+    const bool f8t = s->wdtype == MOE_WDTYPE_FP8_TENSOR;
+    moe_status r;
+    // the status word and both GEMM tile counters, zeroed before the first kernel so
+    // that no memset separates the kernels of the chain (each may start early)
+    if (cudaMemsetAsync(status, 0, kHeaderZeroBytes, st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (!mark(0)) return MOE_ERR_CUDA;
+    if ((r = route_device(s, w, x, ws, L, st, events)) != MOE_OK) return r;
     const void* a_in = x;
     const void* a_scale = nullptr;
     if (f8t) {
@@ -332,9 +364,10 @@ moe_status forward_device(const moe_shape* s, const moe_weights* w, const uint16
     void* h = at<uint8_t>(ws, L.h);
     void* hs = (fp8 || mx) ? at<uint8_t>(ws, L.hs) : nullptr;
     __half* o = at<__half>(ws, L.o);
-    if ((r = run_gateup(s, w, a_in, a_scale, perm, offsets, h, hs, status, st)) != MOE_OK) return r;
+    if ((r = run_gateup(s, w, a_in, a_scale, perm, offsets, h, hs, status, st, true)) != MOE_OK)
+        return r;
     if (!mark(5)) return MOE_ERR_CUDA;
-    if ((r = run_down(s, w, h, hs, offsets, o, status, st)) != MOE_OK) return r;
+    if ((r = run_down(s, w, h, hs, offsets, o, status, st, true)) != MOE_OK) return r;
     if (!mark(6)) return MOE_ERR_CUDA;
     if ((r = cuda_status(launch_combine(o, inv, rw, y, s->T, s->d, s->k, s->I_shared > 0 ? 1 : 0,
                                         st))) != MOE_OK)
@@ -635,6 +668,234 @@ moe_status moe_forward_host(const moe_shape* shape, const moe_weights* weights,
     if (cudaMemcpyAsync(y_host, yout, bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
         return MOE_ERR_CUDA;
     return cuda_status(cudaStreamSynchronize(st));
+}
+
+moe_status moe_workspace_offsets(const moe_shape* shape, moe_workspace_map* map) {
+    if (map == nullptr) return MOE_ERR_INVALID_ARG;
+    const moe_status r = check_shape(shape);
+    if (r != MOE_OK) return r;
+    const WsLayout L = ws_layout(*shape);
+    map->logits = L.logits;
+    map->ids = L.ids;
+    map->w = L.w;
+    map->counts = L.counts;
+    map->offsets = L.offsets;
+    map->perm = L.perm;
+    map->inv = L.inv;
+    map->h = L.h;
+    map->total = L.total;
+    return MOE_OK;
+}
+
+moe_status moe_calibrate_fp8_static(const moe_shape* shape, const moe_weights* weights,
+                                    const uint16_t* x, float* scales, void* ws, size_t ws_bytes,
+                                    void* stream) {
+    moe_status r = check_shape(shape);
+    if (r != MOE_OK) return r;
+    if (shape->wdtype != MOE_WDTYPE_BF16) return MOE_ERR_UNSUPPORTED;
+    if ((r = check_weights(shape, weights, true, false, true)) != MOE_OK) return r;
+    if (shape->T == 0 || x == nullptr || scales == nullptr ||
+        (reinterpret_cast<uintptr_t>(x) & 15u) != 0)
+        return MOE_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(*shape);
+    if ((r = check_ws(ws, ws_bytes, L.total)) != MOE_OK) return r;
+    if (!device_ok()) return MOE_ERR_UNSUPPORTED;
+    cudaStream_t st = as_stream(stream);
+    int32_t* status = at<int32_t>(ws, 0);
+    if (cudaMemsetAsync(status, 0, kHeaderZeroBytes, st) != cudaSuccess) return MOE_ERR_CUDA;
+    if ((r = route_device(shape, weights, x, ws, L, st, nullptr)) != MOE_OK) return r;
+    uint16_t* h = at<uint16_t>(ws, L.h);
+    if ((r = run_gateup(shape, weights, x, nullptr, at<int32_t>(ws, L.perm),
+                        at<int32_t>(ws, L.offsets), h, nullptr, status, st, true)) != MOE_OK)
+        return r;
+    const int64_t R = (int64_t)shape->T * shape->k + (shape->I_shared > 0 ? shape->T : 0);
+    if ((r = cuda_status(launch_amax_scale(x, (int64_t)shape->T * shape->d, scales, st))) != MOE_OK)
+        return r;
+    return cuda_status(launch_amax_scale(h, R * shape->I, scales + 1, st));
+}
+
+moe_status moe_route(const moe_shape* shape, const moe_weights* weights, const uint16_t* x,
+                     void* ws, size_t ws_bytes, void* stream) {
+    moe_status r = check_shape(shape);
+    if (r != MOE_OK) return r;
+    if (shape->wdtype != MOE_WDTYPE_BF16 && shape->wdtype != MOE_WDTYPE_FP8_BLOCK128 &&
+        shape->wdtype != MOE_WDTYPE_MXFP8 && shape->wdtype != MOE_WDTYPE_FP8_TENSOR)
+        return MOE_ERR_UNSUPPORTED;
+    if ((r = check_weights(shape, weights, false, false, true)) != MOE_OK) return r;
+    if (shape->T == 0) return MOE_OK;
+    if (x == nullptr) return MOE_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(*shape);
+    if ((r = check_ws(ws, ws_bytes, L.total)) != MOE_OK) return r;
+    if (!device_ok()) return MOE_ERR_UNSUPPORTED;
+    cudaStream_t st = as_stream(stream);
+    if (cudaMemsetAsync(ws, 0, kHeaderZeroBytes, st) != cudaSuccess) return MOE_ERR_CUDA;
+    return route_device(shape, weights, x, ws, L, st, nullptr);
+}
+
+moe_status moe_ep_dispatch(const uint16_t* x, const int32_t* ids, const int32_t* perm, int32_t T,
+                           int32_t d, int32_t k, int32_t E_local, uint16_t* send_rows,
+                           int32_t* send_ids, void* stream) {
+    if (T < 0 || d <= 0 || k <= 0 || E_local <= 0) return MOE_ERR_INVALID_ARG;
+    if (d % 8 != 0 || (int64_t)T * k >= ((int64_t)1 << 31)) return MOE_ERR_UNSUPPORTED;
+    if (T == 0) return MOE_OK;
+    if (x == nullptr || ids == nullptr || perm == nullptr || send_rows == nullptr ||
+        send_ids == nullptr || (reinterpret_cast<uintptr_t>(x) & 15u) != 0 ||
+        (reinterpret_cast<uintptr_t>(send_rows) & 15u) != 0)
+        return MOE_ERR_INVALID_ARG;
+    if (!device_ok()) return MOE_ERR_UNSUPPORTED;
+    return cuda_status(launch_ep_dispatch(x, ids, perm, (int64_t)T * k, d, k, E_local, send_rows,
+                                          send_ids, as_stream(stream)));
+}
+
+moe_status moe_gather_rows(const void* src, const int32_t* index, int64_t n, int32_t row_bytes,
+                           void* dst, void* stream) {
+    if (n < 0 || row_bytes <= 0) return MOE_ERR_INVALID_ARG;
+    if (row_bytes % 16 != 0) return MOE_ERR_UNSUPPORTED;
+    if (n == 0) return MOE_OK;
+    if (src == nullptr || index == nullptr || dst == nullptr ||
+        (reinterpret_cast<uintptr_t>(src) & 15u) != 0 || (reinterpret_cast<uintptr_t>(dst) & 15u) != 0)
+        return MOE_ERR_INVALID_ARG;
+    if (!device_ok()) return MOE_ERR_UNSUPPORTED;
+    return cuda_status(launch_gather_rows(src, index, n, row_bytes, dst, as_stream(stream)));
+}
+
+size_t moe_lamport_buffer_bytes(int32_t G, int32_t T_max, int32_t d) {
+    if (G < 1 || G > kArMaxRanks || T_max < 0 || d <= 0) return 0;
+    return lamport_buffer_bytes(G, T_max, d);
+}
+
+moe_status moe_lamport_init(void* buf, size_t bytes, void* stream) {
+    if (bytes == 0) return MOE_OK;
+    if (buf == nullptr || (reinterpret_cast<uintptr_t>(buf) & 15u) != 0 || bytes % 16 != 0)
+        return MOE_ERR_INVALID_ARG;
+    if (!device_ok()) return MOE_ERR_UNSUPPORTED;
+    return cuda_status(launch_lamport_init(buf, bytes, as_stream(stream)));
+}
+
+moe_status moe_peer_buffer_alloc(size_t bytes, void** ptr, void* ipc_handle) {
+    if (ptr == nullptr || ipc_handle == nullptr || bytes == 0) return MOE_ERR_INVALID_ARG;
+    if (!device_ok()) return MOE_ERR_UNSUPPORTED;
+    *ptr = nullptr;
+    if (cudaMalloc(ptr, bytes) != cudaSuccess) return MOE_ERR_CUDA;
+    cudaIpcMemHandle_t h;
+    if (cudaIpcGetMemHandle(&h, *ptr) != cudaSuccess) {
+        cudaFree(*ptr);
+        *ptr = nullptr;
+        return MOE_ERR_CUDA;
+    }
+    memcpy(ipc_handle, &h, sizeof(h));
+    return MOE_OK;
+}
+
+moe_status moe_peer_buffer_open(const void* ipc_handle, void** ptr) {
+    if (ptr == nullptr || ipc_handle == nullptr) return MOE_ERR_INVALID_ARG;
+    cudaIpcMemHandle_t h;
+    memcpy(&h, ipc_handle, sizeof(h));
+    *ptr = nullptr;
+    return cuda_status(cudaIpcOpenMemHandle(ptr, h, cudaIpcMemLazyEnablePeerAccess));
+}
+
+moe_status moe_peer_buffer_close(void* ptr) {
+    if (ptr == nullptr) return MOE_ERR_INVALID_ARG;
+    return cuda_status(cudaIpcCloseMemHandle(ptr));
+}
+
+moe_status moe_peer_buffer_free(void* ptr) {
+    if (ptr == nullptr) return MOE_ERR_INVALID_ARG;
+    return cuda_status(cudaFree(ptr));
+}
+
+namespace {
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+moe_status check_ar(int32_t G, int32_t T_max, int32_t T, int32_t d, const void* gamma) {
+    if (G < 1 || T < 0 || T_max < 0 || d <= 0) return MOE_ERR_INVALID_ARG;
+    if (G > kArMaxRanks || d % 8 != 0 || d > allreduce_norm_max_d() || T > T_max)
+        return MOE_ERR_UNSUPPORTED;
+    if (T > 0 && (gamma == nullptr || !aligned16(gamma))) return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+}  // namespace
+
+moe_status moe_allreduce_rmsnorm(void* const* bufs, int32_t G, int32_t rank, uint32_t call,
+                                 int32_t T_max, const uint16_t* x, const uint16_t* residual,
+                                 const uint16_t* gamma, float eps, int32_t T, int32_t d,
+                                 uint16_t* out, uint16_t* residual_out, void* ws, size_t ws_bytes,
+                                 void* stream) {
+    moe_status r = check_ar(G, T_max, T, d, gamma);
+    if (r != MOE_OK) return r;
+    if (rank < 0 || rank >= G || bufs == nullptr || !(eps >= 0.0f)) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if ((r = check_ws(ws, ws_bytes, kWsHeader)) != MOE_OK) return r;
+    for (int p = 0; p < G; ++p)
+        if (bufs[p] == nullptr || !aligned16(bufs[p])) return MOE_ERR_INVALID_ARG;
+    if (x == nullptr || out == nullptr || !aligned16(x) || !aligned16(out) ||
+        (residual != nullptr && !aligned16(residual)) ||
+        (residual_out != nullptr && !aligned16(residual_out)))
+        return MOE_ERR_INVALID_ARG;
+    if (!device_ok()) return MOE_ERR_UNSUPPORTED;
+    ArNormArgs a{};
+    for (int p = 0; p < G; ++p) a.bufs[p] = static_cast<uint16_t*>(bufs[p]);
+    a.x[0] = x;
+    a.residual[0] = residual;
+    a.out[0] = out;
+    a.res_out[0] = residual_out;
+    a.gamma = gamma;
+    a.G = G;
+    a.T = T;
+    a.T_max = T_max;
+    a.d = d;
+    a.rank0 = rank;
+    a.call = call;
+    a.eps = eps;
+    a.status = at<int32_t>(ws, 0);
+    a.timeout_ns = kDefaultTimeoutNs;
+    return cuda_status(launch_allreduce_rmsnorm(a, 1, false, as_stream(stream)));
+}
+
+moe_status moe_allreduce_rmsnorm_emulated(void* const* bufs, int32_t G, int32_t ranks,
+                                          uint32_t call, int32_t T_max, const uint16_t* const* x,
+                                          const uint16_t* const* residual, const uint16_t* gamma,
+                                          float eps, int32_t T, int32_t d, uint16_t* const* out,
+                                          uint16_t* const* residual_out, int32_t timeout_us,
+                                          void* ws, size_t ws_bytes, void* stream) {
+    moe_status r = check_ar(G, T_max, T, d, gamma);
+    if (r != MOE_OK) return r;
+    if (ranks < 1 || ranks > G || bufs == nullptr || x == nullptr || out == nullptr ||
+        timeout_us <= 0 || !(eps >= 0.0f))
+        return MOE_ERR_INVALID_ARG;
+    if ((r = check_ws(ws, ws_bytes, kWsHeader)) != MOE_OK) return r;
+    for (int p = 0; p < G; ++p)
+        if (bufs[p] == nullptr || !aligned16(bufs[p])) return MOE_ERR_INVALID_ARG;
+    for (int p = 0; p < ranks; ++p)
+        if (x[p] == nullptr || out[p] == nullptr || !aligned16(x[p]) || !aligned16(out[p]) ||
+            (residual != nullptr && residual[p] != nullptr && !aligned16(residual[p])) ||
+            (residual_out != nullptr && residual_out[p] != nullptr && !aligned16(residual_out[p])))
+            return MOE_ERR_INVALID_ARG;
+    if (!device_ok()) return MOE_ERR_UNSUPPORTED;
+    cudaStream_t st = as_stream(stream);
+    int32_t* status = at<int32_t>(ws, 0);
+    if (cudaMemsetAsync(status, 0, sizeof(int32_t), st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (T == 0) return MOE_OK;
+    ArNormArgs a{};
+    for (int p = 0; p < G; ++p) a.bufs[p] = static_cast<uint16_t*>(bufs[p]);
+    for (int p = 0; p < ranks; ++p) {
+        a.x[p] = x[p];
+        a.residual[p] = residual != nullptr ? residual[p] : nullptr;
+        a.out[p] = out[p];
+        a.res_out[p] = residual_out != nullptr ? residual_out[p] : nullptr;
+    }
+    a.gamma = gamma;
+    a.G = G;
+    a.T = T;
+    a.T_max = T_max;
+    a.d = d;
+    a.rank0 = 0;
+    a.call = call;
+    a.eps = eps;
+    a.status = status;
+    a.timeout_ns = (uint64_t)timeout_us * 1000ull;
+    return cuda_status(launch_allreduce_rmsnorm(a, ranks, true, st));
 }
 
 moe_status moe_read_device_status(const void* ws, void* stream) {

@@ -20,14 +20,26 @@
 namespace moe {
 
 // Bytes reserved at the start of every workspace; the device status word is
-// its first int32, the grouped GEMMs' tile counter the int32 at index
-// kWsTileCounter.
+// its first int32, the grouped GEMMs' tile counters the int32s from index
+// kWsTileCounter on (gate-up, then down).
 constexpr size_t kWsHeader = 256;
 constexpr int kWsTileCounter = 32;
 
 // Default bound of every device-side wait: far above any legitimate wait in
 // these kernels (the longest is one k-block of one tile), far below a hang.
 constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;  // 2 s
+
+// Programmatic dependent launch.  The forward's kernels are launched so that
+// each may be scheduled while the previous one in the stream is finishing
+// (launch_pdl): pdl_wait() blocks until that kernel has completed and its
+// memory is visible (a no-op for a kernel launched without the attribute),
+// so every kernel calls it before its first read of data another kernel
+// produced; pdl_trigger() lets the next kernel be scheduled once every block
+// of this one has passed it.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
 
 __device__ __forceinline__ void report_status(int32_t* status, int32_t code) {
     if (status != nullptr) atomicCAS(status, 0, code);

@@ -103,10 +103,12 @@ __device__ __forceinline__ uint32_t prologue(Smem& sm, const GroupedGemmArgs& a,
         b->abort_flag = 0;
         fence_barrier_init();
     }
-    if (warp == 0) build_tile_table(sm.tt, a.offsets, a.E, a.T, a.k, a.has_shared, BM);
     if (warp == MMA_WARP) tmem_alloc(&b->tmem_slot, TMEM_COLS);
+    pdl_wait();  // offsets and the A operand come from the previous kernels
+    if (warp == 0) build_tile_table(sm.tt, a.offsets, a.E, a.T, a.k, a.has_shared, BM);
     tc_fence_before_sync();
     __syncthreads();
+    pdl_trigger();
     tc_fence_after_sync();
     return b->tmem_slot;
 }
@@ -444,8 +446,14 @@ cudaError_t launch_gateup_bf16(const GroupedGemmArgs& a, const uint16_t* x, cons
     static bool flags[64] = {false};
     cudaError_t e = set_smem_once(k_gateup_bf16, flags);
     if (e != cudaSuccess) return e;
-    if ((e = cudaMemsetAsync(a.tile_counter, 0, sizeof(int32_t), s)) != cudaSuccess) return e;
-    k_gateup_bf16<<<current_device_info().num_sms, GATEUP_THREADS, SMEM_BYTES, s>>>(tw, tws, a, x, h);
+    if (!a.counter_zeroed &&
+        (e = cudaMemsetAsync(a.tile_counter, 0, sizeof(int32_t), s)) != cudaSuccess)
+        return e;
+    {
+        const cudaError_t le = launch_pdl(k_gateup_bf16, dim3(current_device_info().num_sms),
+                                          dim3(GATEUP_THREADS), SMEM_BYTES, s, tw, tws, a, x, h);
+        if (le != cudaSuccess) return le;
+    }
     return cudaGetLastError();
 }
 
@@ -461,8 +469,14 @@ cudaError_t launch_down_bf16(const GroupedGemmArgs& a, const uint16_t* h, const 
     static bool flags[64] = {false};
     cudaError_t e = set_smem_once(k_down_bf16, flags);
     if (e != cudaSuccess) return e;
-    if ((e = cudaMemsetAsync(a.tile_counter, 0, sizeof(int32_t), s)) != cudaSuccess) return e;
-    k_down_bf16<<<current_device_info().num_sms, DOWN_THREADS, SMEM_BYTES, s>>>(th, tw, tws, a, o);
+    if (!a.counter_zeroed &&
+        (e = cudaMemsetAsync(a.tile_counter, 0, sizeof(int32_t), s)) != cudaSuccess)
+        return e;
+    {
+        const cudaError_t le = launch_pdl(k_down_bf16, dim3(current_device_info().num_sms),
+                                          dim3(DOWN_THREADS), SMEM_BYTES, s, th, tw, tws, a, o);
+        if (le != cudaSuccess) return le;
+    }
     return cudaGetLastError();
 }
 

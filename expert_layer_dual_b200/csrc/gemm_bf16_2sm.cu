@@ -89,8 +89,10 @@ __device__ __forceinline__ uint32_t prologue(Smem& sm, const GroupedGemmArgs& a,
         b->abort_flag = 0;
         fence_barrier_init();
     }
+    pdl_wait();  // offsets and the A operand come from the previous kernels
     if (warp == 0) build_tile_table(sm.tt, a.offsets, a.E, a.T, a.k, a.has_shared, PM);
     __syncthreads();
+    pdl_trigger();
     cluster_sync();  // both CTAs' barriers exist before either signals the other
     if (warp == MMA_WARP) tmem_alloc_pair(&b->tmem_slot, TMEM_COLS);
     tc_fence_before_sync();
@@ -270,7 +272,11 @@ cudaError_t launch_down_bf16_2sm(const GroupedGemmArgs& a, const uint16_t* h, co
     static bool flags[64] = {false};
     cudaError_t e = set_smem_once(k_down_bf16_2sm, flags);
     if (e != cudaSuccess) return e;
-    k_down_bf16_2sm<<<pair_grid(), DOWN_THREADS, SMEM_BYTES, s>>>(th, tw, tws, a, o);
+    {
+        const cudaError_t le = launch_pdl(k_down_bf16_2sm, dim3(pair_grid()), dim3(DOWN_THREADS),
+                                          SMEM_BYTES, s, th, tw, tws, a, o);
+        if (le != cudaSuccess) return le;
+    }
     return cudaGetLastError();
 }
 

@@ -92,10 +92,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         b->abort_flag = 0;
         fence_barrier_init();
     }
-    if (warp == 0) build_tile_table(tt, a.offsets, a.E, a.T, a.k, a.has_shared, BM);
     if (warp == MMA_WARP) tmem_alloc(&b->tmem_slot, TMEM_COLS);
+    pdl_wait();  // offsets and the A operand come from the previous kernels
+    if (warp == 0) build_tile_table(tt, a.offsets, a.E, a.T, a.k, a.has_shared, BM);
     tc_fence_before_sync();
     __syncthreads();
+    pdl_trigger();
     tc_fence_after_sync();
     const uint32_t tmem = b->tmem_slot;
     const int G = a.E + a.has_shared;
@@ -313,9 +315,14 @@ cudaError_t launch_gateup_bf16_wide(const GroupedGemmArgs& a, const uint16_t* x,
         if (e != cudaSuccess) return e;
         g_smem_set[dev] = true;
     }
-    cudaError_t e = cudaMemsetAsync(a.tile_counter, 0, sizeof(int32_t), s);
+    cudaError_t e =
+        a.counter_zeroed ? cudaSuccess : cudaMemsetAsync(a.tile_counter, 0, sizeof(int32_t), s);
     if (e != cudaSuccess) return e;
-    k_gateup_bf16_wide<<<current_device_info().num_sms, THREADS, SMEM_BYTES, s>>>(tw, tws, a, x, h);
+    {
+        const cudaError_t le = launch_pdl(k_gateup_bf16_wide, dim3(current_device_info().num_sms),
+                                          dim3(THREADS), SMEM_BYTES, s, tw, tws, a, x, h);
+        if (le != cudaSuccess) return le;
+    }
     return cudaGetLastError();
 }
 

@@ -87,10 +87,12 @@ __device__ __forceinline__ uint32_t prologue(Smem& sm, const GroupedGemmArgs& a)
         b->abort_flag = 0;
         fence_barrier_init();
     }
-    if (warp == 0) build_tile_table(sm.tt, a.offsets, a.E, a.T, a.k, a.has_shared, BM);
     if (warp == MMA_WARP) tmem_alloc(&b->tmem_slot, TMEM_COLS);
+    pdl_wait();  // offsets and the A operand come from the previous kernels
+    if (warp == 0) build_tile_table(sm.tt, a.offsets, a.E, a.T, a.k, a.has_shared, BM);
     tc_fence_before_sync();
     __syncthreads();
+    pdl_trigger();
     tc_fence_after_sync();
     return b->tmem_slot;
 }
@@ -357,9 +359,15 @@ cudaError_t launch_gateup_f8t(const GroupedGemmArgs& a, const uint8_t* xq, float
     static bool flags[64] = {false};
     cudaError_t e = set_smem_once(k_gateup_f8t, flags);
     if (e != cudaSuccess) return e;
-    if ((e = cudaMemsetAsync(a.tile_counter, 0, sizeof(int32_t), s)) != cudaSuccess) return e;
-    k_gateup_f8t<<<current_device_info().num_sms, THREADS, SMEM_BYTES, s>>>(
-        ta, tw, tws, a, sx, sh, w_gu_s, a.has_shared ? ws_gu_s : w_gu_s, hq);
+    if (!a.counter_zeroed &&
+        (e = cudaMemsetAsync(a.tile_counter, 0, sizeof(int32_t), s)) != cudaSuccess)
+        return e;
+    {
+        const cudaError_t le = launch_pdl(k_gateup_f8t, dim3(current_device_info().num_sms),
+                                          dim3(THREADS), SMEM_BYTES, s, ta, tw, tws, a, sx, sh,
+                                          w_gu_s, a.has_shared ? ws_gu_s : w_gu_s, hq);
+        if (le != cudaSuccess) return le;
+    }
     return cudaGetLastError();
 }
 
@@ -376,9 +384,15 @@ cudaError_t launch_down_f8t(const GroupedGemmArgs& a, const uint8_t* hq, float s
     static bool flags[64] = {false};
     cudaError_t e = set_smem_once(k_down_f8t, flags);
     if (e != cudaSuccess) return e;
-    if ((e = cudaMemsetAsync(a.tile_counter, 0, sizeof(int32_t), s)) != cudaSuccess) return e;
-    k_down_f8t<<<current_device_info().num_sms, THREADS, SMEM_BYTES, s>>>(
-        ta, tw, tws, a, sh, w_d_s, a.has_shared ? ws_d_s : w_d_s, o);
+    if (!a.counter_zeroed &&
+        (e = cudaMemsetAsync(a.tile_counter, 0, sizeof(int32_t), s)) != cudaSuccess)
+        return e;
+    {
+        const cudaError_t le = launch_pdl(k_down_f8t, dim3(current_device_info().num_sms),
+                                          dim3(THREADS), SMEM_BYTES, s, ta, tw, tws, a, sh, w_d_s,
+                                          a.has_shared ? ws_d_s : w_d_s, o);
+        if (le != cudaSuccess) return le;
+    }
     return cudaGetLastError();
 }
 

@@ -20,6 +20,26 @@ struct DevInfo {
 // Cached per-device properties of the current device.
 const DevInfo& current_device_info();
 
+// Launches `kernel` with programmatic dependent launch allowed: it may be
+// scheduled while the previous kernel in `s` finishes, and must call
+// pdl_wait() before reading anything that kernel (or one before it) wrote.
+// Captured into a CUDA graph, the dependency becomes a programmatic edge.
+template <typename... Params, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t s, Args... args) {
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<Params>(args)...);
+}
+
 // ---- routing.cu
 cudaError_t launch_router_split(const float* W, uint16_t* hi, uint16_t* lo, int64_t n,
                                 cudaStream_t s);
@@ -64,12 +84,26 @@ cudaError_t launch_quant_weights_fp8_tensor(const uint16_t* W, int64_t batch, in
 cudaError_t launch_quant_act_fp8_static(const uint16_t* x, const int32_t* perm, int T, int k,
                                         int64_t rows, int cols, float scale, uint8_t* q,
                                         cudaStream_t s);
+// Static FP8 scale of n bf16 values (n % 8 == 0, v 16-byte aligned): *scale =
+// fp32(max |v|) / 448 (1 when every value is zero).
+cudaError_t launch_amax_scale(const uint16_t* v, int64_t n, float* scale, cudaStream_t s);
 cudaError_t launch_selftest_timeout(int32_t* status, uint64_t limit_ns, cudaStream_t s);
 
 // ---- router.cu (tcgen05 dual-BF16 GEMM)
 cudaError_t launch_router_logits(const uint16_t* x, const uint16_t* hi, const uint16_t* lo,
                                  const float* bias, float* logits, int T, int d, int E,
                                  int32_t* status, cudaStream_t s);
+
+// Router logits with the top-k fused into the kernel (moe_forward, one CTA per
+// tile, i.e. router_ksplit(T, d, E) == 1): ids [T][k], w [T][k] as
+// launch_route_topk writes them.  `scratch`: router_topk_scratch_bytes(T, E)
+// bytes (16-byte aligned) of candidate keys and arrival counters, the
+// counters zeroed here before the launch.
+size_t router_topk_scratch_bytes(int T, int E);
+cudaError_t launch_router_topk(const uint16_t* x, const uint16_t* hi, const uint16_t* lo,
+                               const float* bias, float* logits, int T, int d, int E, int k,
+                               int renorm, int32_t* ids, float* w, void* scratch, int32_t* status,
+                               cudaStream_t s);
 
 // K split of the router GEMM for T tokens (1 = one CTA per tile covers all of d).
 int router_ksplit(int T, int d, int E);
@@ -84,8 +118,10 @@ struct GroupedGemmArgs {
     const int32_t* offsets;  // [E+1]
     const int32_t* perm;     // [T*k]
     int32_t* status;
-    int32_t* tile_counter;   // next tile number of the dynamic schedule (zeroed by the launcher)
+    int32_t* tile_counter;   // next tile number of the dynamic schedule
     uint64_t timeout_ns;
+    int counter_zeroed;      // 1: the caller zeroed tile_counter earlier in the stream;
+                             // 0: the launcher zeroes it before the launch
 };
 cudaError_t launch_gateup_bf16(const GroupedGemmArgs& a, const uint16_t* x, const uint16_t* w_gu,
                                const uint16_t* ws_gu, uint16_t* h, cudaStream_t s);
@@ -129,6 +165,36 @@ cudaError_t launch_gateup_f8t(const GroupedGemmArgs& a, const uint8_t* xq, float
 cudaError_t launch_down_f8t(const GroupedGemmArgs& a, const uint8_t* hq, float sh,
                             const uint8_t* w_d, const float* w_d_s, const uint8_t* ws_d,
                             const float* ws_d_s, __half* o, cudaStream_t s);
+
+// ---- ep.cu (expert parallelism: the rows sent to the experts' owners and back)
+cudaError_t launch_ep_dispatch(const uint16_t* x, const int32_t* ids, const int32_t* perm,
+                               int64_t n, int d, int k, int E_local, uint16_t* send_rows,
+                               int32_t* send_ids, cudaStream_t s);
+cudaError_t launch_gather_rows(const void* src, const int32_t* index, int64_t n, int row_bytes,
+                               void* dst, cudaStream_t s);
+
+// ---- allreduce_norm.cu (tensor-parallel all-reduce + residual + RMSNorm, Lamport P2P)
+constexpr int kArMaxRanks = 8;
+struct ArNormArgs {
+    uint16_t* bufs[kArMaxRanks];             // every rank's Lamport buffer, by rank
+    const uint16_t* x[kArMaxRanks];          // per rank of this launch (grid.y): its input
+    const uint16_t* residual[kArMaxRanks];   // or nullptr
+    uint16_t* out[kArMaxRanks];
+    uint16_t* res_out[kArMaxRanks];          // or nullptr
+    const uint16_t* gamma;
+    int G, T, T_max, d, rank0;               // rank of grid.y == 0
+    uint32_t call;
+    float eps;
+    int32_t* status;
+    uint64_t timeout_ns;
+};
+size_t lamport_buffer_bytes(int G, int T_max, int d);
+int allreduce_norm_max_d();
+cudaError_t launch_lamport_init(void* buf, size_t bytes, cudaStream_t s);
+// One rank (ranks_in_launch = 1, PDL launch) or every rank of an emulated
+// group on one GPU (cooperative launch, grid.y = rank).
+cudaError_t launch_allreduce_rmsnorm(const ArNormArgs& a, int ranks_in_launch, bool cooperative,
+                                     cudaStream_t s);
 
 // ---- tensor maps (api.cu)
 // 2-D row-major tensor [rows][cols] of `elem_bytes`-sized elements, box

@@ -22,6 +22,18 @@
 // correcting FMA; lo (already scaled down by 256) keeps one accumulator.
 // TMEM columns: hi chunk c at c*64 .. c*64+63, lo at C*64 .. C*64+63.
 //
+// Top-k fused into the epilogue (moe_forward, one CTA per tile): the routing
+// step needs all E logits of a token, which span E/64 CTAs.  Each CTA's
+// epilogue thread keeps the best 8 of its row's 64 logits in registers as
+// packed (logit, expert) keys and writes them out; the CTA that completes an
+// m-tile last (an arrival counter per m-tile; writers fence before arriving,
+// so no CTA ever waits on another) merges the E/64 lists of each of its 128
+// tokens and writes ids and weights.  The merge picks exactly what a full
+// sort of the FP32 logits picks (descending, ties to the lower expert id), and
+// the weights use the same exponentials, summed in the same order, as
+// moe_route_topk, so both give the same bits.  The split-K form below keeps
+// the top-k in its own kernel: there no CTA holds a complete logit.
+//
 // Few tokens (decode): one 128-token tile row gives only E/64 CTAs, so the
 // K dimension is also split across CTAs (grid z = ksplit); each CTA then
 // writes its partial hi and lo sums, and the top-k kernel adds the ksplit
@@ -41,12 +53,110 @@ constexpr int MAX_CHUNKS = 4;
 constexpr uint32_t TMEM_COLS = 512;  // (MAX_CHUNKS + 1) * BN = 320 used
 constexpr size_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
 
+constexpr int CAND = 8;  // candidates kept per token and 64-expert tile (k <= 8)
+
+// Fused top-k: outputs, per-token candidate keys [T][E/64][CAND] and one
+// arrival counter per m-tile (zeroed by the launcher).
+struct TopkArgs {
+    int32_t* ids;              // [T][k]; nullptr: logits only (no fused top-k)
+    float* w;                  // [T][k]
+    unsigned long long* cand;  // [T][ntiles][CAND]
+    int32_t* arrive_m;         // [m-tiles]: CTAs of the m-tile done
+    int k, renorm;
+};
+
+// A logit and its expert id packed so that a larger key is a better choice:
+// the high word orders like the FP32 value, the low word is ~e, so equal
+// logits rank the lower id first.  Every real key is > 0; 0 marks "none".
+__device__ __forceinline__ unsigned long long topk_key(float v, int e) {
+    const uint32_t b = __float_as_uint(v);
+    const uint32_t ord = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+    return ((unsigned long long)ord << 32) | (uint32_t)~e;
+}
+
+__device__ __forceinline__ float key_value(unsigned long long key) {
+    const uint32_t ord = (uint32_t)(key >> 32);
+    return __uint_as_float((ord & 0x80000000u) ? (ord & 0x7fffffffu) : ~ord);
+}
+
+__device__ __forceinline__ int key_expert(unsigned long long key) { return (int)~(uint32_t)key; }
+
+// The best CAND of N keys, in order (keys are distinct: each carries its
+// expert id).  Each round takes the maximum by a tree of independent max
+// operations and knocks the winner out, so the rounds are short dependency
+// chains rather than one long insertion chain.
+template <int N>
+__device__ __forceinline__ void best_keys(unsigned long long (&k)[N], unsigned long long (&best)[CAND]) {
+#pragma unroll
+    for (int j = 0; j < CAND; ++j) {
+        unsigned long long m[N];
+#pragma unroll
+        for (int i = 0; i < N; ++i) m[i] = k[i];
+#pragma unroll
+        for (int w = 1; w < N; w <<= 1)
+#pragma unroll
+            for (int i = 0; i + w < N; i += 2 * w) m[i] = m[i] > m[i + w] ? m[i] : m[i + w];
+        best[j] = m[0];
+#pragma unroll
+        for (int i = 0; i < N; ++i) k[i] = k[i] == m[0] ? 0ull : k[i];
+    }
+}
+
+// Token t's routing from its candidate keys (read through L2: other CTAs
+// wrote them): the k best in order, then the weights.  Softmax over the
+// selected k (renorm) or over all E logits of the token (read back from
+// `logits`); the exponentials and the order of their sum are those of
+// moe_route_topk's warp reduction, so the weights agree to the bit.
+__device__ void merge_topk(const TopkArgs& tk, const float* logits, int64_t t, int ntiles, int E) {
+    unsigned long long k[4 * CAND], best[CAND];
+#pragma unroll
+    for (int i = 0; i < 4 * CAND; ++i)
+        k[i] = i < ntiles * CAND ? __ldcg(tk.cand + t * ntiles * CAND + i) : 0ull;
+    best_keys<4 * CAND>(k, best);
+    float sv[CAND];
+#pragma unroll
+    for (int j = 0; j < CAND; ++j) sv[j] = key_value(best[j]);
+    const float lmax = sv[0];
+    float sum;
+    if (tk.renorm) {
+        float p[CAND];
+#pragma unroll
+        for (int j = 0; j < CAND; ++j) p[j] = j < tk.k ? expf(sv[j] - lmax) : 0.0f;
+        // the xor-butterfly of a warp over lanes 0..7 (lanes >= k hold 0)
+        sum = ((p[0] + p[4]) + (p[2] + p[6])) + ((p[1] + p[5]) + (p[3] + p[7]));
+    } else {
+        // lane L sums experts L, L+32, ... in order; the lanes then add in
+        // pairs (L, L+16), (L, L+8), ... as the xor-butterfly does
+        float part[32];
+        const float* row = logits + t * E;
+#pragma unroll
+        for (int L = 0; L < 32; ++L) {
+            float acc = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                if (L + 32 * i < E) acc += expf(__ldcg(row + L + 32 * i) - lmax);
+            part[L] = acc;
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+            for (int L = 0; L < off; ++L) part[L] = part[L] + part[L + off];
+        sum = part[0];
+    }
+#pragma unroll
+    for (int j = 0; j < CAND; ++j)
+        if (j < tk.k) {
+            tk.ids[t * tk.k + j] = key_expert(best[j]);
+            tk.w[t * tk.k + j] = expf(sv[j] - lmax) / sum;
+        }
+}
+
 __global__ void __launch_bounds__(THREADS, 1)
     k_router_dual(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_hi,
                   const __grid_constant__ CUtensorMap tm_lo, const float* __restrict__ bias,
                   float* __restrict__ logits, float* __restrict__ part_hi,
                   float* __restrict__ part_lo, int T, int d, int E, int32_t* status,
-                  uint64_t timeout_ns) {
+                  uint64_t timeout_ns, const TopkArgs tk) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -78,6 +188,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem = *tmem_slot;
+    pdl_wait();  // x may come from the previous kernel in the stream
+    pdl_trigger();
 
     if (warp == 5 && lane == 0) {
         // ---------------- TMA producer
@@ -142,6 +254,10 @@ __global__ void __launch_bounds__(THREADS, 1)
             const int row = warp * 32 + lane;
             const int t = m0 + row;
             const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+            const bool fuse = tk.ids != nullptr && ksplit == 1;
+            unsigned long long best[CAND];
+#pragma unroll
+            for (int j = 0; j < CAND; ++j) best[j] = 0ull;
 #pragma unroll 1
             for (int c = 0; c < BN / 32; ++c) {
                 float h[32], l[32], h2[32], h3[32];
@@ -159,14 +275,22 @@ __global__ void __launch_bounds__(THREADS, 1)
                 }
                 if (t < T && ksplit == 1) {
                     float* dst = logits + (int64_t)t * E;
+                    unsigned long long keys[CAND + 32];
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
                         const int e = e0 + c * 32 + i;
+                        keys[CAND + i] = 0ull;
                         if (e < E) {
                             float v = fmaf(l[i], 0.00390625f, h[i]);
                             if (bias != nullptr) v += bias[e];
                             dst[e] = v;
+                            keys[CAND + i] = topk_key(v, e);
                         }
+                    }
+                    if (fuse) {   // the best CAND of this row's logits so far
+#pragma unroll
+                        for (int j = 0; j < CAND; ++j) keys[j] = best[j];
+                        best_keys<CAND + 32>(keys, best);
                     }
                 } else if (t < T) {
                     float* dh = part_hi + ((int64_t)ks * T + t) * E;
@@ -181,6 +305,12 @@ __global__ void __launch_bounds__(THREADS, 1)
                     }
                 }
             }
+            if (fuse && t < T) {
+                ulonglong2* dst = reinterpret_cast<ulonglong2*>(
+                    tk.cand + ((int64_t)t * gridDim.y + blockIdx.y) * CAND);
+#pragma unroll
+                for (int j = 0; j < CAND / 2; ++j) dst[j] = make_ulonglong2(best[2 * j], best[2 * j + 1]);
+            }
         }
     }
     tc_fence_before_sync();
@@ -189,23 +319,25 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_fence_after_sync();
         tmem_dealloc(tmem, TMEM_COLS);
     }
-}
+    if (tk.ids == nullptr || ksplit > 1 || *abort_flag) return;
 
-}  // namespace
-
-int router_ksplit(int T, int d, int E) {
-    const int tiles = ((T + BM - 1) / BM) * ((E + BN - 1) / BN);
-    const int nk = d / BK;
-    int ks = 1;
-    // split K while the grid fills less than half the SMs, keeping >= 4 k-blocks per CTA
-    while (ks < 8 && tiles * ks * 2 <= 148 && nk / (ks * 2) >= 4) ks *= 2;
-    return ks;
+    // ---------------- fused top-k: the last CTA of each tile row routes its 128 tokens
+    __shared__ int s_last;
+    const int ntiles = gridDim.y;
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_last = atomicAdd(&tk.arrive_m[blockIdx.x], 1) == ntiles - 1;
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    if (threadIdx.x < BM && m0 + (int)threadIdx.x < T)
+        merge_topk(tk, logits, m0 + threadIdx.x, ntiles, E);
 }
 
 static cudaError_t launch_router_impl(const uint16_t* x, const uint16_t* hi, const uint16_t* lo,
                                       const float* bias, float* logits, float* part_hi,
                                       float* part_lo, int ksplit, int T, int d, int E,
-                                      int32_t* status, cudaStream_t s) {
+                                      int32_t* status, const TopkArgs& tk, cudaStream_t s) {
     if (T == 0) return cudaSuccess;
     CUtensorMap tx, th, tl;
     if (!make_tmap_2d(&tx, x, 2, (uint64_t)T, (uint64_t)d, BM, BK) ||
@@ -221,22 +353,63 @@ static cudaError_t launch_router_impl(const uint16_t* x, const uint16_t* hi, con
         attr_set[dev] = true;
     }
     dim3 grid((T + BM - 1) / BM, (E + BN - 1) / BN, ksplit);
-    k_router_dual<<<grid, THREADS, SMEM_BYTES, s>>>(tx, th, tl, bias, logits, part_hi, part_lo, T, d,
-                                                    E, status, kDefaultTimeoutNs);
+    if (tk.ids != nullptr) {
+        cudaError_t e = cudaMemsetAsync(tk.arrive_m, 0, sizeof(int32_t) * grid.x, s);
+        if (e != cudaSuccess) return e;
+    }
+    {
+        const cudaError_t le = launch_pdl(k_router_dual, dim3(grid), dim3(THREADS), SMEM_BYTES, s,
+                                          tx, th, tl, bias, logits, part_hi, part_lo, T, d, E,
+                                          status, kDefaultTimeoutNs, tk);
+        if (le != cudaSuccess) return le;
+    }
     return cudaGetLastError();
+}
+
+}  // namespace
+
+int router_ksplit(int T, int d, int E) {
+    const int tiles = ((T + BM - 1) / BM) * ((E + BN - 1) / BN);
+    const int nk = d / BK;
+    int ks = 1;
+    // split K while the grid fills less than half the SMs, keeping >= 4 k-blocks per CTA
+    while (ks < 8 && tiles * ks * 2 <= 148 && nk / (ks * 2) >= 4) ks *= 2;
+    return ks;
+}
+
+size_t router_topk_scratch_bytes(int T, int E) {
+    const size_t mt = (size_t)(T + BM - 1) / BM, nt = (size_t)(E + BN - 1) / BN;
+    return (size_t)T * nt * CAND * 8 + mt * 4;
 }
 
 cudaError_t launch_router_logits(const uint16_t* x, const uint16_t* hi, const uint16_t* lo,
                                  const float* bias, float* logits, int T, int d, int E,
                                  int32_t* status, cudaStream_t s) {
-    return launch_router_impl(x, hi, lo, bias, logits, nullptr, nullptr, 1, T, d, E, status, s);
+    TopkArgs tk{};
+    return launch_router_impl(x, hi, lo, bias, logits, nullptr, nullptr, 1, T, d, E, status, tk, s);
 }
 
 cudaError_t launch_router_partials(const uint16_t* x, const uint16_t* hi, const uint16_t* lo,
                                    float* part_hi, float* part_lo, int ksplit, int T, int d, int E,
                                    int32_t* status, cudaStream_t s) {
+    TopkArgs tk{};
     return launch_router_impl(x, hi, lo, nullptr, nullptr, part_hi, part_lo, ksplit, T, d, E,
-                              status, s);
+                              status, tk, s);
+}
+
+cudaError_t launch_router_topk(const uint16_t* x, const uint16_t* hi, const uint16_t* lo,
+                               const float* bias, float* logits, int T, int d, int E, int k,
+                               int renorm, int32_t* ids, float* w, void* scratch, int32_t* status,
+                               cudaStream_t s) {
+    const size_t nt = (size_t)(E + BN - 1) / BN;
+    TopkArgs tk;
+    tk.ids = ids;
+    tk.w = w;
+    tk.cand = static_cast<unsigned long long*>(scratch);
+    tk.arrive_m = reinterpret_cast<int32_t*>(tk.cand + (size_t)T * nt * CAND);
+    tk.k = k;
+    tk.renorm = renorm;
+    return launch_router_impl(x, hi, lo, bias, logits, nullptr, nullptr, 1, T, d, E, status, tk, s);
 }
 
 }  // namespace moe

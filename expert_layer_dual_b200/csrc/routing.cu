@@ -233,6 +233,8 @@ int permute_segments(int64_t n) { return (int)((n + kSeg - 1) / kSeg); }
 __global__ void __launch_bounds__(256)
     k_perm_count(const int32_t* __restrict__ ids, int64_t n, int E, int32_t* __restrict__ seg_hist,
                  int32_t* status) {
+    pdl_wait();  // inputs come from the previous kernel of the forward
+    pdl_trigger();
     __shared__ int32_t hist[256];
     for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
     __syncthreads();
@@ -250,17 +252,30 @@ __global__ void __launch_bounds__(256)
         seg_hist[(int64_t)blockIdx.x * E + e] = hist[e];
 }
 
+// One thread per expert walks the segments in order: seg_hist[s][e] becomes
+// the number of expert-e assignments before segment s (loads issued 16 at a
+// time, so the walk costs a few memory round trips, not one per segment);
+// then the exclusive scan of the totals over the experts gives offsets.  The
+// scatter adds offsets[e] to its segment's bases itself.
 __global__ void __launch_bounds__(256)
     k_perm_scan(int32_t* __restrict__ seg_hist, int nseg, int E, int32_t* __restrict__ counts,
                 int32_t* __restrict__ offsets) {
+    pdl_wait();  // inputs come from the previous kernel of the forward
+    pdl_trigger();
     __shared__ int32_t buf[2][256];
     const int e = threadIdx.x;
     int32_t run = 0;
     if (e < E) {
-        for (int s = 0; s < nseg; ++s) {
-            const int32_t c = seg_hist[(int64_t)s * E + e];
-            seg_hist[(int64_t)s * E + e] = run;
-            run += c;
+        for (int s0 = 0; s0 < nseg; s0 += 16) {
+            int32_t c[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                c[i] = s0 + i < nseg ? seg_hist[(int64_t)(s0 + i) * E + e] : 0;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                if (s0 + i < nseg) seg_hist[(int64_t)(s0 + i) * E + e] = run;
+                run += c[i];
+            }
         }
         counts[e] = run;
     }
@@ -278,17 +293,18 @@ __global__ void __launch_bounds__(256)
     if (e < E) {
         offsets[e] = excl;
         if (e == E - 1) offsets[E] = excl + run;
-        for (int s = 0; s < nseg; ++s) seg_hist[(int64_t)s * E + e] += excl;
     }
 }
 
 __global__ void __launch_bounds__(32)
     k_perm_scatter(const int32_t* __restrict__ ids, int64_t n, int E,
-                   const int32_t* __restrict__ seg_base, int32_t* __restrict__ perm,
-                   int32_t* __restrict__ inv) {
+                   const int32_t* __restrict__ seg_base, const int32_t* __restrict__ offsets,
+                   int32_t* __restrict__ perm, int32_t* __restrict__ inv) {
+    pdl_wait();  // inputs come from the previous kernel of the forward
+    pdl_trigger();
     __shared__ int32_t cur[256];
     const int lane = threadIdx.x;
-    for (int e = lane; e < E; e += 32) cur[e] = seg_base[(int64_t)blockIdx.x * E + e];
+    for (int e = lane; e < E; e += 32) cur[e] = seg_base[(int64_t)blockIdx.x * E + e] + offsets[e];
     __syncwarp();
     const int64_t a0 = (int64_t)blockIdx.x * kSeg;
     const int64_t a1 = (a0 + kSeg < n) ? a0 + kSeg : n;
@@ -317,6 +333,8 @@ __global__ void __launch_bounds__(256)
     k_perm_small(const int32_t* __restrict__ ids, int n, int E, int32_t* __restrict__ counts,
                  int32_t* __restrict__ offsets, int32_t* __restrict__ perm,
                  int32_t* __restrict__ inv, int32_t* status) {
+    pdl_wait();  // inputs come from the previous kernel of the forward
+    pdl_trigger();
     __shared__ int32_t hist[256];
     __shared__ int32_t buf[2][256];
     const int e = threadIdx.x;
@@ -375,12 +393,28 @@ cudaError_t launch_permute(const int32_t* ids, int T, int E, int k, int32_t* cou
     const int64_t n = (int64_t)T * k;
     const int nseg = permute_segments(n);
     if (nseg <= 1) {
-        k_perm_small<<<1, 256, 0, s>>>(ids, (int)n, E, counts, offsets, perm, inv, status);
+        {
+            const cudaError_t le = launch_pdl(k_perm_small, dim3(1), dim3(256), 0, s, ids, (int)n,
+                                              E, counts, offsets, perm, inv, status);
+            if (le != cudaSuccess) return le;
+        }
         return cudaGetLastError();
     }
-    k_perm_count<<<nseg, 256, 0, s>>>(ids, n, E, seg_hist, status);
-    k_perm_scan<<<1, 256, 0, s>>>(seg_hist, nseg, E, counts, offsets);
-    k_perm_scatter<<<nseg, 32, 0, s>>>(ids, n, E, seg_hist, perm, inv);
+    {
+        const cudaError_t le = launch_pdl(k_perm_count, dim3(nseg), dim3(256), 0, s, ids, n, E,
+                                          seg_hist, status);
+        if (le != cudaSuccess) return le;
+    }
+    {
+        const cudaError_t le = launch_pdl(k_perm_scan, dim3(1), dim3(256), 0, s, seg_hist, nseg, E,
+                                          counts, offsets);
+        if (le != cudaSuccess) return le;
+    }
+    {
+        const cudaError_t le = launch_pdl(k_perm_scatter, dim3(nseg), dim3(32), 0, s, ids, n, E,
+                                          seg_hist, offsets, perm, inv);
+        if (le != cudaSuccess) return le;
+    }
     return cudaGetLastError();
 }
 
@@ -413,6 +447,8 @@ __global__ void __launch_bounds__(128)
     k_combine(const __half* __restrict__ o, const int32_t* __restrict__ inv,
               const float* __restrict__ w, uint16_t* __restrict__ y, int T, int d, int k,
               int has_shared) {
+    pdl_wait();  // inputs come from the previous kernel of the forward
+    pdl_trigger();
     __shared__ int32_t rows[8];
     __shared__ float wts[8];
     const int t = blockIdx.x;
@@ -461,7 +497,11 @@ cudaError_t launch_combine(const __half* o, const int32_t* inv, const float* w, 
     const int passes = (d + 1023) / 1024;
     const int want = (2 * current_device_info().num_sms + T - 1) / T;
     const int ysplit = want < passes ? want : passes;
-    k_combine<<<dim3(T, ysplit > 1 ? ysplit : 1), 128, 0, s>>>(o, inv, w, y, T, d, k, has_shared);
+    {
+        const cudaError_t le = launch_pdl(k_combine, dim3(T, ysplit > 1 ? ysplit : 1), dim3(128), 0,
+                                          s, o, inv, w, y, T, d, k, has_shared);
+        if (le != cudaSuccess) return le;
+    }
     return cudaGetLastError();
 }
 
@@ -531,6 +571,8 @@ __global__ void __launch_bounds__(256)
     k_quant_act_permuted(const uint16_t* __restrict__ x, const int32_t* __restrict__ perm, int T,
                          int k, int64_t rows, int cols, uint8_t* __restrict__ q,
                          float* __restrict__ scale) {
+    pdl_wait();  // inputs come from the previous kernel of the forward
+    pdl_trigger();
     const int64_t p = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
     if (p >= rows) return;
     const int64_t Tk = (int64_t)T * k;
@@ -543,8 +585,11 @@ cudaError_t launch_quant_act_fp8_permuted(const uint16_t* x, const int32_t* perm
                                           cudaStream_t s) {
     const int64_t rows = (int64_t)T * k + (has_shared ? T : 0);
     if (rows == 0) return cudaSuccess;
-    k_quant_act_permuted<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(x, perm, T, k, rows, cols, q,
-                                                                     scale);
+    {
+        const cudaError_t le = launch_pdl(k_quant_act_permuted, dim3((unsigned)((rows + 7) / 8)),
+                                          dim3(256), 0, s, x, perm, T, k, rows, cols, q, scale);
+        if (le != cudaSuccess) return le;
+    }
     return cudaGetLastError();
 }
 
@@ -626,6 +671,8 @@ __global__ void __launch_bounds__(256)
     k_quant_mx_permuted(const uint16_t* __restrict__ x, const int32_t* __restrict__ perm, int T,
                         int k, int64_t rows, int cols, uint8_t* __restrict__ q,
                         uint8_t* __restrict__ scale) {
+    pdl_wait();  // inputs come from the previous kernel of the forward
+    pdl_trigger();
     const int64_t p = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
     if (p >= rows) return;
     const int64_t Tk = (int64_t)T * k;
@@ -655,8 +702,11 @@ cudaError_t launch_quant_mx_permuted(const uint16_t* x, const int32_t* perm, int
                                      cudaStream_t s) {
     const int64_t rows = (int64_t)T * k + (has_shared ? T : 0);
     if (rows == 0) return cudaSuccess;
-    k_quant_mx_permuted<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(x, perm, T, k, rows, cols, q,
-                                                                   scale);
+    {
+        const cudaError_t le = launch_pdl(k_quant_mx_permuted, dim3((unsigned)((rows + 7) / 8)),
+                                          dim3(256), 0, s, x, perm, T, k, rows, cols, q, scale);
+        if (le != cudaSuccess) return le;
+    }
     return cudaGetLastError();
 }
 
@@ -706,6 +756,12 @@ __global__ void k_scale_from_amax(float* __restrict__ scale, int64_t batch) {
     if (m < batch) scale[m] = group_scale(scale[m]);
 }
 
+// amax (as float bits) -> the static scale, for one value.
+static cudaError_t launch_one_scale(float* scale, cudaStream_t s) {
+    k_scale_from_amax<<<1, 32, 0, s>>>(scale, 1);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_quant_weights_fp8_tensor(const uint16_t* W, int64_t batch, int rows, int cols,
                                             uint8_t* q, float* scale, cudaStream_t s) {
     const int64_t per = (int64_t)rows * cols;
@@ -719,6 +775,15 @@ cudaError_t launch_quant_weights_fp8_tensor(const uint16_t* W, int64_t batch, in
     k_quant_matrices<<<grid, 256, 0, s>>>(W, per, reinterpret_cast<const uint32_t*>(scale), q);
     k_scale_from_amax<<<(unsigned)((batch + 255) / 256), 256, 0, s>>>(scale, batch);
     return cudaGetLastError();
+}
+
+cudaError_t launch_amax_scale(const uint16_t* v, int64_t n, float* scale, cudaStream_t s) {
+    cudaError_t e = cudaMemsetAsync(scale, 0, sizeof(float), s);
+    if (e != cudaSuccess || n == 0) return e == cudaSuccess ? launch_one_scale(scale, s) : e;
+    const int64_t want = (n / 8 + 255) / 256;
+    const unsigned bx = (unsigned)(want < 1024 ? want : 1024);
+    k_amax_matrices<<<dim3(bx, 1), 256, 0, s>>>(v, n, reinterpret_cast<uint32_t*>(scale));
+    return launch_one_scale(scale, s);
 }
 
 // v / s rounded to nearest in FP32 -- the IEEE quotient -- for a divisor that
@@ -754,6 +819,8 @@ __device__ __forceinline__ uint32_t quant4_e4m3_fixed(float a, float b, float c,
 __global__ void __launch_bounds__(256)
     k_quant_static(const uint16_t* __restrict__ x, const int32_t* __restrict__ perm, int T, int k,
                    int64_t rows, int cols, float s, uint8_t* __restrict__ q) {
+    pdl_wait();  // inputs come from the previous kernel of the forward
+    pdl_trigger();
     const int64_t p = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
     if (p >= rows) return;
     const int lane = threadIdx.x & 31;
@@ -777,7 +844,11 @@ cudaError_t launch_quant_act_fp8_static(const uint16_t* x, const int32_t* perm, 
                                         int64_t rows, int cols, float scale, uint8_t* q,
                                         cudaStream_t s) {
     if (rows == 0) return cudaSuccess;
-    k_quant_static<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(x, perm, T, k, rows, cols, scale, q);
+    {
+        const cudaError_t le = launch_pdl(k_quant_static, dim3((unsigned)((rows + 7) / 8)),
+                                          dim3(256), 0, s, x, perm, T, k, rows, cols, scale, q);
+        if (le != cudaSuccess) return le;
+    }
     return cudaGetLastError();
 }
 

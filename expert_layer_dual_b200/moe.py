@@ -39,7 +39,11 @@ EXPORTS = ["moe_status_string", "moe_workspace_bytes", "moe_permute_workspace_by
            "moe_gemm_gateup",
            "moe_gemm_down", "moe_combine", "moe_forward", "moe_forward_profiled", "moe_forward_host",
            "moe_forward_host_async",
-           "moe_read_device_status", "moe_selftest_timeout"]
+           "moe_read_device_status", "moe_selftest_timeout", "moe_workspace_offsets",
+           "moe_calibrate_fp8_static", "moe_route", "moe_ep_dispatch", "moe_gather_rows",
+           "moe_lamport_buffer_bytes", "moe_lamport_init", "moe_allreduce_rmsnorm",
+           "moe_allreduce_rmsnorm_emulated", "moe_peer_buffer_alloc", "moe_peer_buffer_open",
+           "moe_peer_buffer_close", "moe_peer_buffer_free"]
 
 
 class moe_shape(ctypes.Structure):
@@ -53,6 +57,11 @@ class moe_weights(ctypes.Structure):
                 ("w_gu", "w_d", "w_gu_scale", "w_d_scale", "ws_gu", "ws_d", "ws_gu_scale",
                  "ws_d_scale", "router_hi", "router_lo", "router_bias")] + \
                [("act_scale_x", ctypes.c_float), ("act_scale_h", ctypes.c_float)]
+
+
+class moe_workspace_map(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_size_t) for n in
+                ("logits", "ids", "w", "counts", "offsets", "perm", "inv", "h", "total")]
 
 
 _vp, _i32, _i64, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
@@ -85,6 +94,23 @@ _sig = {
     "moe_forward_host_async": (_i32, [_S, _W, _vp, _vp, _vp, _sz, _vp]),
     "moe_read_device_status": (_i32, [_vp, _vp]),
     "moe_selftest_timeout": (_i32, [_vp, _i32, _vp]),
+    "moe_workspace_offsets": (_i32, [_S, ctypes.POINTER(moe_workspace_map)]),
+    "moe_calibrate_fp8_static": (_i32, [_S, _W, _vp, _vp, _vp, _sz, _vp]),
+    "moe_route": (_i32, [_S, _W, _vp, _vp, _sz, _vp]),
+    "moe_ep_dispatch": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
+    "moe_gather_rows": (_i32, [_vp, _vp, _i64, _i32, _vp, _vp]),
+    "moe_lamport_buffer_bytes": (_sz, [_i32, _i32, _i32]),
+    "moe_lamport_init": (_i32, [_vp, _sz, _vp]),
+    "moe_allreduce_rmsnorm": (_i32, [ctypes.POINTER(_vp), _i32, _i32, ctypes.c_uint32, _i32, _vp, _vp,
+                                     _vp, ctypes.c_float, _i32, _i32, _vp, _vp, _vp, _sz, _vp]),
+    "moe_allreduce_rmsnorm_emulated": (_i32, [ctypes.POINTER(_vp), _i32, _i32, ctypes.c_uint32, _i32,
+                                              ctypes.POINTER(_vp), ctypes.POINTER(_vp), _vp,
+                                              ctypes.c_float, _i32, _i32, ctypes.POINTER(_vp),
+                                              ctypes.POINTER(_vp), _i32, _vp, _sz, _vp]),
+    "moe_peer_buffer_alloc": (_i32, [_sz, ctypes.POINTER(_vp), _vp]),
+    "moe_peer_buffer_open": (_i32, [_vp, ctypes.POINTER(_vp)]),
+    "moe_peer_buffer_close": (_i32, [_vp]),
+    "moe_peer_buffer_free": (_i32, [_vp]),
 }
 for _name, (_res, _args) in _sig.items():
     _f = getattr(_lib, _name)
@@ -128,6 +154,127 @@ def shape_of(cfg: MoEConfig, T: Optional[int] = None) -> moe_shape:
 # ------------------------------------------------------------------ entry points
 def workspace_bytes(shape: moe_shape) -> int:
     return int(_lib.moe_workspace_bytes(ctypes.byref(shape)))
+
+
+def workspace_offsets(shape: moe_shape) -> moe_workspace_map:
+    m = moe_workspace_map()
+    _check(_lib.moe_workspace_offsets(ctypes.byref(shape), ctypes.byref(m)), "moe_workspace_offsets")
+    return m
+
+
+def workspace_view(ws: torch.Tensor, shape: moe_shape) -> dict:
+    """Views (no copies) of the routing intermediates and h that moe_forward
+    leaves in `ws`, at the offsets moe_workspace_offsets reports."""
+    m = workspace_offsets(shape)
+    T, E, k = shape.T, shape.E, shape.k
+    R = T * k + (T if shape.I_shared else 0)
+
+    def region(off, n, dtype):
+        nbytes = n * torch.empty((), dtype=dtype).element_size()
+        return ws[off: off + nbytes].view(dtype)
+
+    out = {"logits": region(m.logits, T * E, torch.float32).view(T, E),
+           "ids": region(m.ids, T * k, torch.int32).view(T, k),
+           "w": region(m.w, T * k, torch.float32).view(T, k),
+           "counts": region(m.counts, E, torch.int32),
+           "offsets": region(m.offsets, E + 1, torch.int32),
+           "perm": region(m.perm, T * k, torch.int32),
+           "inv": region(m.inv, T * k, torch.int32)}
+    if shape.wdtype == WDTYPE_BF16:
+        out["h"] = region(m.h, R * shape.I, torch.bfloat16).view(R, shape.I)
+    return out
+
+
+def calibrate_fp8_static(shape, weights, x, scales, ws, stream=None):
+    """moe_calibrate_fp8_static: scales (float32 [2], device) <- the static
+    activation scales of x and of the BF16 gate-up output h."""
+    _check(_lib.moe_calibrate_fp8_static(ctypes.byref(shape), ctypes.byref(weights), _p(x), _p(scales),
+                                         _p(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "moe_calibrate_fp8_static")
+
+
+def route(shape, weights, x, ws, stream=None):
+    """moe_route: router logits, fused top-k and permute into `ws`."""
+    _check(_lib.moe_route(ctypes.byref(shape), ctypes.byref(weights), _p(x), _p(ws),
+                          ws.numel() * ws.element_size(), _stream(stream)), "moe_route")
+
+
+def ep_dispatch(x, ids, perm, E_local, send_rows, send_ids, stream=None):
+    T, d = x.shape
+    k = ids.shape[1]
+    _check(_lib.moe_ep_dispatch(_p(x), _p(ids), _p(perm), T, d, k, E_local, _p(send_rows),
+                                _p(send_ids), _stream(stream)), "moe_ep_dispatch")
+
+
+def gather_rows(src, index, dst, stream=None):
+    n = index.numel()
+    row_bytes = dst.numel() * dst.element_size() // max(n, 1) if n else 16
+    _check(_lib.moe_gather_rows(_p(src), _p(index), n, row_bytes, _p(dst), _stream(stream)),
+           "moe_gather_rows")
+
+
+def _ptrs(items) -> "ctypes.Array":
+    """HOST array of device pointers (ints or tensors; None -> NULL)."""
+    vals = [None if v is None else (v if isinstance(v, int) else v.data_ptr()) for v in items]
+    return (_vp * len(vals))(*vals)
+
+
+def lamport_buffer_bytes(G: int, T_max: int, d: int) -> int:
+    return int(_lib.moe_lamport_buffer_bytes(G, T_max, d))
+
+
+def lamport_init(buf, nbytes: int, stream=None):
+    ptr = buf if isinstance(buf, int) else buf.data_ptr()
+    _check(_lib.moe_lamport_init(ctypes.c_void_p(ptr), nbytes, _stream(stream)), "moe_lamport_init")
+
+
+def allreduce_rmsnorm(bufs, rank, call, T_max, x, residual, gamma, eps, out, residual_out, ws,
+                      stream=None):
+    """One rank's moe_allreduce_rmsnorm; `bufs`: every rank's Lamport buffer
+    (device pointers as ints, or tensors) in rank order."""
+    T, d = x.shape
+    _check(_lib.moe_allreduce_rmsnorm(_ptrs(bufs), len(bufs), rank, call & 0xffffffff, T_max, _p(x),
+                                      _p(residual), _p(gamma), float(eps), T, d, _p(out),
+                                      _p(residual_out), _p(ws), ws.numel() * ws.element_size(),
+                                      _stream(stream)), "moe_allreduce_rmsnorm")
+
+
+def allreduce_rmsnorm_emulated(bufs, call, T_max, xs, residuals, gamma, eps, outs, residual_outs,
+                               ws, ranks=None, timeout_us=2_000_000, stream=None):
+    """moe_allreduce_rmsnorm_emulated: every rank of the group in one launch
+    on this GPU (lists indexed by rank; `ranks` < len(bufs) leaves the last
+    ranks out)."""
+    G = len(bufs)
+    n = G if ranks is None else ranks
+    T, d = xs[0].shape
+    _check(_lib.moe_allreduce_rmsnorm_emulated(
+        _ptrs(bufs), G, n, call & 0xffffffff, T_max, _ptrs(xs[:n]),
+        None if residuals is None else _ptrs(residuals[:n]), _p(gamma), float(eps), T, d,
+        _ptrs(outs[:n]), None if residual_outs is None else _ptrs(residual_outs[:n]), int(timeout_us),
+        _p(ws), ws.numel() * ws.element_size(), _stream(stream)), "moe_allreduce_rmsnorm_emulated")
+
+
+def peer_buffer_alloc(nbytes: int):
+    """(device pointer, 64-byte IPC handle) of a new cudaMalloc'd buffer."""
+    ptr = ctypes.c_void_p()
+    handle = ctypes.create_string_buffer(64)
+    _check(_lib.moe_peer_buffer_alloc(nbytes, ctypes.byref(ptr), handle), "moe_peer_buffer_alloc")
+    return int(ptr.value), handle.raw
+
+
+def peer_buffer_open(handle: bytes) -> int:
+    ptr = ctypes.c_void_p()
+    buf = ctypes.create_string_buffer(bytes(handle), 64)
+    _check(_lib.moe_peer_buffer_open(buf, ctypes.byref(ptr)), "moe_peer_buffer_open")
+    return int(ptr.value)
+
+
+def peer_buffer_close(ptr: int):
+    _check(_lib.moe_peer_buffer_close(ctypes.c_void_p(ptr)), "moe_peer_buffer_close")
+
+
+def peer_buffer_free(ptr: int):
+    _check(_lib.moe_peer_buffer_free(ctypes.c_void_p(ptr)), "moe_peer_buffer_free")
 
 
 def permute_workspace_bytes(T: int, E: int, k: int) -> int:
@@ -288,9 +435,12 @@ class MoELayer:
     `inputs` holds the BF16 expert weights and the FP32 router weight (as
     drawn by expert_layer_dual_b200.inputs.make_layer).  Preparation runs the
     library's offline kernels: the dual-BF16 router split and, for FP8
-    layers, the 128x128 block quantisation of every expert matrix."""
+    layers, the 128x128 block quantisation of every expert matrix.  `act_scales`:
+    the static activation scales of a per-tensor FP8 layer when they are known
+    already (otherwise calibrated here on the input's first tokens)."""
 
-    def __init__(self, cfg: MoEConfig, inputs: dict, device="cuda", max_tokens: Optional[int] = None):
+    def __init__(self, cfg: MoEConfig, inputs: dict, device="cuda", max_tokens: Optional[int] = None,
+                 act_scales=None):
         self.cfg = cfg
         dev = torch.device(device)
         self.max_tokens = cfg.T if max_tokens is None else max_tokens
@@ -330,7 +480,8 @@ class MoELayer:
                 self.mats[name], self.scales[name] = t.view(torch.uint16), None
         self.act_scales = (1.0, 1.0)
         if cfg.wdtype == WDTYPE_FP8_TENSOR:
-            self.act_scales = self._calibrate_static_scales(cfg, inputs, dev)
+            self.act_scales = (tuple(act_scales) if act_scales is not None
+                               else self._calibrate_static_scales(cfg, inputs, dev))
         self.weights = moe_weights(*[_p(v) for v in (
             self.mats["w_gu"], self.mats["w_d"], self.scales["w_gu"], self.scales["w_d"],
             self.mats["ws_gu"], self.mats["ws_d"], self.scales["ws_gu"], self.scales["ws_d"],
@@ -343,38 +494,22 @@ class MoELayer:
     CALIBRATION_TOKENS = 64
 
     def _calibrate_static_scales(self, cfg: MoEConfig, inputs: dict, dev):
-        """Static activation scales of the per-tensor FP8 layer, calibrated on the
-        first CALIBRATION_TOKENS tokens of the input: amax(x) / 448 and amax(h) / 448,
-        h the gate-up output of those tokens computed with the BF16 weights by this
-        library's own stages (router, top-k, permute, BF16 gate-up)."""
+        """Static activation scales of the per-tensor FP8 layer, calibrated by
+        moe_calibrate_fp8_static on the first CALIBRATION_TOKENS tokens of the
+        input with the BF16 weights; the two device floats are copied to the
+        host, where moe_weights carries them."""
         x = inputs["x"][: self.CALIBRATION_TOKENS].to(dev, torch.bfloat16).contiguous()
-        T, E, k = x.shape[0], cfg.E, cfg.k
-        amax_x = float(x.float().abs().max().item())
         bf = {n: (None if inputs.get(n) is None else inputs[n].to(dev, torch.bfloat16).contiguous())
               for n in ("w_gu", "w_d", "ws_gu", "ws_d")}
         w16 = moe_weights(_p(bf["w_gu"]), _p(bf["w_d"]), None, None, _p(bf["ws_gu"]), _p(bf["ws_d"]),
                           None, None, _p(self.router_hi), _p(self.router_lo), _p(self.router_bias),
                           1.0, 1.0)
-        shape16 = moe_shape(T, cfg.d, E, k, cfg.I, cfg.Is, WDTYPE_BF16, int(cfg.renorm))
-        logits = torch.empty((T, E), dtype=torch.float32, device=dev)
-        router_logits(x.view(torch.uint16), self.router_hi, self.router_lo, self.router_bias, logits)
-        ids = torch.empty((T, k), dtype=torch.int32, device=dev)
-        wts = torch.empty((T, k), dtype=torch.float32, device=dev)
-        route_topk(logits, k, int(cfg.renorm), ids, wts)
-        counts = torch.empty(E, dtype=torch.int32, device=dev)
-        offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
-        perm = torch.empty(T * k, dtype=torch.int32, device=dev)
-        inv = torch.empty(T * k, dtype=torch.int32, device=dev)
-        pws = torch.empty(permute_workspace_bytes(T, E, k), dtype=torch.uint8, device=dev)
-        permute(ids, E, counts, offsets, perm, inv, pws)
-        R = T * k + (T if cfg.Is else 0)
-        h = torch.empty((R, cfg.I), dtype=torch.bfloat16, device=dev)
-        ws = torch.empty(4096, dtype=torch.uint8, device=dev)
-        gemm_gateup(shape16, w16, x.view(torch.uint16), None, perm, offsets, h.view(torch.uint16),
-                    None, ws)
-        amax_h = float(h.float().abs().max().item())
-        sx = amax_x / 448.0 if amax_x > 0 else 1.0
-        sh = amax_h / 448.0 if amax_h > 0 else 1.0
+        shape16 = moe_shape(x.shape[0], cfg.d, cfg.E, cfg.k, cfg.I, cfg.Is, WDTYPE_BF16,
+                            int(cfg.renorm))
+        ws = torch.empty(workspace_bytes(shape16), dtype=torch.uint8, device=dev)
+        scales = torch.empty(2, dtype=torch.float32, device=dev)
+        calibrate_fp8_static(shape16, w16, x.view(torch.uint16), scales, ws)
+        sx, sh = scales.cpu().tolist()
         return (sx, sh)
 
     def shape(self, T: int) -> moe_shape:

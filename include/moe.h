@@ -120,6 +120,25 @@ const char* moe_status_string(moe_status s);
  * across calls that are ordered on one stream. */
 size_t moe_workspace_bytes(const moe_shape* shape);
 
+/* Where moe_forward (and moe_forward_profiled / moe_forward_host) leaves
+ * the layer's intermediates in its workspace: byte offsets from the
+ * workspace's start, each region 256-byte aligned.  After a forward on
+ * `shape` returns and its stream has reached that point, until the
+ * workspace is used again:
+ *   logits float [T][E]   the router logits the routing was decided on
+ *                         (bias included)
+ *   ids int32 [T][k], w float [T][k]           moe_route_topk's outputs
+ *   counts int32 [E], offsets int32 [E+1], perm, inv int32 [T*k]
+ *                                              moe_permute's outputs
+ *   h   the gate-up output (wdtype 0: bf16 [R][I], R = T*k + (I_shared ? T : 0))
+ *   total  = moe_workspace_bytes(shape).
+ * Inspection and testing aid; returns MOE_ERR_INVALID_ARG / UNSUPPORTED as
+ * moe_workspace_bytes would return 0. */
+typedef struct moe_workspace_map {
+    size_t logits, ids, w, counts, offsets, perm, inv, h, total;
+} moe_workspace_map;
+moe_status moe_workspace_offsets(const moe_shape* shape, moe_workspace_map* map);
+
 /* Workspace bytes moe_permute needs for T tokens, E experts, top-k. */
 size_t moe_permute_workspace_bytes(int32_t T, int32_t E, int32_t k);
 
@@ -175,6 +194,24 @@ moe_status moe_quantize_act_mxfp8_permuted(const uint16_t* x, const int32_t* per
  * scale float [batch] (also used as scratch while it runs). */
 moe_status moe_quantize_weights_fp8_tensor(const uint16_t* W, int64_t batch, int32_t rows,
                                            int32_t cols, uint8_t* q, float* scale, void* stream);
+
+/* [HY] Calibration of the static activation scales of a per-tensor FP8 layer
+ * ("腾讯混元大模型：从多场景适配到高效部署的全栈技术解析", section 量化压缩技术实践 /
+ * FP8量化方案: static FP8 scales precomputed from calibration data; the page
+ * gives no recipe, so the plainest one is used).  On the shape->T tokens of
+ * x [T][d] (bf16, 16-byte aligned), with the layer's BF16 weights (shape->wdtype
+ * must be MOE_WDTYPE_BF16; `weights` the BF16 originals of the experts and the
+ * router split), runs the router, top-k, permute and the BF16 gate-up, then
+ * writes two device floats:
+ *   scales[0] = fp32(max |x|) / 448,   scales[1] = fp32(max |h|) / 448
+ * over every element of x and of the bf16 gate-up output h [R][I] (routed and
+ * shared rows), divided in FP32 (IEEE), 1 where the maximum is 0.  These are
+ * the act_scale_x and act_scale_h of moe_weights for wdtype 3.  ws:
+ * moe_workspace_bytes(shape); T == 0 is MOE_ERR_INVALID_ARG (nothing to
+ * calibrate on).  Asynchronous on `stream`. */
+moe_status moe_calibrate_fp8_static(const moe_shape* shape, const moe_weights* weights,
+                                    const uint16_t* x, float* scales, void* ws, size_t ws_bytes,
+                                    void* stream);
 
 /* [HY] Static activation quantisation with a calibrated scale (> 0):
  * q = e4m3_rne_satfinite(fp32(x / scale)); x [rows][cols] bf16, cols % 8 == 0. */
@@ -321,6 +358,96 @@ moe_status moe_forward_host(const moe_shape* shape, const moe_weights* weights,
 moe_status moe_forward_host_async(const moe_shape* shape, const moe_weights* weights,
                                   const uint16_t* x_host, uint16_t* y_host, void* ws,
                                   size_t ws_bytes, void* stream);
+
+/* [FM][FP] The routing part of moe_forward alone: router logits with the
+ * top-k fused into the router kernel, then the permute, into the workspace
+ * regions moe_workspace_offsets reports (logits, ids, w, counts, offsets,
+ * perm, inv).  Needs only the router weights of `weights`.  ws:
+ * moe_workspace_bytes(shape).  Used by expert parallelism, which routes
+ * locally and runs the experts where they live. */
+moe_status moe_route(const moe_shape* shape, const moe_weights* weights, const uint16_t* x,
+                     void* ws, size_t ws_bytes, void* stream);
+
+/* Expert parallelism ("HPC-Ops ...", HPC-Ops的主要功能, "GroupGEMM FP8": the
+ * grouped GEMM suits expert parallelism; "PR #54160 完整报告", 实现拆解: the
+ * layer deployed over 8 GPUs).  Experts are split into contiguous ranges of
+ * E_local per rank (rank r owns r*E_local .. (r+1)*E_local-1).  With the
+ * routing of moe_route (ids [T][k], perm [T*k]), the permuted row order is
+ * grouped by expert and therefore by owning rank:
+ *   send_rows[p] = x[perm[p] / k]   (bf16 [T*k][d], d % 8 == 0)
+ *   send_ids[p]  = ids[perm[p]] % E_local  (the expert's id at its owner)
+ * Rows offsets[r*E_local] .. offsets[(r+1)*E_local]-1 go to rank r.  x and
+ * send_rows 16-byte aligned. */
+moe_status moe_ep_dispatch(const uint16_t* x, const int32_t* ids, const int32_t* perm, int32_t T,
+                           int32_t d, int32_t k, int32_t E_local, uint16_t* send_rows,
+                           int32_t* send_ids, void* stream);
+
+/* Row gather: dst[i] = src[index[i]] for i < n, rows of row_bytes bytes (a
+ * multiple of 16; src and dst 16-byte aligned).  Expert parallelism uses it
+ * to put the expert outputs of received rows back in arrival order (index =
+ * the inverse permutation of their local grouping) before returning them. */
+moe_status moe_gather_rows(const void* src, const int32_t* index, int64_t n, int32_t row_bytes,
+                           void* dst, void* stream);
+
+/* [AN] Tensor-parallel all-reduce fused with the residual add and RMSNorm,
+ * low-latency P2P form ("HPC-Ops - 騰訊混元開源的工業級高性能大模型推理算子庫",
+ * HPC-Ops的技術原理, "Fused AllReduce+Norm": RMSNorm(AllReduce(x) + residual,
+ * weight) as one NVLink operation; the decode version exchanges data by
+ * Lamport P2P stores and overlaps the previous kernel through PDL).  Per token
+ * t of each of the G ranks' x_r [T][d] bf16:
+ *   s = sum_{r<G} x_r[t] + residual[t]   (FP32, ranks summed in order 0..G-1,
+ *                                        then the residual: every rank gets the
+ *                                        same bits)
+ *   residual_out[t] = RNE_bf16(s),  out[t] = RNE_bf16(s * rsqrt(mean(s^2) + eps) * gamma)
+ * Transport: every rank owns a Lamport buffer of moe_lamport_buffer_bytes(G,
+ * T_max, d) bytes, filled once with moe_lamport_init; every rank maps every
+ * other rank's buffer (CUDA IPC: moe_peer_buffer_alloc / _open).  Call number
+ * `call` must be the same on all ranks and advance by one per call.  No
+ * multicast and no TMA: plain 16-byte stores to peer memory and polling loads
+ * of local memory.  Limits: 1 <= G <= 8, d % 8 == 0, d <= 8192, T <= T_max,
+ * every pointer 16-byte aligned.  Each wait for a peer's data is bounded (2 s):
+ * it then records MOE_ERR_DEVICE_TIMEOUT in ws's status word (not cleared by
+ * this call, so that nothing separates it from the previous kernel; the
+ * buffers must be re-initialised after a timeout).  Launched with
+ * programmatic dependent launch: it may start while the previous kernel in
+ * `stream` finishes and waits for it before reading x or the residual.
+ *   bufs: HOST array of G device pointers, the buffers of ranks 0..G-1 as
+ *         mapped in this process (bufs[rank] its own);
+ *   residual, residual_out: may be NULL (no residual / not written);
+ *   gamma [d] bf16; ws >= 256 bytes. */
+size_t moe_lamport_buffer_bytes(int32_t G, int32_t T_max, int32_t d);
+moe_status moe_lamport_init(void* buf, size_t bytes, void* stream);
+moe_status moe_allreduce_rmsnorm(void* const* bufs, int32_t G, int32_t rank, uint32_t call,
+                                 int32_t T_max, const uint16_t* x, const uint16_t* residual,
+                                 const uint16_t* gamma, float eps, int32_t T, int32_t d,
+                                 uint16_t* out, uint16_t* residual_out, void* ws, size_t ws_bytes,
+                                 void* stream);
+
+/* The same kernel for `ranks` ranks of a G-rank group emulated on ONE GPU, in
+ * one cooperative launch (every rank's blocks resident at once, so the ranks
+ * can wait on one another): bufs, x, residual, out, residual_out are HOST
+ * arrays of device pointers indexed by rank (residual / residual_out arrays may
+ * be NULL).  ranks < G leaves the missing ranks' data unsent, so the others'
+ * waits run out after timeout_us and report MOE_ERR_DEVICE_TIMEOUT (the
+ * failure path, without a GPU fault).  Clears ws's status word first.  For
+ * tests of the protocol on one GPU. */
+moe_status moe_allreduce_rmsnorm_emulated(void* const* bufs, int32_t G, int32_t ranks,
+                                          uint32_t call, int32_t T_max, const uint16_t* const* x,
+                                          const uint16_t* const* residual, const uint16_t* gamma,
+                                          float eps, int32_t T, int32_t d, uint16_t* const* out,
+                                          uint16_t* const* residual_out, int32_t timeout_us,
+                                          void* ws, size_t ws_bytes, void* stream);
+
+/* Peer-memory set-up for moe_allreduce_rmsnorm (set-up time only; the one
+ * place this library allocates): moe_peer_buffer_alloc cudaMallocs `bytes`
+ * on the current device and writes the 64-byte CUDA IPC handle of it;
+ * another process opens it with moe_peer_buffer_open (mapped with peer access)
+ * and unmaps it with moe_peer_buffer_close; the owner frees it with
+ * moe_peer_buffer_free after every mapping is closed. */
+moe_status moe_peer_buffer_alloc(size_t bytes, void** ptr, void* ipc_handle);
+moe_status moe_peer_buffer_open(const void* ipc_handle, void** ptr);
+moe_status moe_peer_buffer_close(void* ptr);
+moe_status moe_peer_buffer_free(void* ptr);
 
 /* Synchronises `stream` and returns the device status word of `ws`
  * (MOE_OK, MOE_ERR_DEVICE_TIMEOUT or MOE_ERR_DEVICE_BAD_INDEX). */

@@ -89,6 +89,7 @@ def lib():
         L.orc_forward.argtypes = [ctypes.POINTER(_Layer), vp, ctypes.POINTER(_Out)]
         L.orc_forward.restype = i32
         L.orc_num_threads.restype = i32
+        L.orc_allreduce_rmsnorm.argtypes = [vp, i32, i32, i32, vp, vp, ctypes.c_double, vp, vp]
         _lib = L
     return _lib
 
@@ -320,3 +321,18 @@ def forward(L: Layer, x: np.ndarray) -> dict:
     if rc != 0:
         raise MemoryError("oracle forward could not allocate its buffers")
     return r
+
+
+def allreduce_rmsnorm(x: np.ndarray, residual: Optional[np.ndarray], gamma: np.ndarray,
+                      eps: float):
+    """x: bf16 bits [G, T, d]; residual: bf16 bits [T, d] or None; gamma: bf16
+    bits [d] -> (res, out), both float64 [T, d]: the summed residual stream and
+    its RMSNorm times gamma."""
+    x = _c(x, np.uint16)
+    G, T, d = x.shape
+    r = None if residual is None else _c(residual, np.uint16)
+    g = _c(gamma, np.uint16)
+    res = np.empty((T, d), np.float64)
+    out = np.empty((T, d), np.float64)
+    lib().orc_allreduce_rmsnorm(_p(x), G, T, d, _p(r), _p(g), float(eps), _p(res), _p(out))
+    return res, out

@@ -519,3 +519,24 @@ int orc_forward(const orc_layer* L, const uint16_t* x, orc_out* out) {
     free(counts); free(offsets); free(perm); free(inv); free(h); free(o);
     return 0;
 }
+
+/* ---------------------------------------------------------------------------
+ * Fused all-reduce + residual + RMSNorm (tensor parallelism)
+ * ------------------------------------------------------------------------- */
+
+void orc_allreduce_rmsnorm(const uint16_t* x, int G, int T, int d, const uint16_t* residual,
+                           const uint16_t* gamma, double eps, double* res, double* out) {
+    #pragma omp parallel for schedule(static)
+    for (int t = 0; t < T; ++t) {
+        double ss = 0.0;
+        for (int i = 0; i < d; ++i) {
+            double s = residual ? orc_bf16_decode(residual[(int64_t)t * d + i]) : 0.0;
+            for (int r = 0; r < G; ++r) s += orc_bf16_decode(x[((int64_t)r * T + t) * d + i]);
+            res[(int64_t)t * d + i] = s;
+            ss += s * s;
+        }
+        const double inv = 1.0 / sqrt(ss / d + eps);
+        for (int i = 0; i < d; ++i)
+            out[(int64_t)t * d + i] = res[(int64_t)t * d + i] * inv * orc_bf16_decode(gamma[i]);
+    }
+}

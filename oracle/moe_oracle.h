@@ -162,6 +162,17 @@ int orc_forward(const orc_layer* L, const uint16_t* x, orc_out* out);
 
 int orc_num_threads(void);
 
+/* [AN] "HPC-Ops - 騰訊混元開源的工業級高性能大模型推理算子庫", section
+ * HPC-Ops的技術原理, "Fused AllReduce+Norm": the tensor-parallel all-reduce of the
+ * G ranks' partial outputs fused with the residual add and RMSNorm,
+ * out = RMSNorm(AllReduce(x) + residual, weight).  In FP64, per token t:
+ *   s[t][i]   = sum_{r < G} x[r][t][i] + residual[t][i]   (residual may be NULL)
+ *   res[t][i] = s[t][i]                 (the new residual stream)
+ *   out[t][i] = s[t][i] / sqrt(mean_i s[t][i]^2 + eps) * gamma[i]
+ * x bf16 [G][T][d], residual bf16 [T][d], gamma bf16 [d]. */
+void orc_allreduce_rmsnorm(const uint16_t* x, int G, int T, int d, const uint16_t* residual,
+                           const uint16_t* gamma, double eps, double* res, double* out);
+
 #ifdef __cplusplus
 }
 #endif

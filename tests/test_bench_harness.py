@@ -100,9 +100,13 @@ def test_gateup_kernel_follows_the_library_dispatch():
 def test_launch_count_follows_the_library_dispatch():
     from expert_layer_dual_b200.configs import CONFIGS
     n = {k: bench.kernels_per_step(c, c.T) for k, c in CONFIGS.items()}
-    # router, top-k, the one-block permute (<= 1024 assignments), gate-up, down, combine
-    assert n["decode"] == n["tiny"] == 6
+    # decode splits the router's K: router, top-k, the one-block permute (<= 1024
+    # assignments), gate-up, down, combine
+    assert n["decode"] == 6
+    assert bench.router_ksplit(64, 4096, 256) == 8 and bench.router_ksplit(8192, 4096, 256) == 1
+    # one CTA per router tile: the top-k runs inside the router kernel
+    assert n["tiny"] == 5
     # the permute in three kernels (count, scan, scatter)
-    assert n["prefill"] == n["skew"] == 8
+    assert n["prefill"] == n["skew"] == 7
     # + the activation quantiser
-    assert n["fp8"] == n["mxfp8"] == n["fp8t"] == 9
+    assert n["fp8"] == n["mxfp8"] == n["fp8t"] == 8

@@ -90,12 +90,58 @@ def test_quantize_act_fp8_static_permuted_bit_exact(cfg):
 
 
 @pytest.mark.parametrize("cfg", F8T, ids=IDS)
-def test_calibrated_scales_cover_the_calibration_tokens(cfg):
+@pytest.mark.parametrize("n_tokens", [64, 1, 77])
+def test_calibrate_fp8_static_bit_exact(cfg, n_tokens):
+    # moe_calibrate_fp8_static computes, on the GPU, the static scales of x and of the
+    # BF16 gate-up output h of the calibration tokens.  Both must equal the oracle's
+    # per-tensor quantiser rule s = fp32(amax) / 448 (FP32 division) applied to the same
+    # values: x itself, and the h the library's BF16 gate-up left in the workspace (whose
+    # own parity is checked against the oracle here, and by the gate-up stage tests).
     inp = make_layer(cfg)
     layer = M.MoELayer(cfg, inp)
-    sx, sh = layer.act_scales
-    amax_x = float(inp["x"][: layer.CALIBRATION_TOKENS].float().abs().max())
-    assert sx == pytest.approx(amax_x / 448.0, rel=1e-6) and sh > 0
+    n = min(n_tokens, cfg.T)
+    x = inp["x"][:n].contiguous()
+    bf = {k: inp[k].to(DEV) if inp.get(k) is not None else None for k in ("w_gu", "w_d", "ws_gu", "ws_d")}
+    p = M._p
+    w16 = M.moe_weights(p(bf["w_gu"]), p(bf["w_d"]), None, None, p(bf["ws_gu"]), p(bf["ws_d"]), None, None,
+                        p(layer.router_hi), p(layer.router_lo), p(layer.router_bias), 1.0, 1.0)
+    shape16 = M.moe_shape(n, cfg.d, cfg.E, cfg.k, cfg.I, cfg.Is, M.WDTYPE_BF16, int(cfg.renorm))
+    ws = torch.empty(M.workspace_bytes(shape16), dtype=torch.uint8, device=DEV)
+    scales = torch.empty(2, dtype=torch.float32, device=DEV)
+    M.calibrate_fp8_static(shape16, w16, _u16(x.to(DEV)), scales, ws)
+    st = M.workspace_view(ws, shape16)
+    h = st["h"].clone()
+    torch.cuda.synchronize()
+    assert M.read_device_status(ws) == M.OK
+    sx, sh = scales.cpu().numpy()
+    _, osx = oracle.quant_fp8_tensor(bits(x)[None])
+    _, osh = oracle.quant_fp8_tensor(bits(h)[None])
+    assert sx.tobytes() == osx[0].tobytes() and sh.tobytes() == osh[0].tobytes()
+    # the h the scale was taken over is the layer's gate-up output of these tokens
+    ids = st["ids"].cpu().numpy()
+    _, ooff, operm, _ = oracle.permute(ids, cfg.E)
+    L = oracle_layer(MoEConfig(**{**cfg.__dict__, "wdtype": 0}), inp, T=n)
+    ref = oracle.gateup(L, bits(x), operm, ooff)[:, : cfg.I]
+    assert_close_rel(bf16_to_f64(h), ref, rtol=2.0 ** -8, atol=1e-3 * rms(ref), what="h")
+    # the layer object calibrates with the same entry point on its first 64 tokens
+    if n == min(layer.CALIBRATION_TOKENS, cfg.T):
+        assert layer.act_scales == (float(sx), float(sh))
+
+
+def test_calibrate_fp8_static_rejects_bad_arguments():
+    cfg = F8T[0]
+    inp = make_layer(cfg)
+    layer = M.MoELayer(cfg, inp)
+    scales = torch.empty(2, dtype=torch.float32, device=DEV)
+    x = inp["x"][:8].to(DEV)
+    ws = torch.empty(1 << 20, dtype=torch.uint8, device=DEV)
+    with pytest.raises(M.MoEError) as e:              # the weights must be the BF16 originals
+        M.calibrate_fp8_static(layer.shape(8), layer.weights, _u16(x), scales, ws)
+    assert e.value.code == M.UNSUPPORTED
+    shape0 = M.moe_shape(0, cfg.d, cfg.E, cfg.k, cfg.I, cfg.Is, M.WDTYPE_BF16, 1)
+    with pytest.raises(M.MoEError) as e:              # nothing to calibrate on
+        M.calibrate_fp8_static(shape0, layer.weights, _u16(x), scales, ws)
+    assert e.value.code == M.INVALID_ARG
 
 
 @pytest.mark.parametrize("cfg", F8T, ids=IDS)

@@ -1,13 +1,26 @@
 """GPU parity of the whole layer (moe_forward through the C ABI) against the
-oracle: small configs in full, and the full-size workloads on sampled tokens
-plus properties that hold at any size.
+oracle: small configs over a sweep of seeds in full, and the full-size
+workloads on sampled tokens plus properties checked on every token.
 
-Bars: expert ids exact on every token whose top-(k+1) oracle logits are not
-within 1e-4 * rms of each other (elsewhere the FP32 kernel and the FP64
-oracle may both be right; the GPU choice is then checked for validity);
-BF16 outputs max |y - y_ref| <= 2e-2 * rms(y_ref); FP8 outputs <= 6e-2 *
-rms(y_ref) against the oracle run on its own quantisation of the same
-weights."""
+The routing contract is checked on the forward's own intermediates (read from
+its workspace at the offsets moe_workspace_offsets reports):
+  - the oracle's top-k run on the GPU's FP32 logits gives the GPU's expert ids
+    on EVERY token (bit-exact, ties to the lower id) and its weights within
+    2e-6; the oracle's permute of the GPU's ids gives the GPU's counts,
+    offsets, perm and inv bit-exact;
+  - independently, the GPU's logits are within 1e-5 relative of the oracle's
+    own FP64 logits, and the ids the oracle picks from those equal the GPU's
+    except on tokens whose top-(k+1) logits lie within 1e-4 * rms of each
+    other (both choices are then right within the logits bound; the GPU's is
+    checked for validity).
+The output is compared on every token (every sampled token at full size)
+with the oracle run on that routing:
+  - BF16: |y - y64| <= 2e-2 * rms(y64) + 2^-8 |y64| elementwise.  The second
+    term allows for the output's own bf16 rounding: even the correctly rounded
+    RNE_bf16(y64) misses 2e-2 * rms on some seeds, so the bound applies to the
+    computation before that rounding (the raw error is reported alongside);
+  - FP8 / MXFP8 / per-tensor FP8: max |y - y64| <= 6e-2 * rms(y64), the
+    oracle on its own quantisation of the same weights."""
 import numpy as np
 import pytest
 import torch
@@ -15,8 +28,9 @@ import torch
 import oracle
 from expert_layer_dual_b200.configs import CONFIGS, MoEConfig
 from expert_layer_dual_b200.inputs import make_layer
-from gpu_util import (ambiguous_tokens, assert_close_rel, bf16_to_f64, bits, logit_rel_error,
-                      oracle_layer, row_scale, rms)
+from gpu_util import (ambiguous_tokens, assert_close_rel, bf16_allowance, bf16_to_f64, bits,
+                      layer_errors, logit_rel_error, oracle_layer, oracle_routed,
+                      oracle_routed_sampled, pick_tokens, report, rms, row_scale)
 
 pytestmark = pytest.mark.gpu
 
@@ -36,12 +50,9 @@ SMALL = [
     MoEConfig("manyrows", T=600, d=384, E=8, k=4, I=256, Is=256, seed=28),
     # 241..282 rows per expert: tiles whose second 128-row half is empty, and 3 N tiles
     MoEConfig("manyedge", T=520, d=256, E=8, k=4, I=384, Is=0, seed=29),
-    # few router tiles, so the router splits K, with more than 512 tokens (a warp per token sums
-    # the partials); the smaller configs above take the block-per-token top-k.  (The BF16 y
-    # itself is within 2^-8 |y| of exact, which at |y| ~ 5 rms is already ~2e-2 rms: with
-    # seed 30 the exact chain of BF16 h, FP16 o and BF16 y, modelled on the CPU, lands at
-    # 0.0228 rms, so the bar is met by this seed's values, not by a looser computation.)
-    MoEConfig("splitk", T=640, d=512, E=32, k=4, I=256, Is=256, seed=31),
+    # few router tiles, so the router splits K, with more than 512 tokens (a warp per token
+    # sums the partials); the smaller configs above take the block-per-token top-k
+    MoEConfig("splitk", T=640, d=512, E=32, k=4, I=256, Is=256, seed=30),
     MoEConfig("fp8small", T=200, d=512, E=16, k=4, I=256, Is=256, wdtype=1, seed=31),
     MoEConfig("fp8odd", T=77, d=384, E=8, k=2, I=128, Is=0, wdtype=1, seed=32),
     MoEConfig("mxsmall", T=200, d=512, E=16, k=4, I=256, Is=256, wdtype=2, seed=33),
@@ -50,11 +61,14 @@ SMALL = [
     MoEConfig("f8todd", T=77, d=384, E=8, k=2, I=128, Is=0, wdtype=3, seed=36),
 ]
 BY_NAME = {c.name: c for c in SMALL}
+# every small config runs on its own seed and on each of these; none is left out
+SEEDS = list(range(100, 108))
+CASES = [(c, s) for c in SMALL for s in [c.seed] + SEEDS]
 
 
 def _stage_outputs(layer, cfg, x_dev):
     """Routing intermediates through the stage entry points (same kernels as
-    moe_forward): logits, ids, w, counts, offsets, perm, inv."""
+    moe_forward's non-split router): logits, ids, w, counts, offsets, perm, inv."""
     T, E, k = x_dev.shape[0], cfg.E, cfg.k
     logits = torch.empty((T, E), dtype=torch.float32, device=DEV)
     M.router_logits(x_dev.view(torch.uint16), layer.router_hi, layer.router_lo, layer.router_bias, logits)
@@ -70,62 +84,78 @@ def _stage_outputs(layer, cfg, x_dev):
     return dict(logits=logits, ids=ids, w=w, counts=counts, offsets=offsets, perm=perm, inv=inv)
 
 
-def _check_routing_validity(st, cfg, T):
-    ids = st["ids"].cpu().numpy()
-    w = st["w"].cpu().double().numpy()
-    counts = st["counts"].cpu().numpy()
-    offsets = st["offsets"].cpu().numpy()
-    perm = st["perm"].cpu().numpy()
-    inv = st["inv"].cpu().numpy()
-    k = cfg.k
-    assert counts.sum() == T * k and offsets[0] == 0 and offsets[-1] == T * k
-    assert np.array_equal(np.diff(offsets), counts)
-    assert np.array_equal(inv[perm], np.arange(T * k))
-    flat = ids.reshape(-1)
-    assert np.array_equal(np.bincount(flat, minlength=cfg.E), counts)
-    grp = np.repeat(np.arange(cfg.E), counts)
-    assert np.array_equal(flat[perm], grp)                      # rows grouped by expert
-    same = grp[1:] == grp[:-1]
-    assert np.all(np.diff(perm)[same] > 0)                       # token order inside a group
-    assert np.all((np.sort(ids, axis=1)[:, 1:] != np.sort(ids, axis=1)[:, :-1]))  # distinct
-    if cfg.renorm:
-        assert np.max(np.abs(w.sum(axis=1) - 1.0)) < 1e-5
-    assert np.all(np.diff(w, axis=1) <= 1e-7)                   # descending weights
+def forward_with_routing(layer, x):
+    """y of moe_forward and host copies of the routing it decided on (logits,
+    ids, w, counts, offsets, perm, inv from its workspace)."""
+    y = layer.forward(x)
+    st = M.workspace_view(layer.ws, layer.shape(x.shape[0]))
+    torch.cuda.synchronize()
+    out = {n: st[n].cpu().numpy() for n in ("logits", "ids", "w", "counts", "offsets", "perm", "inv")}
+    assert layer.device_status() == M.OK
+    return y, out
 
 
-def _compare_tokens(cfg, y_gpu, st, ref, tol):
-    """Compare GPU rows with oracle rows (`ref` from oracle.forward on the same tokens)."""
-    amb = ambiguous_tokens(ref["logits"], cfg.k)
-    gids = st["ids"]
-    ok = ~amb
-    assert np.array_equal(gids[ok], ref["ids"][ok]), "expert ids differ on unambiguous tokens"
-    # ambiguous tokens: every chosen expert's logit is within the tie band of the k-th best
-    scales = row_scale(ref["logits"])
+def check_routing_contract(cfg, st):
+    """The oracle's top-k on the GPU's logits and its permute of the GPU's ids
+    reproduce the GPU's routing exactly, on every token."""
+    oids, ow = oracle.route_topk(st["logits"].astype(np.float32), cfg.k, cfg.renorm)
+    bad = np.nonzero(np.any(oids != st["ids"], axis=1))[0]
+    assert bad.size == 0, f"expert ids differ from the oracle's top-k of the GPU logits on tokens {bad[:8]}"
+    assert np.max(np.abs(st["w"].astype(np.float64) - ow)) <= 2e-6
+    counts, offsets, perm, inv = oracle.permute(st["ids"], cfg.E)
+    for name, ref in (("counts", counts), ("offsets", offsets), ("perm", perm), ("inv", inv)):
+        assert np.array_equal(st[name], ref), f"{name} differs from the oracle's permute of the GPU ids"
+    return oids, ow
+
+
+def check_logits_independent(cfg, logits32, lg64, ids):
+    """The GPU's logits against the oracle's own FP64 logits of the same
+    tokens, and the oracle's own expert choice outside the tie band."""
+    assert logit_rel_error(logits32, lg64).max() <= 1e-5
+    oids, _ = oracle.route_topk(lg64.astype(np.float32), cfg.k, cfg.renorm)
+    amb = ambiguous_tokens(lg64, cfg.k)
+    assert np.array_equal(ids[~amb], oids[~amb]), "expert ids differ on unambiguous tokens"
+    scales = row_scale(lg64)
     for t in np.where(amb)[0]:
-        row = ref["logits"][t]
-        kth = -np.sort(-row)[cfg.k - 1]
-        assert np.all(row[gids[t]] >= kth - 2e-4 * scales[t, 0])
-    assert ok.sum() >= 0.9 * len(ok), f"{int(amb.sum())} of {len(ok)} tokens ambiguous"
-    err = np.abs(y_gpu[ok] - ref["y"][ok])
-    scale = rms(ref["y"])
-    assert err.max() <= tol * scale, f"max |dy| = {err.max() / scale:.3g} * rms(y)"
-    return err.max() / scale, int(amb.sum())
+        kth = -np.sort(-lg64[t])[cfg.k - 1]
+        assert np.all(lg64[t][ids[t]] >= kth - 2e-4 * scales[t, 0])
+    return int(amb.sum())
 
 
-@pytest.mark.parametrize("cfg", SMALL, ids=[c.name for c in SMALL])
-def test_forward_small(cfg):
+def check_output(cfg, y, y64, label):
+    errs = layer_errors(y, y64)
+    report({"case": label, "wdtype": cfg.wdtype, "tokens": int(y.shape[0]), **errs})
+    if cfg.wdtype == 0:
+        excess = np.abs(y - y64) - bf16_allowance(y64) - 2e-2 * errs["rms"]
+        assert excess.max() <= 0, (f"{label}: |y - y64| exceeds 2e-2 rms + 2^-8 |y64| "
+                                   f"(raw {errs['raw']:.4f}, comp {errs['comp']:.4f} rms)")
+    else:
+        assert errs["raw"] <= 6e-2, f"{label}: max |y - y64| = {errs['raw']:.4f} rms"
+    return errs
+
+
+@pytest.mark.parametrize("cfg,seed", CASES, ids=[f"{c.name}-s{s}" for c, s in CASES])
+def test_forward_small(cfg, seed):
+    cfg = cfg if seed == cfg.seed else MoEConfig(**{**cfg.__dict__, "seed": seed})
     inp = make_layer(cfg)
     layer = M.MoELayer(cfg, inp)
     x = inp["x"].to(DEV)
-    y = layer.forward(x)
-    assert layer.device_status() == M.OK
-    st = _stage_outputs(layer, cfg, x)
-    _check_routing_validity(st, cfg, cfg.T)
-    st_np = {k: v.cpu().numpy() for k, v in st.items()}
-    ref = oracle.forward(oracle_layer(cfg, inp, act=layer.act_scales), bits(inp["x"]))
-    rel, namb = _compare_tokens(cfg, bf16_to_f64(y), st_np, ref, 6e-2 if cfg.wdtype else 2e-2)
-    # the logits feeding the routing are FP32-accurate
-    assert logit_rel_error(st_np["logits"], ref["logits"]).max() <= 1e-5
+    y, st = forward_with_routing(layer, x)
+    oids, ow = check_routing_contract(cfg, st)
+    # the top-k fused into the forward's router kernel gives the same bits as the
+    # top-k stage entry point on the same logits
+    ids2 = torch.empty((cfg.T, cfg.k), dtype=torch.int32, device=DEV)
+    w2 = torch.empty((cfg.T, cfg.k), dtype=torch.float32, device=DEV)
+    M.route_topk(torch.from_numpy(st["logits"]).to(DEV), cfg.k, int(cfg.renorm), ids2, w2)
+    assert np.array_equal(ids2.cpu().numpy(), st["ids"])
+    assert w2.cpu().numpy().tobytes() == st["w"].tobytes()
+    L = oracle_layer(cfg, inp, act=layer.act_scales)
+    xb = bits(inp["x"])
+    hi, lo = oracle.router_split(inp["router_w"].numpy())
+    lg64 = oracle.router_logits(xb, hi, lo, None if inp["router_bias"] is None else inp["router_bias"].numpy())
+    check_logits_independent(cfg, st["logits"], lg64, st["ids"])
+    y64 = oracle_routed(L, xb, oids, ow)
+    check_output(cfg, bf16_to_f64(y), y64, f"{cfg.name}-s{seed}")
     # y computed twice is identical (no atomics anywhere on the path)
     y2 = layer.forward(x)
     assert torch.equal(y, y2)
@@ -239,46 +269,29 @@ def test_status_and_validation_paths():
 
 
 # ---------------------------------------------------------------- full size
-def _full_size_case(name, n_sample):
+def _full_size_case(name, n_sample=64):
     cfg = CONFIGS[name]
     inp = make_layer(cfg, device=DEV)
     layer = M.MoELayer(cfg, inp)
     x = inp["x"]
-    y = layer.forward(x)
-    assert layer.device_status() == M.OK
-    st = _stage_outputs(layer, cfg, x)
-    _check_routing_validity(st, cfg, cfg.T)
-    g = torch.Generator().manual_seed(99)
-    sample = torch.sort(torch.randperm(cfg.T, generator=g)[:n_sample]).values.numpy()
+    y, st = forward_with_routing(layer, x)
+    oids, ow = check_routing_contract(cfg, st)          # every token, and the whole permutation
+    sample = pick_tokens(st["offsets"], st["perm"], cfg.k, cfg.T, n_sample)
     xs = bits(x[torch.as_tensor(sample, device=DEV)])
-    # the oracle reads only the experts its own routing picks: copy those
     rw = inp["router_w"].cpu().numpy()
     hi, lo = oracle.router_split(rw)
     bias = None if inp["router_bias"] is None else inp["router_bias"].cpu().numpy()
-    lg = oracle.router_logits(xs, hi, lo, bias)
-    oids, _ = oracle.route_topk(lg.astype(np.float32), cfg.k)
-    need = np.unique(oids)
-    w_gu = np.empty((cfg.E, 2 * cfg.I, cfg.d), np.uint16)
-    w_d = np.empty((cfg.E, cfg.d, cfg.I), np.uint16)
-    for e in need:
-        w_gu[e] = bits(inp["w_gu"][int(e)])
-        w_d[e] = bits(inp["w_d"][int(e)])
-    L = oracle.Layer(T=len(sample), d=cfg.d, E=cfg.E, k=cfg.k, I=cfg.I, Is=cfg.Is, w_gu=w_gu, w_d=w_d,
-                     ws_gu=bits(inp["ws_gu"]), ws_d=bits(inp["ws_d"]), router_w=rw, router_bias=bias,
-                     wdtype=cfg.wdtype, renorm=cfg.renorm, act_sx=layer.act_scales[0],
-                     act_sh=layer.act_scales[1])
-    ref = oracle.forward(L, xs)
-    st_np = {k: v.cpu().numpy()[sample] for k, v in st.items() if k in ("logits", "ids", "w")}
-    tol = 6e-2 if cfg.wdtype else 2e-2
-    rel, namb = _compare_tokens(cfg, bf16_to_f64(y)[sample], st_np, ref, tol)
-    assert logit_rel_error(st_np["logits"], ref["logits"]).max() <= 1e-5
-    return cfg, st
+    lg64 = oracle.router_logits(xs, hi, lo, bias)
+    check_logits_independent(cfg, st["logits"][sample], lg64, st["ids"][sample])
+    y64 = oracle_routed_sampled(cfg, inp, xs, oids[sample], ow[sample], act=layer.act_scales)
+    check_output(cfg, bf16_to_f64(y)[sample], y64, f"{name}-full")
+    return cfg, st, sample
 
 
-@pytest.mark.parametrize("name,n", [("decode", 64), ("prefill", 12), ("fp8", 4), ("mxfp8", 4),
-                                    ("fp8t", 4)])
-def test_forward_full_size(name, n):
-    _full_size_case(name, n)
+@pytest.mark.parametrize("name", ["decode", "prefill", "fp8", "mxfp8", "fp8t"])
+def test_forward_full_size(name):
+    cfg, st, sample = _full_size_case(name)
+    assert len(sample) >= min(64, cfg.T)
 
 
 def test_gemm_gateup_full_size_wide_tiles_on_sampled_rows():
@@ -325,8 +338,9 @@ def test_gemm_gateup_full_size_wide_tiles_on_sampled_rows():
 
 
 def test_forward_full_size_skew():
-    cfg, st = _full_size_case("skew", 8)
-    counts = st["counts"].cpu().numpy()
+    cfg, st, sample = _full_size_case("skew")
+    assert len(sample) >= 64
+    counts = st["counts"]
     assert (counts == 0).sum() >= 8                          # the masked experts stay empty
     top = np.sort(counts)[::-1]
     assert top[: int(0.1 * cfg.E) + 1].sum() >= 0.4 * counts.sum()   # ~10% of experts take ~half
