@@ -284,11 +284,11 @@ def router_ksplit(T: int, d: int, E: int) -> int:
 
 def kernels_per_step(cfg: MoEConfig, T: int) -> int:
     """Kernels of this library one moe_forward launches, by its dispatch: the
-    router (with the top-k fused into it when one CTA covers a tile's whole K,
-    else followed by the top-k kernel), the permute (one kernel for at most
+    router (with the top-k fused into it when one CTA covers a tile's whole K
+    and E <= 64, else followed by the top-k kernel), the permute (one kernel for at most
     1024 assignments, else count, scan and scatter), gate-up, down and
     combine, plus the activation quantiser on the FP8 paths."""
-    router = 1 if router_ksplit(T, cfg.d, cfg.E) == 1 else 2
+    router = 1 if router_ksplit(T, cfg.d, cfg.E) == 1 and cfg.E <= 64 else 2
     permute = 1 if T * cfg.k <= 1024 else 3
     return router + permute + 3 + (1 if cfg.wdtype else 0)
 

@@ -93,7 +93,8 @@ WsLayout ws_layout(const moe_shape& s) {
     L.logits = take(T * E * 4);
     L.ksplit = router_ksplit(s.T, s.d, s.E);
     L.part = L.ksplit > 1 ? take(2 * (size_t)L.ksplit * T * E * 4) : 0;  // split-K router partials
-    L.rtk = L.ksplit == 1 ? take(router_topk_scratch_bytes(s.T, s.E)) : 0;  // fused top-k scratch
+    L.rtk = L.ksplit == 1 && router_fuses_topk(s.E) ? take(router_topk_scratch_bytes(s.T, s.E))
+                                                     : 0;  // fused top-k scratch
     L.ids = take(T * k * 4);
     L.w = take(T * k * 4);
     L.counts = take(E * 4);
@@ -283,7 +284,7 @@ moe_status route_device(const moe_shape* s, const moe_weights* w, const uint16_t
     int32_t* ids = at<int32_t>(ws, L.ids);
     float* rw = at<float>(ws, L.w);
     moe_status r;
-    if (L.ksplit == 1) {
+    if (L.ksplit == 1 && router_fuses_topk(s->E)) {
         // router logits with the top-k fused into the same kernel
         if ((r = cuda_status(launch_router_topk(x, w->router_hi, w->router_lo, w->router_bias,
                                                 logits, s->T, s->d, s->E, s->k, s->renormalize,
@@ -291,6 +292,14 @@ moe_status route_device(const moe_shape* s, const moe_weights* w, const uint16_t
             MOE_OK)
             return r;
         if (!record_event(events, 1, st)) return MOE_ERR_CUDA;
+    } else if (L.ksplit == 1) {
+        if ((r = cuda_status(launch_router_logits(x, w->router_hi, w->router_lo, w->router_bias,
+                                                  logits, s->T, s->d, s->E, status, st))) != MOE_OK)
+            return r;
+        if (!record_event(events, 1, st)) return MOE_ERR_CUDA;
+        if ((r = cuda_status(launch_route_topk(logits, s->T, s->E, s->k, s->renormalize, ids, rw,
+                                               st))) != MOE_OK)
+            return r;
     } else {
         // few tokens: K split across CTAs, partials combined inside the top-k kernel
         float* ph = at<float>(ws, L.part);

@@ -100,6 +100,11 @@ cudaError_t launch_router_logits(const uint16_t* x, const uint16_t* hi, const ui
 // bytes (16-byte aligned) of candidate keys and arrival counters, the
 // counters zeroed here before the launch.
 size_t router_topk_scratch_bytes(int T, int E);
+// Whether moe_forward fuses the top-k into a one-CTA-per-tile router: with one
+// 64-expert tile per token (E <= 64).  With more, the epilogue's per-row
+// selection and the cross-CTA merge cost more than the separate top-k kernel
+// (measured on the 256-expert workloads); there the top-k runs on its own.
+inline bool router_fuses_topk(int E) { return E <= 64; }
 cudaError_t launch_router_topk(const uint16_t* x, const uint16_t* hi, const uint16_t* lo,
                                const float* bias, float* logits, int T, int d, int E, int k,
                                int renorm, int32_t* ids, float* w, void* scratch, int32_t* status,

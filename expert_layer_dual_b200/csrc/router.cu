@@ -167,7 +167,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int m0 = blockIdx.x * BM, e0 = blockIdx.y * BN;
+    // grid x runs over the expert tiles, so the CTAs that share a 128-token x tile
+    // are launched together and read it from DRAM once
+    const int m0 = blockIdx.y * BM, e0 = blockIdx.x * BN;
     const int ksplit = gridDim.z, ks = blockIdx.z;
     const int nk_all = d / BK;
     const int kb0 = ks * nk_all / ksplit;                // this CTA's k-blocks: kb0 .. kb0+nk-1
@@ -307,7 +309,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
             if (fuse && t < T) {
                 ulonglong2* dst = reinterpret_cast<ulonglong2*>(
-                    tk.cand + ((int64_t)t * gridDim.y + blockIdx.y) * CAND);
+                    tk.cand + ((int64_t)t * gridDim.x + blockIdx.x) * CAND);
 #pragma unroll
                 for (int j = 0; j < CAND / 2; ++j) dst[j] = make_ulonglong2(best[2 * j], best[2 * j + 1]);
             }
@@ -323,10 +325,10 @@ __global__ void __launch_bounds__(THREADS, 1)
 
     // ---------------- fused top-k: the last CTA of each tile row routes its 128 tokens
     __shared__ int s_last;
-    const int ntiles = gridDim.y;
+    const int ntiles = gridDim.x;
     __threadfence();
     __syncthreads();
-    if (threadIdx.x == 0) s_last = atomicAdd(&tk.arrive_m[blockIdx.x], 1) == ntiles - 1;
+    if (threadIdx.x == 0) s_last = atomicAdd(&tk.arrive_m[blockIdx.y], 1) == ntiles - 1;
     __syncthreads();
     if (!s_last) return;
     __threadfence();
@@ -352,9 +354,9 @@ static cudaError_t launch_router_impl(const uint16_t* x, const uint16_t* hi, con
         if (e != cudaSuccess) return e;
         attr_set[dev] = true;
     }
-    dim3 grid((T + BM - 1) / BM, (E + BN - 1) / BN, ksplit);
+    dim3 grid((E + BN - 1) / BN, (T + BM - 1) / BM, ksplit);
     if (tk.ids != nullptr) {
-        cudaError_t e = cudaMemsetAsync(tk.arrive_m, 0, sizeof(int32_t) * grid.x, s);
+        cudaError_t e = cudaMemsetAsync(tk.arrive_m, 0, sizeof(int32_t) * grid.y, s);
         if (e != cudaSuccess) return e;
     }
     {
