@@ -116,6 +116,7 @@ class ClockSampler:
         self.path = None
         self.thread = None
         self.stop = False
+        self.power_limit_w = None
 
     def _nvml_loop(self, nv, h):
         names = [("hw_slowdown", nv.nvmlClocksEventReasonHwSlowdown),
@@ -123,6 +124,10 @@ class ClockSampler:
                  ("sw_thermal_slowdown", nv.nvmlClocksEventReasonSwThermalSlowdown),
                  ("sw_power_cap", nv.nvmlClocksEventReasonSwPowerCap)]
         smax = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        try:
+            self.power_limit_w = nv.nvmlDeviceGetEnforcedPowerLimit(h) / 1000.0
+        except nv.NVMLError:
+            pass
         while not self.stop:
             try:
                 sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
@@ -173,6 +178,8 @@ class ClockSampler:
         if self.thread is not None:
             out = parse_clock_samples(self.lines)
             out["source"] = f"NVML every {self.period * 1e3:.0f} ms"
+            if self.power_limit_w is not None:
+                out["power_limit_w"] = self.power_limit_w
             return out
         if self.proc is None or not self.path or not os.path.exists(self.path):
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
