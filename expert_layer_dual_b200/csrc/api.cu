@@ -346,25 +346,25 @@ moe_status forward_device(const moe_shape* s, const moe_weights* w, const uint16
     const void* a_in = x;
     const void* a_scale = nullptr;
     if (f8t) {
-        const int64_t R = (int64_t)s->T * s->k + (s->I_shared > 0 ? s->T : 0);
-        if ((r = cuda_status(launch_quant_act_fp8_static(x, perm, s->T, s->k, R, s->d,
-                                                         w->act_scale_x, at<uint8_t>(ws, L.xq),
-                                                         st))) != MOE_OK)
+        if ((r = cuda_status(launch_quant_act_fp8_static_scatter(
+                 x, inv, s->T, s->k, s->I_shared > 0 ? 1 : 0, s->d, w->act_scale_x,
+                 at<uint8_t>(ws, L.xq), st))) != MOE_OK)
             return r;
         a_in = at<uint8_t>(ws, L.xq);
     }
     if (mx) {
-        if ((r = cuda_status(launch_quant_mx_permuted(x, perm, s->T, s->k, s->I_shared > 0 ? 1 : 0,
-                                                      s->d, at<uint8_t>(ws, L.xq),
-                                                      at<uint8_t>(ws, L.xs), st))) != MOE_OK)
+        if ((r = cuda_status(launch_quant_mx_scatter(x, inv, s->T, s->k, s->I_shared > 0 ? 1 : 0,
+                                                     s->d, at<uint8_t>(ws, L.xq),
+                                                     at<uint8_t>(ws, L.xs), st))) != MOE_OK)
             return r;
         a_in = at<uint8_t>(ws, L.xq);
         a_scale = at<uint8_t>(ws, L.xs);
     }
     if (fp8) {
-        if ((r = cuda_status(launch_quant_act_fp8_permuted(x, perm, s->T, s->k, s->I_shared > 0 ? 1 : 0,
-                                                           s->d, at<uint8_t>(ws, L.xq),
-                                                           at<float>(ws, L.xs), st))) != MOE_OK)
+        if ((r = cuda_status(launch_quant_act_fp8_scatter(x, inv, s->T, s->k,
+                                                          s->I_shared > 0 ? 1 : 0, s->d,
+                                                          at<uint8_t>(ws, L.xq),
+                                                          at<float>(ws, L.xs), st))) != MOE_OK)
             return r;
         a_in = at<uint8_t>(ws, L.xq);
         a_scale = at<float>(ws, L.xs);
@@ -691,6 +691,8 @@ moe_status moe_workspace_offsets(const moe_shape* shape, moe_workspace_map* map)
     map->offsets = L.offsets;
     map->perm = L.perm;
     map->inv = L.inv;
+    map->xq = L.xq;
+    map->xs = L.xs;
     map->h = L.h;
     map->total = L.total;
     return MOE_OK;

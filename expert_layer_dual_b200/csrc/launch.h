@@ -63,6 +63,11 @@ cudaError_t launch_quant_act_fp8(const uint16_t* x, int64_t rows, int cols, uint
 cudaError_t launch_quant_act_fp8_permuted(const uint16_t* x, const int32_t* perm, int T, int k,
                                           int has_shared, int cols, uint8_t* q, float* scale,
                                           cudaStream_t s);
+// The same outputs token-major: each token's row quantised once and stored to
+// its rows inv[t*k + j] (and T*k + t with the shared expert).
+cudaError_t launch_quant_act_fp8_scatter(const uint16_t* x, const int32_t* inv, int T, int k,
+                                         int has_shared, int cols, uint8_t* q, float* scale,
+                                         cudaStream_t s);
 cudaError_t launch_quant_weights_fp8(const uint16_t* W, int64_t batch, int rows, int cols,
                                      uint8_t* q, float* scale, cudaStream_t s);
 // MXFP8 (e4m3 + E8M0 scale per 1x32 along the row): rows as they are, or in
@@ -76,6 +81,9 @@ cudaError_t launch_quant_mx_weights(const uint16_t* W, int64_t batch, int rows, 
 cudaError_t launch_quant_mx_permuted(const uint16_t* x, const int32_t* perm, int T, int k,
                                      int has_shared, int cols, uint8_t* q, uint8_t* scale,
                                      cudaStream_t s);
+cudaError_t launch_quant_mx_scatter(const uint16_t* x, const int32_t* inv, int T, int k,
+                                    int has_shared, int cols, uint8_t* q, uint8_t* scale,
+                                    cudaStream_t s);
 // Per-tensor FP8: weights with one scale per matrix (scale [batch]);
 // activations with a static scale, rows as they are (perm NULL) or in the
 // permuted order of the grouped GEMMs (rows = T*k + shared T).
@@ -84,6 +92,9 @@ cudaError_t launch_quant_weights_fp8_tensor(const uint16_t* W, int64_t batch, in
 cudaError_t launch_quant_act_fp8_static(const uint16_t* x, const int32_t* perm, int T, int k,
                                         int64_t rows, int cols, float scale, uint8_t* q,
                                         cudaStream_t s);
+cudaError_t launch_quant_act_fp8_static_scatter(const uint16_t* x, const int32_t* inv, int T,
+                                                int k, int has_shared, int cols, float scale,
+                                                uint8_t* q, cudaStream_t s);
 // Static FP8 scale of n bf16 values (n % 8 == 0, v 16-byte aligned): *scale =
 // fp32(max |v|) / 448 (1 when every value is zero).
 cudaError_t launch_amax_scale(const uint16_t* v, int64_t n, float* scale, cudaStream_t s);

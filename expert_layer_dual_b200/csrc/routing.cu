@@ -524,6 +524,40 @@ __device__ __forceinline__ float group_scale(float amax) {
     return amax == 0.0f ? 1.0f : __fdiv_rn(amax, 448.0f);
 }
 
+// The permuted rows that hold token t in the grouped GEMMs' row order: row
+// inv[t*k + j] for each of its k assignments (j < k <= 8), and row T*k + t for
+// the shared expert.  Every lane of the warp gets all of them (rows[j], j < k;
+// rows[8] the shared row).  Used by the token-major quantisers below: a
+// token's row is quantised once and its codes stored to each of these rows,
+// instead of quantising each permuted row on its own.
+struct TokenRows {
+    int64_t row[9];
+    int k;
+    bool shared;
+};
+
+__device__ __forceinline__ TokenRows token_rows(const int32_t* __restrict__ inv, int64_t t, int T,
+                                                int k, int has_shared) {
+    const int lane = threadIdx.x & 31;
+    const int32_t mine = lane < k ? inv[t * k + lane] : 0;
+    TokenRows r;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) r.row[j] = __shfl_sync(0xffffffffu, mine, j);
+    r.row[8] = (int64_t)T * k + t;
+    r.k = k;
+    r.shared = has_shared != 0;
+    return r;
+}
+
+// f(row) for every row of the token, with indices known at compile time.
+template <typename F>
+__device__ __forceinline__ void for_token_rows(const TokenRows& r, F f) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+        if (j < r.k) f(r.row[j]);
+    if (r.shared) f(r.row[8]);
+}
+
 // One warp quantises one row: each step covers two 128-column groups, lanes
 // 0-15 the first and 16-31 the second, 8 values (16 bytes) per lane; the
 // group amax is a 16-lane shuffle reduction.
@@ -588,6 +622,61 @@ cudaError_t launch_quant_act_fp8_permuted(const uint16_t* x, const int32_t* perm
     {
         const cudaError_t le = launch_pdl(k_quant_act_permuted, dim3((unsigned)((rows + 7) / 8)),
                                           dim3(256), 0, s, x, perm, T, k, rows, cols, q, scale);
+        if (le != cudaSuccess) return le;
+    }
+    return cudaGetLastError();
+}
+
+// The same codes and scales as k_quant_act_permuted, token-major: one warp per
+// token quantises its row once (the same quant_row arithmetic, so the same
+// bits) and stores the codes and scales to each of its k (+1) permuted rows.
+// The permuted kernel repeats the row's divisions for every copy; here each
+// value is divided once and only the stores are repeated.
+__global__ void __launch_bounds__(256)
+    k_quant_act_scatter(const uint16_t* __restrict__ x, const int32_t* __restrict__ inv, int T,
+                        int k, int has_shared, int cols, uint8_t* __restrict__ q,
+                        float* __restrict__ scale) {
+    pdl_wait();  // inputs come from the previous kernel of the forward
+    pdl_trigger();
+    const int64_t t = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+    if (t >= T) return;
+    const TokenRows tr = token_rows(inv, t, T, k, has_shared);
+    const uint16_t* src = x + t * cols;
+    const int lane = threadIdx.x & 31;
+    const int groups = cols / 128;
+    const int half = lane >> 4, l16 = lane & 15;
+    for (int g0 = 0; g0 < groups; g0 += 2) {
+        const int g = g0 + half;
+        const bool active = g < groups;
+        uint4 u = make_uint4(0, 0, 0, 0);
+        if (active) u = *reinterpret_cast<const uint4*>(src + g * 128 + l16 * 8);
+        float f[8];
+        bf16x8_to_f32(u, f);
+        float amax = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        const float sc = group_scale(amax);
+        if (active) {
+            uint2 c;
+            c.x = quant4_e4m3(f[0], f[1], f[2], f[3], sc);
+            c.y = quant4_e4m3(f[4], f[5], f[6], f[7], sc);
+            for_token_rows(tr, [&](int64_t p) {
+                *reinterpret_cast<uint2*>(q + p * cols + g * 128 + l16 * 8) = c;
+                if (l16 == 0) scale[p * groups + g] = sc;
+            });
+        }
+    }
+}
+
+cudaError_t launch_quant_act_fp8_scatter(const uint16_t* x, const int32_t* inv, int T, int k,
+                                         int has_shared, int cols, uint8_t* q, float* scale,
+                                         cudaStream_t s) {
+    if (T == 0) return cudaSuccess;
+    {
+        const cudaError_t le = launch_pdl(k_quant_act_scatter, dim3((unsigned)((T + 7) / 8)),
+                                          dim3(256), 0, s, x, inv, T, k, has_shared, cols, q, scale);
         if (le != cudaSuccess) return le;
     }
     return cudaGetLastError();
@@ -678,6 +767,62 @@ __global__ void __launch_bounds__(256)
     const int64_t Tk = (int64_t)T * k;
     const int64_t tok = p < Tk ? (int64_t)(perm[p] / k) : p - Tk;
     mx_row(x + tok * cols, cols, q + p * cols, scale, MxScaleLayout{rows, cols, false}, p);
+}
+
+// The same codes and scale bytes as k_quant_mx_permuted, token-major (one warp
+// per token, its row quantised once by mx_row's arithmetic, the results stored
+// to each of its k (+1) permuted rows).  rows = T*k (+T): the scale layout's
+// row count.
+__global__ void __launch_bounds__(256)
+    k_quant_mx_scatter(const uint16_t* __restrict__ x, const int32_t* __restrict__ inv, int T,
+                       int k, int has_shared, int64_t rows, int cols, uint8_t* __restrict__ q,
+                       uint8_t* __restrict__ scale) {
+    pdl_wait();  // inputs come from the previous kernel of the forward
+    pdl_trigger();
+    const int64_t t = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+    if (t >= T) return;
+    const TokenRows tr = token_rows(inv, t, T, k, has_shared);
+    const MxScaleLayout lay{rows, cols, false};
+    const uint16_t* src = x + t * cols;
+    const int lane = threadIdx.x & 31;
+    for (int c0 = 0; c0 < cols; c0 += 256) {
+        const int c = c0 + lane * 8;
+        const bool active = c < cols;
+        uint4 u = make_uint4(0, 0, 0, 0);
+        if (active) u = *reinterpret_cast<const uint4*>(src + c);
+        float f[8];
+        bf16x8_to_f32(u, f);
+        float amax = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+        const uint32_t b = mx_scale_byte(amax);
+        const float inv2 = __uint_as_float((254u - b) << 23);  // 2^(127 - b), b <= 253 here
+        if (active) {
+            uint2 cq;
+            cq.x = mx_quant4(f, inv2);
+            cq.y = mx_quant4(f + 4, inv2);
+            for_token_rows(tr, [&](int64_t p) {
+                *reinterpret_cast<uint2*>(q + p * cols + c) = cq;
+                if ((lane & 3) == 0) scale[lay.at(p, c / 32)] = static_cast<uint8_t>(b);
+            });
+        }
+    }
+}
+
+cudaError_t launch_quant_mx_scatter(const uint16_t* x, const int32_t* inv, int T, int k,
+                                    int has_shared, int cols, uint8_t* q, uint8_t* scale,
+                                    cudaStream_t s) {
+    const int64_t rows = (int64_t)T * k + (has_shared ? T : 0);
+    if (T == 0) return cudaSuccess;
+    {
+        const cudaError_t le = launch_pdl(k_quant_mx_scatter, dim3((unsigned)((T + 7) / 8)),
+                                          dim3(256), 0, s, x, inv, T, k, has_shared, rows, cols, q,
+                                          scale);
+        if (le != cudaSuccess) return le;
+    }
+    return cudaGetLastError();
 }
 
 cudaError_t launch_quant_mx_rows(const uint16_t* x, int64_t rows, int cols, uint8_t* q,
@@ -838,6 +983,43 @@ __global__ void __launch_bounds__(256)
         o.y = quant4_e4m3_fixed(f[4], f[5], f[6], f[7], s, r, s_in_range);
         *reinterpret_cast<uint2*>(dst + c) = o;
     }
+}
+
+// The same codes as k_quant_static over permuted rows, token-major: one warp
+// per token divides its row once and stores the codes to each of its k (+1)
+// permuted rows.
+__global__ void __launch_bounds__(256)
+    k_quant_static_scatter(const uint16_t* __restrict__ x, const int32_t* __restrict__ inv, int T,
+                           int k, int has_shared, int cols, float s, uint8_t* __restrict__ q) {
+    pdl_wait();  // inputs come from the previous kernel of the forward
+    pdl_trigger();
+    const int64_t t = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+    if (t >= T) return;
+    const TokenRows tr = token_rows(inv, t, T, k, has_shared);
+    const int lane = threadIdx.x & 31;
+    const uint16_t* src = x + t * cols;
+    const float r = __frcp_rn(s);
+    const bool s_in_range = s >= 0x1p-26f && s <= 0x1p26f;
+    for (int c = lane * 8; c < cols; c += 256) {
+        float f[8];
+        bf16x8_to_f32(*reinterpret_cast<const uint4*>(src + c), f);
+        uint2 o;
+        o.x = quant4_e4m3_fixed(f[0], f[1], f[2], f[3], s, r, s_in_range);
+        o.y = quant4_e4m3_fixed(f[4], f[5], f[6], f[7], s, r, s_in_range);
+        for_token_rows(tr, [&](int64_t p) { *reinterpret_cast<uint2*>(q + p * cols + c) = o; });
+    }
+}
+
+cudaError_t launch_quant_act_fp8_static_scatter(const uint16_t* x, const int32_t* inv, int T,
+                                                int k, int has_shared, int cols, float scale,
+                                                uint8_t* q, cudaStream_t s) {
+    if (T == 0) return cudaSuccess;
+    {
+        const cudaError_t le = launch_pdl(k_quant_static_scatter, dim3((unsigned)((T + 7) / 8)),
+                                          dim3(256), 0, s, x, inv, T, k, has_shared, cols, scale, q);
+        if (le != cudaSuccess) return le;
+    }
+    return cudaGetLastError();
 }
 
 cudaError_t launch_quant_act_fp8_static(const uint16_t* x, const int32_t* perm, int T, int k,

@@ -61,7 +61,7 @@ class moe_weights(ctypes.Structure):
 
 class moe_workspace_map(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in
-                ("logits", "ids", "w", "counts", "offsets", "perm", "inv", "h", "total")]
+                ("logits", "ids", "w", "counts", "offsets", "perm", "inv", "xq", "xs", "h", "total")]
 
 
 _vp, _i32, _i64, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
@@ -163,8 +163,9 @@ def workspace_offsets(shape: moe_shape) -> moe_workspace_map:
 
 
 def workspace_view(ws: torch.Tensor, shape: moe_shape) -> dict:
-    """Views (no copies) of the routing intermediates and h that moe_forward
-    leaves in `ws`, at the offsets moe_workspace_offsets reports."""
+    """Views (no copies) of the routing intermediates, the quantised
+    activations (FP8 formats) and h (BF16) that moe_forward leaves in `ws`,
+    at the offsets moe_workspace_offsets reports."""
     m = workspace_offsets(shape)
     T, E, k = shape.T, shape.E, shape.k
     R = T * k + (T if shape.I_shared else 0)
@@ -182,6 +183,13 @@ def workspace_view(ws: torch.Tensor, shape: moe_shape) -> dict:
            "inv": region(m.inv, T * k, torch.int32)}
     if shape.wdtype == WDTYPE_BF16:
         out["h"] = region(m.h, R * shape.I, torch.bfloat16).view(R, shape.I)
+    else:
+        d = shape.d
+        out["xq"] = region(m.xq, R * d, torch.uint8).view(R, d)
+        if shape.wdtype == WDTYPE_FP8_BLOCK128:
+            out["xs"] = region(m.xs, R * (d // 128), torch.float32).view(R, d // 128)
+        elif shape.wdtype == WDTYPE_MXFP8:
+            out["xs"] = region(m.xs, R * (d // 32), torch.uint8)
     return out
 
 

@@ -130,12 +130,18 @@ size_t moe_workspace_bytes(const moe_shape* shape);
  *   ids int32 [T][k], w float [T][k]           moe_route_topk's outputs
  *   counts int32 [E], offsets int32 [E+1], perm, inv int32 [T*k]
  *                                              moe_permute's outputs
+ *   xq, xs  the quantised activations the gate-up read (FP8 formats), in the
+ *           permuted row order: the outputs moe_quantize_act_fp8_permuted,
+ *           moe_quantize_act_mxfp8_permuted or moe_quantize_act_fp8_static_permuted
+ *           give for this routing's perm (xs: FP32 [R][d/128] for wdtype 1,
+ *           the E8M0 bytes for wdtype 2, absent for wdtype 3); 0 where the
+ *           format has no such region (wdtype 0; xs of wdtype 3)
  *   h   the gate-up output (wdtype 0: bf16 [R][I], R = T*k + (I_shared ? T : 0))
  *   total  = moe_workspace_bytes(shape).
  * Inspection and testing aid; returns MOE_ERR_INVALID_ARG / UNSUPPORTED as
  * moe_workspace_bytes would return 0. */
 typedef struct moe_workspace_map {
-    size_t logits, ids, w, counts, offsets, perm, inv, h, total;
+    size_t logits, ids, w, counts, offsets, perm, inv, xq, xs, h, total;
 } moe_workspace_map;
 moe_status moe_workspace_offsets(const moe_shape* shape, moe_workspace_map* map);
 

@@ -63,3 +63,23 @@ def test_validation_happens_before_any_launch(lib):
     assert lib.moe_forward(ctypes.byref(zero), ctypes.byref(w2), None, None, None, 0, None) == M.OK
     assert lib.moe_route_topk(None, 4, 300, 2, 1, None, None, None) == M.UNSUPPORTED
     assert lib.moe_router_split(None, None, None, ctypes.c_int64(-1), None) == M.INVALID_ARG
+
+
+def test_workspace_map_regions(lib):
+    # moe_workspace_offsets is host-only: the regions are 256-byte aligned, inside the
+    # workspace, and the quantised-activation regions exist exactly for the formats
+    # that have them (xq for the FP8 formats; xs for block-scaled FP8 and MXFP8)
+    from expert_layer_dual_b200 import moe as M
+    for wd in (0, 1, 2, 3):
+        s = M.moe_shape(200, 512, 16, 4, 256, 256, wd, 1)
+        m = M.workspace_offsets(s)
+        assert m.total == M.workspace_bytes(s)
+        regs = {n: getattr(m, n) for n in ("logits", "ids", "w", "counts", "offsets", "perm", "inv",
+                                           "xq", "xs", "h")}
+        for n, off in regs.items():
+            assert off % 256 == 0 and off < m.total, (wd, n)
+        R = 200 * 4 + 200
+        assert (regs["xq"] > 0) == (wd != 0)
+        assert (regs["xs"] > 0) == (wd in (1, 2))
+        if wd:
+            assert regs["xq"] + R * 512 <= m.total
