@@ -549,6 +549,20 @@ __device__ __forceinline__ TokenRows token_rows(const int32_t* __restrict__ inv,
     return r;
 }
 
+// The token-major quantisers give each warp one chunk of kScatterCols columns
+// of one token (more warps in flight than one per token; the chunk is a whole
+// number of every format's 256-column step).
+constexpr int kScatterCols = 1024;
+
+__device__ __forceinline__ int scatter_chunks(int cols) {
+    return (cols + kScatterCols - 1) / kScatterCols;
+}
+
+inline unsigned scatter_blocks(int T, int cols) {
+    const int64_t warps = (int64_t)T * ((cols + kScatterCols - 1) / kScatterCols);
+    return (unsigned)((warps + 7) / 8);
+}
+
 // f(row) for every row of the token, with indices known at compile time.
 template <typename F>
 __device__ __forceinline__ void for_token_rows(const TokenRows& r, F f) {
@@ -638,16 +652,20 @@ __global__ void __launch_bounds__(256)
                         float* __restrict__ scale) {
     pdl_wait();  // inputs come from the previous kernel of the forward
     pdl_trigger();
-    const int64_t t = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+    const int64_t wid = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+    const int nch = scatter_chunks(cols);
+    const int64_t t = wid / nch;
     if (t >= T) return;
+    const int ch = (int)(wid - t * nch);
     const TokenRows tr = token_rows(inv, t, T, k, has_shared);
     const uint16_t* src = x + t * cols;
     const int lane = threadIdx.x & 31;
     const int groups = cols / 128;
     const int half = lane >> 4, l16 = lane & 15;
-    for (int g0 = 0; g0 < groups; g0 += 2) {
+    const int g_end = min(groups, (ch + 1) * (kScatterCols / 128));
+    for (int g0 = ch * (kScatterCols / 128); g0 < g_end; g0 += 2) {
         const int g = g0 + half;
-        const bool active = g < groups;
+        const bool active = g < g_end;
         uint4 u = make_uint4(0, 0, 0, 0);
         if (active) u = *reinterpret_cast<const uint4*>(src + g * 128 + l16 * 8);
         float f[8];
@@ -675,7 +693,7 @@ cudaError_t launch_quant_act_fp8_scatter(const uint16_t* x, const int32_t* inv, 
                                          cudaStream_t s) {
     if (T == 0) return cudaSuccess;
     {
-        const cudaError_t le = launch_pdl(k_quant_act_scatter, dim3((unsigned)((T + 7) / 8)),
+        const cudaError_t le = launch_pdl(k_quant_act_scatter, dim3(scatter_blocks(T, cols)),
                                           dim3(256), 0, s, x, inv, T, k, has_shared, cols, q, scale);
         if (le != cudaSuccess) return le;
     }
@@ -779,15 +797,19 @@ __global__ void __launch_bounds__(256)
                        uint8_t* __restrict__ scale) {
     pdl_wait();  // inputs come from the previous kernel of the forward
     pdl_trigger();
-    const int64_t t = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+    const int64_t wid = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+    const int nch = scatter_chunks(cols);
+    const int64_t t = wid / nch;
     if (t >= T) return;
+    const int ch = (int)(wid - t * nch);
     const TokenRows tr = token_rows(inv, t, T, k, has_shared);
     const MxScaleLayout lay{rows, cols, false};
     const uint16_t* src = x + t * cols;
     const int lane = threadIdx.x & 31;
-    for (int c0 = 0; c0 < cols; c0 += 256) {
+    const int c_end = min(cols, (ch + 1) * kScatterCols);
+    for (int c0 = ch * kScatterCols; c0 < c_end; c0 += 256) {
         const int c = c0 + lane * 8;
-        const bool active = c < cols;
+        const bool active = c < c_end;
         uint4 u = make_uint4(0, 0, 0, 0);
         if (active) u = *reinterpret_cast<const uint4*>(src + c);
         float f[8];
@@ -817,7 +839,7 @@ cudaError_t launch_quant_mx_scatter(const uint16_t* x, const int32_t* inv, int T
     const int64_t rows = (int64_t)T * k + (has_shared ? T : 0);
     if (T == 0) return cudaSuccess;
     {
-        const cudaError_t le = launch_pdl(k_quant_mx_scatter, dim3((unsigned)((T + 7) / 8)),
+        const cudaError_t le = launch_pdl(k_quant_mx_scatter, dim3(scatter_blocks(T, cols)),
                                           dim3(256), 0, s, x, inv, T, k, has_shared, rows, cols, q,
                                           scale);
         if (le != cudaSuccess) return le;
@@ -993,14 +1015,18 @@ __global__ void __launch_bounds__(256)
                            int k, int has_shared, int cols, float s, uint8_t* __restrict__ q) {
     pdl_wait();  // inputs come from the previous kernel of the forward
     pdl_trigger();
-    const int64_t t = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+    const int64_t wid = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+    const int nch = scatter_chunks(cols);
+    const int64_t t = wid / nch;
     if (t >= T) return;
+    const int ch = (int)(wid - t * nch);
     const TokenRows tr = token_rows(inv, t, T, k, has_shared);
     const int lane = threadIdx.x & 31;
     const uint16_t* src = x + t * cols;
     const float r = __frcp_rn(s);
     const bool s_in_range = s >= 0x1p-26f && s <= 0x1p26f;
-    for (int c = lane * 8; c < cols; c += 256) {
+    const int c_end = min(cols, (ch + 1) * kScatterCols);
+    for (int c = ch * kScatterCols + lane * 8; c < c_end; c += 256) {
         float f[8];
         bf16x8_to_f32(*reinterpret_cast<const uint4*>(src + c), f);
         uint2 o;
@@ -1015,7 +1041,7 @@ cudaError_t launch_quant_act_fp8_static_scatter(const uint16_t* x, const int32_t
                                                 uint8_t* q, cudaStream_t s) {
     if (T == 0) return cudaSuccess;
     {
-        const cudaError_t le = launch_pdl(k_quant_static_scatter, dim3((unsigned)((T + 7) / 8)),
+        const cudaError_t le = launch_pdl(k_quant_static_scatter, dim3(scatter_blocks(T, cols)),
                                           dim3(256), 0, s, x, inv, T, k, has_shared, cols, scale, q);
         if (le != cudaSuccess) return le;
     }
