@@ -7,20 +7,25 @@
 // once, two accumulators hold the partial results and the epilogue applies a
 // single FMA (acc_hi + acc_lo / 256) before writing.
 //
-// B200 form: one CTA per 128-token x 64-expert tile.  A TMA warp streams the
-// x tile and the hi and lo tiles of each 64-wide k-block into a 4-stage
-// shared-memory ring (128-byte swizzle); one thread issues two tcgen05.mma per
-// 16-wide k-step, sharing the A descriptor, into TMEM accumulators; four
-// epilogue warps read them with tcgen05.ld and write FP32 logits.  Every wait
-// is bounded.
+// B200 form: one CTA per tile of 128 tokens x 64 experts, or x 128 experts
+// for an unsplit router over more than 64 experts that needs more than one
+// wave of 64-expert tiles (every tcgen05.mma costs at least ~120 cycles, so an
+// N = 64 MMA wastes half of an N = 128 one).  Two TMA warps (one loads x and
+// hi, the other lo: one thread completes a TMA load only about every 300
+// cycles) stream each 64-wide k-block into a 4-stage shared-memory ring
+// (128-byte swizzle); one thread issues two tcgen05.mma per 16-wide k-step,
+// sharing the A descriptor, into TMEM accumulators; four epilogue warps read
+// them with tcgen05.ld and write FP32 logits.  Every wait is bounded.
 //
 // Accuracy: the tensor core's FP32 accumulation loses a little at every MMA
 // step, in proportion to the running sum, and over d = 4096 (256 steps) that
 // alone reaches ~1e-5 of a logit.  The hi product therefore accumulates in
-// C = min(4, k-blocks) separate TMEM accumulators, one per contiguous quarter
-// of the k-blocks, summed pairwise in FP32 by the epilogue before the single
-// correcting FMA; lo (already scaled down by 256) keeps one accumulator.
-// TMEM columns: hi chunk c at c*64 .. c*64+63, lo at C*64 .. C*64+63.
+// C = min(4, k-blocks) separate TMEM accumulators (3 with 128-expert tiles,
+// where C + 1 accumulators fill TMEM), one per contiguous part of the
+// k-blocks, summed in FP32 by the epilogue ((c0 + c1) + (c2 + c3), or
+// (c0 + c1) + c2) before the single correcting FMA; lo (already scaled down by
+// 256) keeps one accumulator.  TMEM columns: hi chunk c at c*W .. c*W+W-1, lo
+// at C*W .. C*W+W-1, W the tile's expert count.
 //
 // Top-k fused into the epilogue (moe_forward, one CTA per tile): the routing
 // step needs all E logits of a token, which span E/64 CTAs.  Each CTA's
@@ -45,13 +50,20 @@ namespace moe {
 namespace {
 
 constexpr int BM = 128, BN = 64, BK = 64, STAGES = 4;
+// Wide tiles (128 experts, three hi chunks) for the unsplit router with more
+// than 64 experts: a tcgen05.mma with N <= 128 takes about as long as one with
+// N = 128 (measured: ~120 cycles each for N = 16 .. 128 at M = 128), so the
+// 64-expert tile spends half its MMA time on the fixed cost.  Three hi chunks
+// and lo fill the 512 TMEM columns.
+constexpr int BN_WIDE = 128, CHUNKS_WIDE = 3;
 constexpr int A_BYTES = BM * BK * 2;
-constexpr int B_BYTES = BN * BK * 2;
-constexpr int STAGE_BYTES = A_BYTES + 2 * B_BYTES;
-constexpr int THREADS = 192;  // warps 0-3 epilogue, 4 MMA + TMEM owner, 5 TMA
+template <int TN>
+constexpr int stage_bytes() { return A_BYTES + 2 * TN * BK * 2; }
+template <int TN>
+constexpr size_t smem_bytes() { return 1024 + STAGES * stage_bytes<TN>() + 256; }
+constexpr int THREADS = 224;  // warps 0-3 epilogue, 4 MMA + TMEM owner, 5 and 6 TMA
 constexpr int MAX_CHUNKS = 4;
-constexpr uint32_t TMEM_COLS = 512;  // (MAX_CHUNKS + 1) * BN = 320 used
-constexpr size_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
+constexpr uint32_t TMEM_COLS = 512;  // (chunks + 1) * tile width: 320 or 512 used
 
 constexpr int CAND = 8;  // candidates kept per token and 64-expert tile (k <= 8)
 
@@ -151,6 +163,7 @@ __device__ void merge_topk(const TopkArgs& tk, const float* logits, int64_t t, i
         }
 }
 
+template <int TN, int MAXC>
 __global__ void __launch_bounds__(THREADS, 1)
     k_router_dual(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_hi,
                   const __grid_constant__ CUtensorMap tm_lo, const float* __restrict__ bias,
@@ -160,7 +173,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+    constexpr int SB = stage_bytes<TN>(), TB = TN * BK * 2;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * SB);
     uint64_t* empty = full + STAGES;
     uint64_t* done = empty + STAGES;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
@@ -169,16 +183,16 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // grid x runs over the expert tiles, so the CTAs that share a 128-token x tile
     // are launched together and read it from DRAM once
-    const int m0 = blockIdx.y * BM, e0 = blockIdx.x * BN;
+    const int m0 = blockIdx.y * BM, e0 = blockIdx.x * TN;
     const int ksplit = gridDim.z, ks = blockIdx.z;
     const int nk_all = d / BK;
     const int kb0 = ks * nk_all / ksplit;                // this CTA's k-blocks: kb0 .. kb0+nk-1
     const int nk = (ks + 1) * nk_all / ksplit - kb0;
-    const int nchunks = nk < MAX_CHUNKS ? nk : MAX_CHUNKS;
+    const int nchunks = nk < MAXC ? nk : MAXC;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&full[s], 1);
+            mbar_init(&full[s], 2);  // one arrival per TMA producer
             mbar_init(&empty[s], 1);
         }
         mbar_init(done, 1);
@@ -193,11 +207,14 @@ __global__ void __launch_bounds__(THREADS, 1)
     pdl_wait();  // x may come from the previous kernel in the stream
     pdl_trigger();
 
-    if (warp == 5 && lane == 0) {
-        // ---------------- TMA producer
-        tma_prefetch_desc(&tm_x);
-        tma_prefetch_desc(&tm_hi);
-        tma_prefetch_desc(&tm_lo);
+    if ((warp == 5 || warp == 6) && lane == 0) {
+        // ---------------- TMA producers: warp 5 loads x and hi, warp 6 lo, each arming
+        // the stage's barrier for its own bytes before issuing them (one thread
+        // completes a TMA load only every ~300 cycles, so a stage's three loads from
+        // one thread would bound the k-loop)
+        const bool second = warp == 6;
+        tma_prefetch_desc(second ? &tm_lo : &tm_x);
+        if (!second) tma_prefetch_desc(&tm_hi);
         int issued = 0;
         for (int kb = 0; kb < nk; ++kb) {
             const int s = kb % STAGES;
@@ -207,11 +224,15 @@ __global__ void __launch_bounds__(THREADS, 1)
                 *abort_flag = 1;
                 break;
             }
-            uint8_t* st = smem + s * STAGE_BYTES;
-            mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
-            tma_load_2d(st, &tm_x, &full[s], (kb0 + kb) * BK, m0);
-            tma_load_2d(st + A_BYTES, &tm_hi, &full[s], (kb0 + kb) * BK, e0);
-            tma_load_2d(st + A_BYTES + B_BYTES, &tm_lo, &full[s], (kb0 + kb) * BK, e0);
+            uint8_t* st = smem + s * SB;
+            if (!second) {
+                mbar_arrive_expect_tx(&full[s], A_BYTES + TB);
+                tma_load_2d(st, &tm_x, &full[s], (kb0 + kb) * BK, m0);
+                tma_load_2d(st + A_BYTES, &tm_hi, &full[s], (kb0 + kb) * BK, e0);
+            } else {
+                mbar_arrive_expect_tx(&full[s], TB);
+                tma_load_2d(st + A_BYTES + TB, &tm_lo, &full[s], (kb0 + kb) * BK, e0);
+            }
             ++issued;
         }
         if (*abort_flag) {  // let the copies still in flight land before the block exits
@@ -220,7 +241,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
     } else if (warp == 4 && lane == 0) {
         // ---------------- MMA issuer
-        constexpr uint32_t idesc = idesc_bf16(BM, BN);
+        constexpr uint32_t idesc = idesc_bf16(BM, TN);
         for (int kb = 0; kb < nk; ++kb) {
             const int s = kb % STAGES;
             const uint32_t ph = (kb / STAGES) & 1;
@@ -230,11 +251,11 @@ __global__ void __launch_bounds__(THREADS, 1)
                 break;
             }
             tc_fence_after_sync();
-            const uint32_t a = smem_u32(smem + s * STAGE_BYTES);
-            const uint32_t bh = a + A_BYTES, bl = a + A_BYTES + B_BYTES;
+            const uint32_t a = smem_u32(smem + s * SB);
+            const uint32_t bh = a + A_BYTES, bl = a + A_BYTES + TB;
             const int chunk = kb * nchunks / nk;
             const bool chunk_start = kb * nchunks % nk < nchunks;  // first k-block of its chunk
-            const uint32_t d_hi = tmem + chunk * BN, d_lo = tmem + nchunks * BN;
+            const uint32_t d_hi = tmem + chunk * TN, d_lo = tmem + nchunks * TN;
 #pragma unroll
             for (int kk = 0; kk < BK / 16; ++kk) {
                 const uint64_t ad = sdesc_k_sw128(a + kk * 32);
@@ -261,17 +282,17 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
             for (int j = 0; j < CAND; ++j) best[j] = 0ull;
 #pragma unroll 1
-            for (int c = 0; c < BN / 32; ++c) {
+            for (int c = 0; c < TN / 32; ++c) {
                 float h[32], l[32], h2[32], h3[32];
-                tmem_load32x2(lane_base + c * 32, lane_base + nchunks * BN + c * 32, h, l);
+                tmem_load32x2(lane_base + c * 32, lane_base + nchunks * TN + c * 32, h, l);
                 if (nchunks >= 2) {
-                    tmem_load32(lane_base + BN + c * 32, h2);
+                    tmem_load32(lane_base + TN + c * 32, h2);
 #pragma unroll
                     for (int i = 0; i < 32; ++i) h[i] += h2[i];
                 }
                 if (nchunks >= 3) {
-                    tmem_load32(lane_base + 2 * BN + c * 32, h2);
-                    if (nchunks == 4) tmem_load32(lane_base + 3 * BN + c * 32, h3);
+                    tmem_load32(lane_base + 2 * TN + c * 32, h2);
+                    if (nchunks == 4) tmem_load32(lane_base + 3 * TN + c * 32, h3);
 #pragma unroll
                     for (int i = 0; i < 32; ++i) h[i] += (nchunks == 4) ? (h2[i] + h3[i]) : h2[i];
                 }
@@ -336,36 +357,55 @@ __global__ void __launch_bounds__(THREADS, 1)
         merge_topk(tk, logits, m0 + threadIdx.x, ntiles, E);
 }
 
-static cudaError_t launch_router_impl(const uint16_t* x, const uint16_t* hi, const uint16_t* lo,
-                                      const float* bias, float* logits, float* part_hi,
-                                      float* part_lo, int ksplit, int T, int d, int E,
-                                      int32_t* status, const TopkArgs& tk, cudaStream_t s) {
-    if (T == 0) return cudaSuccess;
+template <int TN, int MAXC>
+cudaError_t launch_router_tiles(const uint16_t* x, const uint16_t* hi, const uint16_t* lo,
+                                const float* bias, float* logits, float* part_hi, float* part_lo,
+                                int ksplit, int T, int d, int E, int32_t* status, const TopkArgs& tk,
+                                cudaStream_t s) {
     CUtensorMap tx, th, tl;
     if (!make_tmap_2d(&tx, x, 2, (uint64_t)T, (uint64_t)d, BM, BK) ||
-        !make_tmap_2d(&th, hi, 2, (uint64_t)E, (uint64_t)d, BN, BK) ||
-        !make_tmap_2d(&tl, lo, 2, (uint64_t)E, (uint64_t)d, BN, BK))
+        !make_tmap_2d(&th, hi, 2, (uint64_t)E, (uint64_t)d, TN, BK) ||
+        !make_tmap_2d(&tl, lo, 2, (uint64_t)E, (uint64_t)d, TN, BK))
         return cudaErrorInvalidValue;
     static bool attr_set[64] = {false};
     const int dev = current_device_info().device;
     if (dev < 64 && !attr_set[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(k_router_dual, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)SMEM_BYTES);
+        cudaError_t e = cudaFuncSetAttribute(k_router_dual<TN, MAXC>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem_bytes<TN>());
         if (e != cudaSuccess) return e;
         attr_set[dev] = true;
     }
-    dim3 grid((E + BN - 1) / BN, (T + BM - 1) / BM, ksplit);
+    dim3 grid((E + TN - 1) / TN, (T + BM - 1) / BM, ksplit);
     if (tk.ids != nullptr) {
         cudaError_t e = cudaMemsetAsync(tk.arrive_m, 0, sizeof(int32_t) * grid.y, s);
         if (e != cudaSuccess) return e;
     }
     {
-        const cudaError_t le = launch_pdl(k_router_dual, dim3(grid), dim3(THREADS), SMEM_BYTES, s,
-                                          tx, th, tl, bias, logits, part_hi, part_lo, T, d, E,
-                                          status, kDefaultTimeoutNs, tk);
+        const cudaError_t le = launch_pdl(k_router_dual<TN, MAXC>, dim3(grid), dim3(THREADS),
+                                          smem_bytes<TN>(), s, tx, th, tl, bias, logits, part_hi,
+                                          part_lo, T, d, E, status, kDefaultTimeoutNs, tk);
         if (le != cudaSuccess) return le;
     }
     return cudaGetLastError();
+}
+
+static cudaError_t launch_router_impl(const uint16_t* x, const uint16_t* hi, const uint16_t* lo,
+                                      const float* bias, float* logits, float* part_hi,
+                                      float* part_lo, int ksplit, int T, int d, int E,
+                                      int32_t* status, const TopkArgs& tk, cudaStream_t s) {
+    if (T == 0) return cudaSuccess;
+    // the wide tile for an unsplit router over more than 64 experts without the
+    // fused top-k (its merge assumes 64-expert tiles), when the 64-expert tiles
+    // would take more than one wave of the GPU (fewer, wider CTAs lose below
+    // that: 4096 tokens x 256 experts, 99.9 vs 94.7 us); the 64-expert tile otherwise
+    const int narrow_ctas = ((T + BM - 1) / BM) * ((E + BN - 1) / BN);
+    const bool wide = ksplit == 1 && E > BN && tk.ids == nullptr &&
+                      narrow_ctas > current_device_info().num_sms;
+    return wide ? launch_router_tiles<BN_WIDE, CHUNKS_WIDE>(x, hi, lo, bias, logits, part_hi, part_lo,
+                                                            ksplit, T, d, E, status, tk, s)
+                : launch_router_tiles<BN, MAX_CHUNKS>(x, hi, lo, bias, logits, part_hi, part_lo,
+                                                      ksplit, T, d, E, status, tk, s);
 }
 
 }  // namespace
