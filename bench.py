@@ -241,6 +241,7 @@ def power_capped(clocks: dict, ms_total: float) -> bool:
 KERNEL_SOURCES = {
     "k_gateup_bf16": ["csrc/gemm_bf16.cu", "csrc/common.cuh", "csrc/grouped_common.cuh"],
     "k_gateup_bf16_wide": ["csrc/gemm_bf16_wide.cu", "csrc/common.cuh", "csrc/grouped_common.cuh"],
+    "k_gateup_bf16_2sm": ["csrc/gemm_bf16_2sm.cu", "csrc/common.cuh", "csrc/grouped_common.cuh"],
     "k_gateup_fp8": ["csrc/gemm_fp8.cu", "csrc/common.cuh", "csrc/grouped_common.cuh"],
     "k_gateup_mx": ["csrc/gemm_mx.cu", "csrc/common.cuh", "csrc/grouped_common.cuh"],
     "k_gateup_f8t": ["csrc/gemm_f8t.cu", "csrc/common.cuh", "csrc/grouped_common.cuh"],
@@ -273,11 +274,13 @@ def recorded_traffic(kernel: str, workload: str):
 
 def gateup_kernel(cfg: MoEConfig, T: int, num_sms: int) -> str:
     """Name of the gate-up kernel moe_forward launches for this shape: the
-    library's dispatch rule (use_wide_gateup in launch.h) for BF16."""
+    library's dispatch rule for BF16 (use_pair_gateup in launch.h: the CTA-pair
+    kernel over x copied into the permuted row order from 256 rows per expert
+    on average, the one-CTA gathering kernel below)."""
     del num_sms
     if cfg.wdtype != 0:
         return "k_gateup_" + {1: "fp8", 2: "mx", 3: "f8t"}[cfg.wdtype]
-    return "k_gateup_bf16_wide" if T * cfg.k >= 256 * cfg.E else "k_gateup_bf16"
+    return "k_gateup_bf16_2sm" if T * cfg.k >= 256 * cfg.E else "k_gateup_bf16"
 
 
 def router_ksplit(T: int, d: int, E: int) -> int:
@@ -294,10 +297,12 @@ def kernels_per_step(cfg: MoEConfig, T: int) -> int:
     router (with the top-k fused into it when one CTA covers a tile's whole K
     and E <= 64, else followed by the top-k kernel), the permute (one kernel for at most
     1024 assignments, else count, scan and scatter), gate-up, down and
-    combine, plus the activation quantiser on the FP8 paths."""
+    combine, plus the activation quantiser on the FP8 paths and the copy of x
+    into the permuted row order before the CTA-pair BF16 gate-up."""
     router = 1 if router_ksplit(T, cfg.d, cfg.E) == 1 and cfg.E <= 64 else 2
     permute = 1 if T * cfg.k <= 1024 else 3
-    return router + permute + 3 + (1 if cfg.wdtype else 0)
+    a_prep = 1 if cfg.wdtype or T * cfg.k >= 256 * cfg.E else 0
+    return router + permute + 3 + a_prep
 
 
 def gateup_algorithmic(cfg: MoEConfig, T: int, n_active: int):

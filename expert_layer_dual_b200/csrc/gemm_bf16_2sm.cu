@@ -1,4 +1,5 @@
-// gemm_bf16_2sm.cu -- the grouped Down GEMM on CTA pairs (tcgen05 cta_group::2),
+// gemm_bf16_2sm.cu -- the grouped Down GEMM, and the Gate-Up GEMM over x
+// already in permuted row order (below), on CTA pairs (tcgen05 cta_group::2),
 // for workloads with many rows per expert.
 //
 // Same computation as the down kernel of gemm_bf16.cu ("HPC-Ops -
@@ -246,6 +247,100 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DOWN_THREADS, 1)
     teardown(tmem);
 }
 
+// ---------------------------------------------------------------------------
+// Gate-Up on a CTA pair: h[p][j] = silu(x_t . Wg[j]) * (x_t . Wu[j]) for a tile
+// of 256 permuted rows x 128 columns j of h.  Both operands arrive by TMA: the
+// rows from xp, x already copied into the permuted row order; CTA 0 loads the
+// tile's 128 gate rows of W_gu and CTA 1 the matching 128 up rows, the two
+// halves of the pair MMA's N = 256, so each CTA's accumulator holds its 128
+// rows x [gate | up].  A CTA-pair MMA runs at the tensor core's full rate
+// (8192 FLOP per SM cycle measured for M = 256, N = 256), the one-CTA M = 128
+// MMA of k_gateup_bf16_wide at 75% of it, and each CTA's two 256-column
+// accumulators alternate by tile, so a tile's epilogue overlaps the next
+// tile's MMAs.
+// ---------------------------------------------------------------------------
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DOWN_THREADS, 1)
+    k_gateup_bf16_2sm(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+                      const __grid_constant__ CUtensorMap tm_ws, GroupedGemmArgs a,
+                      uint16_t* __restrict__ h) {
+    extern __shared__ uint8_t smem_raw[];
+    Smem sm = carve(smem_raw);
+    Bars* b = sm.bars;
+    const volatile int* ab = &b->abort_flag;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const uint32_t tmem = prologue(sm, a, rank);
+    const int G = a.E + a.has_shared;
+    const int n_tiles = a.I / 128;
+    const int total = sm.tt->mstart[G] * n_tiles;
+    const int nk = a.d / BK;
+    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+
+    if (warp == TMA_WARP) {
+        if (lane == 0) {
+            tma_prefetch_desc(&tm_x);
+            tma_prefetch_desc(&tm_w);
+            tma_prefetch_desc(&tm_ws);
+            const uint32_t full_b_leader = smem_in_rank(&b->full_b[0], 0);
+            uint32_t it = 0;
+            bool ok = true;
+            for (int tile = pair; ok && tile < total; tile += npairs) {
+                const PairTile p = decode_pair(sm.tt, G, n_tiles, tile, rank);
+                const bool shared = p.t.g >= a.E;
+                const CUtensorMap* map = shared ? &tm_ws : &tm_w;
+                // CTA 0: the tile's gate rows, CTA 1: the matching up rows
+                const int rb = (shared ? 0 : p.t.g * 2 * a.I) + (int)rank * a.I + p.t.n * 128;
+                for (int kb = 0; kb < nk; ++kb, ++it) {
+                    const int s = it % STAGES;
+                    const uint32_t ph = (it / STAGES) & 1;
+                    if (!mbar_wait(&b->empty[s], ph ^ 1, a.timeout_ns, ab)) {
+                        fail(b, a.status);
+                        ok = false;
+                        break;
+                    }
+                    if (rank == 0) mbar_arrive_expect_tx(&b->full_b[s], 2 * (A_BYTES + B_BYTES));
+                    uint8_t* st = sm.stages + s * STAGE_BYTES;
+                    const uint32_t bar = full_b_leader + s * (uint32_t)sizeof(uint64_t);
+                    tma_load_2d_pair(st, &tm_x, bar, kb * BK, p.row0);
+                    tma_load_2d_pair(st + A_BYTES, map, bar, kb * BK, rb);
+                }
+            }
+        }
+    } else if (warp == MMA_WARP) {
+        if (lane == 0 && rank == 0) mma_role(sm, a, tmem, G, n_tiles, nk);
+    } else if (warp < EPI_WARPS) {
+        const int row = warp * 32 + lane;
+        uint32_t lt = 0;
+        for (int tile = pair; tile < total; tile += npairs, ++lt) {
+            const PairTile p = decode_pair(sm.tt, G, n_tiles, tile, rank);
+            const uint32_t buf = lt & 1, tph = (lt >> 1) & 1;
+            if (!warp_wait(&b->tfull[buf], tph, a.timeout_ns, ab)) { fail(b, a.status); break; }
+            tc_fence_after_sync();
+            const uint32_t taddr = tmem + (static_cast<uint32_t>(warp * 32) << 16) + buf * BN;
+            uint16_t* dst = h + (int64_t)(p.row0 + row) * a.I + p.t.n * 128;
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                float gv[32], uv[32];
+                tmem_load32x2(taddr + c * 32, taddr + 128 + c * 32, gv, uv);
+                if (row < p.nrows) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        pk[i] = pack_bf16x2(silu_f(gv[2 * i]) * uv[2 * i],
+                                            silu_f(gv[2 * i + 1]) * uv[2 * i + 1]);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        st_global_v4(dst + c * 32 + q * 8, pk[4 * q], pk[4 * q + 1], pk[4 * q + 2],
+                                     pk[4 * q + 3]);
+                }
+            }
+            tc_fence_before_sync();
+            warp_arrive_leader(&b->tempty[buf]);
+        }
+    }
+    teardown(tmem);
+}
+
 template <typename K>
 cudaError_t set_smem_once(K kernel, bool* flags) {
     const int dev = current_device_info().device;
@@ -259,6 +354,26 @@ cudaError_t set_smem_once(K kernel, bool* flags) {
 int pair_grid() { return (current_device_info().num_sms / 2) * 2; }
 
 }  // namespace
+
+cudaError_t launch_gateup_bf16_2sm(const GroupedGemmArgs& a, const uint16_t* xp, const uint16_t* w_gu,
+                                   const uint16_t* ws_gu, uint16_t* h, cudaStream_t s) {
+    if (a.T == 0) return cudaSuccess;
+    const uint64_t R = (uint64_t)a.T * a.k + (a.has_shared ? a.T : 0);
+    CUtensorMap tx, tw, tws;
+    if (!make_tmap_2d(&tx, xp, 2, R, (uint64_t)a.d, BM, BK) ||
+        !make_tmap_2d(&tw, w_gu, 2, (uint64_t)a.E * 2 * a.I, (uint64_t)a.d, 128, BK) ||
+        !make_tmap_2d(&tws, a.has_shared ? ws_gu : w_gu, 2, (uint64_t)2 * a.I, (uint64_t)a.d, 128, BK))
+        return cudaErrorInvalidValue;
+    static bool flags[64] = {false};
+    cudaError_t e = set_smem_once(k_gateup_bf16_2sm, flags);
+    if (e != cudaSuccess) return e;
+    {
+        const cudaError_t le = launch_pdl(k_gateup_bf16_2sm, dim3(pair_grid()), dim3(DOWN_THREADS),
+                                          SMEM_BYTES, s, tx, tw, tws, a, h);
+        if (le != cudaSuccess) return le;
+    }
+    return cudaGetLastError();
+}
 
 cudaError_t launch_down_bf16_2sm(const GroupedGemmArgs& a, const uint16_t* h, const uint16_t* w_d,
                                  const uint16_t* ws_d, __half* o, cudaStream_t s) {

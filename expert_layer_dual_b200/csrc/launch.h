@@ -92,6 +92,10 @@ cudaError_t launch_quant_weights_fp8_tensor(const uint16_t* W, int64_t batch, in
 cudaError_t launch_quant_act_fp8_static(const uint16_t* x, const int32_t* perm, int T, int k,
                                         int64_t rows, int cols, float scale, uint8_t* q,
                                         cudaStream_t s);
+// x [T][cols] bf16 copied to the permuted row order (rows inv[t*k + j], and
+// T*k + t with the shared expert): xp [T*k (+T)][cols].
+cudaError_t launch_permute_rows_bf16(const uint16_t* x, const int32_t* inv, int T, int k,
+                                     int has_shared, int cols, uint16_t* xp, cudaStream_t s);
 cudaError_t launch_quant_act_fp8_static_scatter(const uint16_t* x, const int32_t* inv, int T,
                                                 int k, int has_shared, int cols, float scale,
                                                 uint8_t* q, cudaStream_t s);
@@ -152,10 +156,17 @@ cudaError_t launch_gateup_bf16_wide(const GroupedGemmArgs& a, const uint16_t* x,
 inline bool use_wide_gateup(int T, int E, int k) { return (int64_t)T * k >= (int64_t)256 * E; }
 
 // ---- gemm_bf16_2sm.cu (down GEMM on CTA-pair tiles of 256 rows)
+// Gate-up on CTA pairs (256-row tiles, both operands by TMA) over x already in
+// the permuted row order (launch_permute_rows_bf16).
+cudaError_t launch_gateup_bf16_2sm(const GroupedGemmArgs& a, const uint16_t* xp, const uint16_t* w_gu,
+                                   const uint16_t* ws_gu, uint16_t* h, cudaStream_t s);
 cudaError_t launch_down_bf16_2sm(const GroupedGemmArgs& a, const uint16_t* h, const uint16_t* w_d,
                                  const uint16_t* ws_d, __half* o, cudaStream_t s);
 // Whether the CTA-pair down kernel serves this shape (>= 256 rows per expert on average).
 inline bool use_pair_tiles(int T, int E, int k) { return (int64_t)T * k >= (int64_t)256 * E; }
+// Whether the forward copies x into the permuted row order and runs the gate-up
+// on CTA pairs (the same shapes).
+inline bool use_pair_gateup(int T, int E, int k) { return use_pair_tiles(T, E, k); }
 
 // ---- gemm_fp8.cu (tcgen05 grouped GEMMs, e4m3 with 128x128 block scales)
 cudaError_t launch_gateup_fp8(const GroupedGemmArgs& a, const uint8_t* xq, const float* xs,

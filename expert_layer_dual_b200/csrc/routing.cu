@@ -1048,6 +1048,41 @@ cudaError_t launch_quant_act_fp8_static_scatter(const uint16_t* x, const int32_t
     return cudaGetLastError();
 }
 
+// x copied into the grouped GEMMs' permuted row order, token-major (bf16
+// rows; the CTA-pair gate-up then loads its A rows as TMA tiles): a warp per
+// 1024 columns of a token reads them once and stores them to each of the
+// token's k (+1) permuted rows.
+__global__ void __launch_bounds__(256)
+    k_permute_rows_scatter(const uint16_t* __restrict__ x, const int32_t* __restrict__ inv, int T,
+                           int k, int has_shared, int cols, uint16_t* __restrict__ xp) {
+    pdl_wait();  // inputs come from the previous kernel of the forward
+    pdl_trigger();
+    const int64_t wid = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+    const int nch = scatter_chunks(cols);
+    const int64_t t = wid / nch;
+    if (t >= T) return;
+    const int ch = (int)(wid - t * nch);
+    const TokenRows tr = token_rows(inv, t, T, k, has_shared);
+    const int lane = threadIdx.x & 31;
+    const uint16_t* src = x + t * cols;
+    const int c_end = min(cols, (ch + 1) * kScatterCols);
+    for (int c = ch * kScatterCols + lane * 8; c < c_end; c += 256) {
+        const uint4 v = *reinterpret_cast<const uint4*>(src + c);
+        for_token_rows(tr, [&](int64_t p) { *reinterpret_cast<uint4*>(xp + p * cols + c) = v; });
+    }
+}
+
+cudaError_t launch_permute_rows_bf16(const uint16_t* x, const int32_t* inv, int T, int k,
+                                     int has_shared, int cols, uint16_t* xp, cudaStream_t s) {
+    if (T == 0) return cudaSuccess;
+    {
+        const cudaError_t le = launch_pdl(k_permute_rows_scatter, dim3(scatter_blocks(T, cols)),
+                                          dim3(256), 0, s, x, inv, T, k, has_shared, cols, xp);
+        if (le != cudaSuccess) return le;
+    }
+    return cudaGetLastError();
+}
+
 cudaError_t launch_quant_act_fp8_static(const uint16_t* x, const int32_t* perm, int T, int k,
                                         int64_t rows, int cols, float scale, uint8_t* q,
                                         cudaStream_t s) {

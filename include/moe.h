@@ -130,12 +130,14 @@ size_t moe_workspace_bytes(const moe_shape* shape);
  *   ids int32 [T][k], w float [T][k]           moe_route_topk's outputs
  *   counts int32 [E], offsets int32 [E+1], perm, inv int32 [T*k]
  *                                              moe_permute's outputs
- *   xq, xs  the quantised activations the gate-up read (FP8 formats), in the
- *           permuted row order: the outputs moe_quantize_act_fp8_permuted,
- *           moe_quantize_act_mxfp8_permuted or moe_quantize_act_fp8_static_permuted
- *           give for this routing's perm (xs: FP32 [R][d/128] for wdtype 1,
- *           the E8M0 bytes for wdtype 2, absent for wdtype 3); 0 where the
- *           format has no such region (wdtype 0; xs of wdtype 3)
+ *   xq, xs  the gate-up's A operand where the forward writes it in the permuted
+ *           row order.  FP8 formats: the quantised activations, the outputs
+ *           moe_quantize_act_fp8_permuted, moe_quantize_act_mxfp8_permuted or
+ *           moe_quantize_act_fp8_static_permuted give for this routing's perm
+ *           (xs: FP32 [R][d/128] for wdtype 1, the E8M0 bytes for wdtype 2,
+ *           absent for wdtype 3).  wdtype 0 with T*k >= 256*E (the gate-up on
+ *           CTA pairs): xq holds the bf16 rows of x [R][d] in that order, no xs.
+ *           0 where there is no such region
  *   h   the gate-up output (wdtype 0: bf16 [R][I], R = T*k + (I_shared ? T : 0))
  *   total  = moe_workspace_bytes(shape).
  * Inspection and testing aid; returns MOE_ERR_INVALID_ARG / UNSUPPORTED as

@@ -79,7 +79,7 @@ def test_workspace_map_regions(lib):
         for n, off in regs.items():
             assert off % 256 == 0 and off < m.total, (wd, n)
         R = 200 * 4 + 200
-        assert (regs["xq"] > 0) == (wd != 0)
+        assert (regs["xq"] > 0) == (wd != 0)   # 200 x 4 rows over 16 experts: no pair gate-up
         assert (regs["xs"] > 0) == (wd in (1, 2))
         if wd:
             assert regs["xq"] + R * 512 <= m.total

@@ -91,7 +91,7 @@ def test_gateup_kernel_follows_the_library_dispatch():
     from expert_layer_dual_b200.configs import CONFIGS
     names = {n: bench.gateup_kernel(CONFIGS[n], CONFIGS[n].T, 148) for n in CONFIGS}
     assert names["decode"] == names["tiny"] == "k_gateup_bf16"
-    assert names["prefill"] == names["skew"] == "k_gateup_bf16_wide"
+    assert names["prefill"] == names["skew"] == "k_gateup_bf16_2sm"
     assert names["fp8"] == "k_gateup_fp8" and names["mxfp8"] == "k_gateup_mx"
     assert names["fp8t"] == "k_gateup_f8t"
     assert set(names.values()) <= set(bench.KERNEL_SOURCES)
@@ -106,7 +106,8 @@ def test_launch_count_follows_the_library_dispatch():
     assert bench.router_ksplit(64, 4096, 256) == 8 and bench.router_ksplit(8192, 4096, 256) == 1
     # one CTA per router tile and E <= 64: the top-k runs inside the router kernel
     assert n["tiny"] == 5
-    # 256 experts: router, top-k, the permute in three kernels (count, scan, scatter)
-    assert n["prefill"] == n["skew"] == 8
+    # 256 experts: router, top-k, the permute in three kernels (count, scan, scatter), the
+    # copy of x into the permuted row order for the CTA-pair gate-up
+    assert n["prefill"] == n["skew"] == 9
     # + the activation quantiser
     assert n["fp8"] == n["mxfp8"] == n["fp8t"] == 9

@@ -1,7 +1,8 @@
-"""GPU: the activation quantisation inside moe_forward (FP8 formats) is
-token-major -- each token's row is quantised once and its codes stored to
-each permuted row that holds it (the rows inv[t*k + j], and T*k + t with the
-shared expert).  Its output, read from the forward's workspace, must equal
+"""GPU: the preparation of the gate-up's A operand inside moe_forward is
+token-major -- each token's row is read (and, for the FP8 formats, quantised)
+once and stored to each permuted row that holds it (the rows inv[t*k + j],
+and T*k + t with the shared expert).  FP8 formats: the output, read from the
+forward's workspace, must equal
 bit for bit both the stage entry point that quantises each permuted row on
 its own (moe_quantize_act_*_permuted, given the forward's perm) and the
 oracle's quantisation of the rows x[perm / k] (plus x for the shared rows):
@@ -9,7 +10,8 @@ oracle's quantisation of the rows x[perm / k] (plus x for the shared rows):
  - MXFP8: e4m3 codes and E8M0 bytes per 1x32 (oracle.quant_mx_rows);
  - per-tensor FP8: e4m3 codes of v / s_x (oracle.quant_fp8_static).
 Configurations cover k = 2, 4, 8 (every copy slot), with and without the
-shared expert, and ragged token counts."""
+shared expert, and ragged token counts.  BF16 with >= 256 rows per expert on
+average (the CTA-pair gate-up): the bf16 rows of x in that order, bit for bit."""
 import numpy as np
 import pytest
 import torch
@@ -83,3 +85,25 @@ def test_forward_quantisation_is_bit_exact(cfg):
     else:
         oq = oracle.quant_fp8_static(rows, np.float32(layer.act_scales[0]))
     assert np.array_equal(xq.cpu().numpy(), oq)
+
+
+@pytest.mark.parametrize("cfg", [
+    MoEConfig("pair", T=1100, d=512, E=8, k=4, I=256, Is=256, seed=64),
+    MoEConfig("pairodd", T=1100, d=384, E=6, k=3, I=128, Is=0, seed=65),
+], ids=lambda c: c.name)
+def test_forward_permuted_x_bf16(cfg):
+    # BF16 with >= 256 rows per expert on average: the forward copies x into the
+    # permuted row order (token-major) for the CTA-pair gate-up; row p must be
+    # x[perm[p] / k] (routed rows) or x[p - T*k] (shared rows), bit for bit
+    inp = make_layer(cfg)
+    layer = M.MoELayer(cfg, inp)
+    x_dev = inp["x"].to(DEV)
+    layer.forward(x_dev)
+    torch.cuda.synchronize()
+    assert layer.device_status() == M.OK
+    view = M.workspace_view(layer.ws, layer.shape(cfg.T))
+    assert "xq" in view
+    p = view["perm"].cpu().numpy().astype(np.int64)
+    tok = np.concatenate([p // cfg.k, np.arange(cfg.T) if cfg.Is else np.zeros(0, np.int64)])
+    want = inp["x"].view(torch.int16).numpy()[tok]
+    assert np.array_equal(view["xq"].cpu().view(torch.int16).numpy(), want)
