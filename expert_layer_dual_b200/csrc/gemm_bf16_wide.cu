@@ -17,7 +17,10 @@
 // timing, against the 128-row kernel, both with the fast SiLU: 4-7% faster
 // per step at prefill (~256 rows per expert), 3% on the skewed workload,
 // 2-3% with ~512 rows per expert, 1-7% on a dense 16384-row problem; so it
-// serves shapes with at least 256 rows per expert on average.
+// serves shapes with at least 256 rows per expert on average when x is
+// gathered through the permutation (the stage entry point moe_gemm_gateup);
+// the forward at those shapes copies x into the permuted order and runs the
+// CTA-pair gate-up of gemm_bf16_2sm.cu instead (~2% faster per step).
 //  - persistent, one CTA per SM, tiles from the dynamic schedule of
 //    grouped_common.cuh;
 //  - three 64 KB stages: 256 rows gathered from x through the permutation by

@@ -11,7 +11,8 @@ oracle's quantisation of the rows x[perm / k] (plus x for the shared rows):
  - per-tensor FP8: e4m3 codes of v / s_x (oracle.quant_fp8_static).
 Configurations cover k = 2, 4, 8 (every copy slot), with and without the
 shared expert, and ragged token counts.  BF16 with >= 256 rows per expert on
-average (the CTA-pair gate-up): the bf16 rows of x in that order, bit for bit."""
+average (the CTA-pair gate-up): the bf16 rows of x in that order, bit for bit,
+and the pair gate-up's h equal to the gathering gate-up's on the same routing."""
 import numpy as np
 import pytest
 import torch
@@ -107,3 +108,29 @@ def test_forward_permuted_x_bf16(cfg):
     tok = np.concatenate([p // cfg.k, np.arange(cfg.T) if cfg.Is else np.zeros(0, np.int64)])
     want = inp["x"].view(torch.int16).numpy()[tok]
     assert np.array_equal(view["xq"].cpu().view(torch.int16).numpy(), want)
+
+
+@pytest.mark.parametrize("cfg", [
+    MoEConfig("pair", T=1100, d=512, E=8, k=4, I=256, Is=256, seed=66),
+    MoEConfig("pairodd", T=1100, d=384, E=6, k=3, I=128, Is=0, seed=67),
+], ids=lambda c: c.name)
+def test_pair_gateup_equals_gathering_gateup(cfg):
+    # the forward's gate-up on CTA pairs (A rows from the permuted copy of x) and
+    # the stage entry point's gate-up (x gathered through perm, one-CTA tiles) on
+    # the same routing give the same h, bit for bit
+    inp = make_layer(cfg)
+    layer = M.MoELayer(cfg, inp)
+    x_dev = inp["x"].to(DEV)
+    layer.forward(x_dev)
+    torch.cuda.synchronize()
+    assert layer.device_status() == M.OK
+    shape = layer.shape(cfg.T)
+    view = M.workspace_view(layer.ws, shape)
+    h_pair = view["h"].clone()
+    perm, offsets = view["perm"].clone(), view["offsets"].clone()
+    h = torch.empty_like(h_pair)
+    ws = torch.zeros(M.workspace_bytes(shape), dtype=torch.uint8, device=DEV)
+    M.gemm_gateup(shape, layer.weights, x_dev.view(torch.uint16), None, perm, offsets, h.view(torch.uint16),
+                  None, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(h.view(torch.int16), h_pair.view(torch.int16))
