@@ -117,8 +117,8 @@ WsLayout ws_layout(const moe_shape& s) {
         L.h = take(R * I);
         L.hs = take(R * (I / 32));
     } else {
-        // x in permuted row order (bf16) when the gate-up runs on CTA pairs
-        L.xq = use_pair_gateup(s.T, s.E, s.k) ? take(R * d * 2) : 0;
+        // x's routed rows in permuted order (bf16) when the gate-up runs on CTA pairs
+        L.xq = use_pair_gateup(s.T, s.E, s.k) ? take(T * k * d * 2) : 0;
         L.xs = L.hs = 0;
         L.h = take(R * I * 2);
     }
@@ -211,17 +211,17 @@ inline P* at(void* ws, size_t off) {
     return reinterpret_cast<P*>(static_cast<uint8_t*>(ws) + off);
 }
 
-// BF16 with `x_permuted`: x is already in the permuted row order (the
-// forward's copy) and the gate-up runs on CTA pairs; otherwise the kernels
-// gather x through perm.
+// BF16 with `xp` (the forward's copy of x's routed rows in the permuted row
+// order): the gate-up runs on CTA pairs; otherwise the kernels gather x
+// through perm.
 moe_status run_gateup(const moe_shape* s, const moe_weights* w, const void* x, const void* xs,
                       const int32_t* perm, const int32_t* offsets, void* h, void* hs,
                       int32_t* status, cudaStream_t st, bool counter_zeroed = false,
-                      bool x_permuted = false) {
+                      const uint16_t* xp = nullptr) {
     const GroupedGemmArgs a = gemm_args(s, offsets, perm, status, kGateupCounter, counter_zeroed);
-    if (s->wdtype == MOE_WDTYPE_BF16 && x_permuted)
+    if (s->wdtype == MOE_WDTYPE_BF16 && xp != nullptr)
         return cuda_status(launch_gateup_bf16_2sm(
-            a, static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(w->w_gu),
+            a, xp, static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(w->w_gu),
             static_cast<const uint16_t*>(w->ws_gu), static_cast<uint16_t*>(h), st));
     if (s->wdtype == MOE_WDTYPE_BF16)
         return cuda_status((use_wide_gateup(s->T, s->E, s->k) ? launch_gateup_bf16_wide
@@ -355,12 +355,13 @@ moe_status forward_device(const moe_shape* s, const moe_weights* w, const uint16
     if ((r = route_device(s, w, x, ws, L, st, events)) != MOE_OK) return r;
     const void* a_in = x;
     const void* a_scale = nullptr;
-    const bool x_permuted = s->wdtype == MOE_WDTYPE_BF16 && use_pair_gateup(s->T, s->E, s->k);
-    if (x_permuted) {
-        if ((r = cuda_status(launch_permute_rows_bf16(x, inv, s->T, s->k, s->I_shared > 0 ? 1 : 0,
-                                                      s->d, at<uint16_t>(ws, L.xq), st))) != MOE_OK)
+    const uint16_t* xp = nullptr;
+    if (s->wdtype == MOE_WDTYPE_BF16 && use_pair_gateup(s->T, s->E, s->k)) {
+        // the routed rows only: the pair gate-up reads the shared expert's rows from x
+        if ((r = cuda_status(launch_permute_rows_bf16(x, inv, s->T, s->k, 0, s->d,
+                                                      at<uint16_t>(ws, L.xq), st))) != MOE_OK)
             return r;
-        a_in = at<uint16_t>(ws, L.xq);
+        xp = at<uint16_t>(ws, L.xq);
     }
     if (f8t) {
         if ((r = cuda_status(launch_quant_act_fp8_static_scatter(
@@ -390,8 +391,7 @@ moe_status forward_device(const moe_shape* s, const moe_weights* w, const uint16
     void* h = at<uint8_t>(ws, L.h);
     void* hs = (fp8 || mx) ? at<uint8_t>(ws, L.hs) : nullptr;
     __half* o = at<__half>(ws, L.o);
-    if ((r = run_gateup(s, w, a_in, a_scale, perm, offsets, h, hs, status, st, true, x_permuted)) !=
-        MOE_OK)
+    if ((r = run_gateup(s, w, a_in, a_scale, perm, offsets, h, hs, status, st, true, xp)) != MOE_OK)
         return r;
     if (!mark(5)) return MOE_ERR_CUDA;
     if ((r = run_down(s, w, h, hs, offsets, o, status, st, true)) != MOE_OK) return r;

@@ -250,7 +250,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DOWN_THREADS, 1)
 // ---------------------------------------------------------------------------
 // Gate-Up on a CTA pair: h[p][j] = silu(x_t . Wg[j]) * (x_t . Wu[j]) for a tile
 // of 256 permuted rows x 128 columns j of h.  Both operands arrive by TMA: the
-// rows from xp, x already copied into the permuted row order; CTA 0 loads the
+// routed rows from xp, x already copied into the permuted row order, the shared
+// expert's rows (token order) from x itself; CTA 0 loads the
 // tile's 128 gate rows of W_gu and CTA 1 the matching 128 up rows, the two
 // halves of the pair MMA's N = 256, so each CTA's accumulator holds its 128
 // rows x [gate | up].  A CTA-pair MMA runs at the tensor core's full rate
@@ -260,9 +261,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DOWN_THREADS, 1)
 // tile's MMAs.
 // ---------------------------------------------------------------------------
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DOWN_THREADS, 1)
-    k_gateup_bf16_2sm(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
-                      const __grid_constant__ CUtensorMap tm_ws, GroupedGemmArgs a,
-                      uint16_t* __restrict__ h) {
+    k_gateup_bf16_2sm(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_xt,
+                      const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_ws,
+                      GroupedGemmArgs a, uint16_t* __restrict__ h) {
     extern __shared__ uint8_t smem_raw[];
     Smem sm = carve(smem_raw);
     Bars* b = sm.bars;
@@ -279,15 +280,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DOWN_THREADS, 1)
     if (warp == TMA_WARP) {
         if (lane == 0) {
             tma_prefetch_desc(&tm_x);
+            tma_prefetch_desc(&tm_xt);
             tma_prefetch_desc(&tm_w);
             tma_prefetch_desc(&tm_ws);
             const uint32_t full_b_leader = smem_in_rank(&b->full_b[0], 0);
+            const int Tk = a.T * a.k;
             uint32_t it = 0;
             bool ok = true;
             for (int tile = pair; ok && tile < total; tile += npairs) {
                 const PairTile p = decode_pair(sm.tt, G, n_tiles, tile, rank);
                 const bool shared = p.t.g >= a.E;
                 const CUtensorMap* map = shared ? &tm_ws : &tm_w;
+                // rows: the routed ones from the permuted copy, the shared expert's from x
+                const CUtensorMap* amap = shared ? &tm_xt : &tm_x;
+                const int arow = shared ? p.row0 - Tk : p.row0;
                 // CTA 0: the tile's gate rows, CTA 1: the matching up rows
                 const int rb = (shared ? 0 : p.t.g * 2 * a.I) + (int)rank * a.I + p.t.n * 128;
                 for (int kb = 0; kb < nk; ++kb, ++it) {
@@ -301,7 +307,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DOWN_THREADS, 1)
                     if (rank == 0) mbar_arrive_expect_tx(&b->full_b[s], 2 * (A_BYTES + B_BYTES));
                     uint8_t* st = sm.stages + s * STAGE_BYTES;
                     const uint32_t bar = full_b_leader + s * (uint32_t)sizeof(uint64_t);
-                    tma_load_2d_pair(st, &tm_x, bar, kb * BK, p.row0);
+                    tma_load_2d_pair(st, amap, bar, kb * BK, arow);
                     tma_load_2d_pair(st + A_BYTES, map, bar, kb * BK, rb);
                 }
             }
@@ -355,12 +361,13 @@ int pair_grid() { return (current_device_info().num_sms / 2) * 2; }
 
 }  // namespace
 
-cudaError_t launch_gateup_bf16_2sm(const GroupedGemmArgs& a, const uint16_t* xp, const uint16_t* w_gu,
-                                   const uint16_t* ws_gu, uint16_t* h, cudaStream_t s) {
+cudaError_t launch_gateup_bf16_2sm(const GroupedGemmArgs& a, const uint16_t* xp, const uint16_t* x,
+                                   const uint16_t* w_gu, const uint16_t* ws_gu, uint16_t* h,
+                                   cudaStream_t s) {
     if (a.T == 0) return cudaSuccess;
-    const uint64_t R = (uint64_t)a.T * a.k + (a.has_shared ? a.T : 0);
-    CUtensorMap tx, tw, tws;
-    if (!make_tmap_2d(&tx, xp, 2, R, (uint64_t)a.d, BM, BK) ||
+    CUtensorMap tx, txt, tw, tws;
+    if (!make_tmap_2d(&tx, xp, 2, (uint64_t)a.T * a.k, (uint64_t)a.d, BM, BK) ||
+        !make_tmap_2d(&txt, x, 2, (uint64_t)a.T, (uint64_t)a.d, BM, BK) ||
         !make_tmap_2d(&tw, w_gu, 2, (uint64_t)a.E * 2 * a.I, (uint64_t)a.d, 128, BK) ||
         !make_tmap_2d(&tws, a.has_shared ? ws_gu : w_gu, 2, (uint64_t)2 * a.I, (uint64_t)a.d, 128, BK))
         return cudaErrorInvalidValue;
@@ -369,7 +376,7 @@ cudaError_t launch_gateup_bf16_2sm(const GroupedGemmArgs& a, const uint16_t* xp,
     if (e != cudaSuccess) return e;
     {
         const cudaError_t le = launch_pdl(k_gateup_bf16_2sm, dim3(pair_grid()), dim3(DOWN_THREADS),
-                                          SMEM_BYTES, s, tx, tw, tws, a, h);
+                                          SMEM_BYTES, s, tx, txt, tw, tws, a, h);
         if (le != cudaSuccess) return le;
     }
     return cudaGetLastError();

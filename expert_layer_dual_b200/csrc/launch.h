@@ -156,10 +156,13 @@ cudaError_t launch_gateup_bf16_wide(const GroupedGemmArgs& a, const uint16_t* x,
 inline bool use_wide_gateup(int T, int E, int k) { return (int64_t)T * k >= (int64_t)256 * E; }
 
 // ---- gemm_bf16_2sm.cu (down GEMM on CTA-pair tiles of 256 rows)
-// Gate-up on CTA pairs (256-row tiles, both operands by TMA) over x already in
-// the permuted row order (launch_permute_rows_bf16).
-cudaError_t launch_gateup_bf16_2sm(const GroupedGemmArgs& a, const uint16_t* xp, const uint16_t* w_gu,
-                                   const uint16_t* ws_gu, uint16_t* h, cudaStream_t s);
+// Gate-up on CTA pairs (256-row tiles, both operands by TMA): the routed rows
+// from xp [T*k][d], x's routed copies in the permuted row order
+// (launch_permute_rows_bf16 without the shared rows), the shared expert's rows
+// from x [T][d].
+cudaError_t launch_gateup_bf16_2sm(const GroupedGemmArgs& a, const uint16_t* xp, const uint16_t* x,
+                                   const uint16_t* w_gu, const uint16_t* ws_gu, uint16_t* h,
+                                   cudaStream_t s);
 cudaError_t launch_down_bf16_2sm(const GroupedGemmArgs& a, const uint16_t* h, const uint16_t* w_d,
                                  const uint16_t* ws_d, __half* o, cudaStream_t s);
 // Whether the CTA-pair down kernel serves this shape (>= 256 rows per expert on average).

@@ -183,8 +183,8 @@ def workspace_view(ws: torch.Tensor, shape: moe_shape) -> dict:
            "inv": region(m.inv, T * k, torch.int32)}
     if shape.wdtype == WDTYPE_BF16:
         out["h"] = region(m.h, R * shape.I, torch.bfloat16).view(R, shape.I)
-        if m.xq:
-            out["xq"] = region(m.xq, R * shape.d, torch.bfloat16).view(R, shape.d)
+        if m.xq:   # the routed rows of x in permuted order (the CTA-pair gate-up's A)
+            out["xq"] = region(m.xq, T * k * shape.d, torch.bfloat16).view(T * k, shape.d)
     else:
         d = shape.d
         out["xq"] = region(m.xq, R * d, torch.uint8).view(R, d)

@@ -136,7 +136,8 @@ size_t moe_workspace_bytes(const moe_shape* shape);
  *           moe_quantize_act_fp8_static_permuted give for this routing's perm
  *           (xs: FP32 [R][d/128] for wdtype 1, the E8M0 bytes for wdtype 2,
  *           absent for wdtype 3).  wdtype 0 with T*k >= 256*E (the gate-up on
- *           CTA pairs): xq holds the bf16 rows of x [R][d] in that order, no xs.
+ *           CTA pairs): xq holds the bf16 routed rows of x [T*k][d] in that order
+ *           (the shared expert's rows are read from x itself), no xs.
  *           0 where there is no such region
  *   h   the gate-up output (wdtype 0: bf16 [R][I], R = T*k + (I_shared ? T : 0))
  *   total  = moe_workspace_bytes(shape).

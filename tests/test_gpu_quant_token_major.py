@@ -11,7 +11,7 @@ oracle's quantisation of the rows x[perm / k] (plus x for the shared rows):
  - per-tensor FP8: e4m3 codes of v / s_x (oracle.quant_fp8_static).
 Configurations cover k = 2, 4, 8 (every copy slot), with and without the
 shared expert, and ragged token counts.  BF16 with >= 256 rows per expert on
-average (the CTA-pair gate-up): the bf16 rows of x in that order, bit for bit,
+average (the CTA-pair gate-up): the bf16 routed rows of x in that order, bit for bit,
 and the pair gate-up's h equal to the gathering gate-up's on the same routing."""
 import numpy as np
 import pytest
@@ -93,9 +93,10 @@ def test_forward_quantisation_is_bit_exact(cfg):
     MoEConfig("pairodd", T=1100, d=384, E=6, k=3, I=128, Is=0, seed=65),
 ], ids=lambda c: c.name)
 def test_forward_permuted_x_bf16(cfg):
-    # BF16 with >= 256 rows per expert on average: the forward copies x into the
-    # permuted row order (token-major) for the CTA-pair gate-up; row p must be
-    # x[perm[p] / k] (routed rows) or x[p - T*k] (shared rows), bit for bit
+    # BF16 with >= 256 rows per expert on average: the forward copies x's routed
+    # rows into the permuted row order (token-major) for the CTA-pair gate-up (which
+    # reads the shared expert's rows from x itself); row p must be x[perm[p] / k],
+    # bit for bit
     inp = make_layer(cfg)
     layer = M.MoELayer(cfg, inp)
     x_dev = inp["x"].to(DEV)
@@ -105,8 +106,7 @@ def test_forward_permuted_x_bf16(cfg):
     view = M.workspace_view(layer.ws, layer.shape(cfg.T))
     assert "xq" in view
     p = view["perm"].cpu().numpy().astype(np.int64)
-    tok = np.concatenate([p // cfg.k, np.arange(cfg.T) if cfg.Is else np.zeros(0, np.int64)])
-    want = inp["x"].view(torch.int16).numpy()[tok]
+    want = inp["x"].view(torch.int16).numpy()[p // cfg.k]
     assert np.array_equal(view["xq"].cpu().view(torch.int16).numpy(), want)
 
 
