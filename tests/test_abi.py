@@ -83,3 +83,13 @@ def test_workspace_map_regions(lib):
         assert (regs["xs"] > 0) == (wd in (1, 2))
         if wd:
             assert regs["xq"] + R * 512 <= m.total
+    # BF16 with >= 256 rows per expert on average (the CTA-pair gate-up): xq holds x's
+    # T*k routed rows in permuted order (the shared expert's rows are read from x), no xs
+    T, d, E, k = 1100, 512, 8, 4
+    s = M.moe_shape(T, d, E, k, 256, 256, 0, 1)
+    m = M.workspace_offsets(s)
+    regs = {n: getattr(m, n) for n in ("logits", "ids", "w", "counts", "offsets", "perm", "inv",
+                                       "xq", "xs", "h")}
+    assert regs["xq"] > 0 and regs["xs"] == 0
+    nxt = min([off for off in regs.values() if off > regs["xq"]] + [m.total])
+    assert nxt - regs["xq"] == T * k * d * 2
