@@ -150,9 +150,17 @@ moe_status check_shape(const moe_shape* s) {
     return MOE_OK;
 }
 
+// Row buffers and weight matrices are read by TMA (whose base must be 16-byte
+// aligned) or with 16-byte vector accesses.
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
 moe_status check_weights(const moe_shape* s, const moe_weights* w, bool need_gateup,
                          bool need_down, bool need_router) {
     if (w == nullptr) return MOE_ERR_INVALID_ARG;
+    // the weight matrices are TMA sources
+    if (!aligned16(w->w_gu) || !aligned16(w->w_d) || !aligned16(w->ws_gu) || !aligned16(w->ws_d) ||
+        !aligned16(w->router_hi) || !aligned16(w->router_lo))
+        return MOE_ERR_INVALID_ARG;
     const bool fp8 = s->wdtype != MOE_WDTYPE_BF16;  // scaled weights (FP8 or MXFP8)
     const bool sh = s->I_shared > 0;
     if (need_gateup && (w->w_gu == nullptr || (fp8 && w->w_gu_scale == nullptr) ||
@@ -441,7 +449,8 @@ moe_status moe_quantize_weights_fp8(const uint16_t* W, int64_t batch, int32_t ro
     if (batch < 0 || rows < 0 || cols < 0) return MOE_ERR_INVALID_ARG;
     if (rows % 128 != 0 || cols % 128 != 0) return MOE_ERR_UNSUPPORTED;
     if (batch * rows * (int64_t)cols == 0) return MOE_OK;
-    if (W == nullptr || q == nullptr || scale == nullptr) return MOE_ERR_INVALID_ARG;
+    if (W == nullptr || q == nullptr || scale == nullptr || !aligned16(W) || !aligned16(q))
+        return MOE_ERR_INVALID_ARG;
     if (!device_ok()) return MOE_ERR_UNSUPPORTED;
     if (batch * (rows / 128) * (int64_t)(cols / 128) >= ((int64_t)1 << 31)) return MOE_ERR_UNSUPPORTED;
     return cuda_status(launch_quant_weights_fp8(W, batch, rows, cols, q, scale, as_stream(stream)));
@@ -452,7 +461,8 @@ moe_status moe_quantize_act_fp8(const uint16_t* x, int64_t rows, int32_t cols, u
     if (rows < 0 || cols < 0) return MOE_ERR_INVALID_ARG;
     if (cols % 128 != 0) return MOE_ERR_UNSUPPORTED;
     if (rows * (int64_t)cols == 0) return MOE_OK;
-    if (x == nullptr || q == nullptr || scale == nullptr) return MOE_ERR_INVALID_ARG;
+    if (x == nullptr || q == nullptr || scale == nullptr || !aligned16(x) || !aligned16(q))
+        return MOE_ERR_INVALID_ARG;
     if (!device_ok()) return MOE_ERR_UNSUPPORTED;
     return cuda_status(launch_quant_act_fp8(x, rows, cols, q, scale, as_stream(stream)));
 }
@@ -462,7 +472,8 @@ moe_status moe_quantize_weights_fp8_tensor(const uint16_t* W, int64_t batch, int
     if (batch < 0 || rows < 0 || cols < 0) return MOE_ERR_INVALID_ARG;
     if (cols % 8 != 0) return MOE_ERR_UNSUPPORTED;
     if (batch * rows * (int64_t)cols == 0) return MOE_OK;
-    if (W == nullptr || q == nullptr || scale == nullptr) return MOE_ERR_INVALID_ARG;
+    if (W == nullptr || q == nullptr || scale == nullptr || !aligned16(W) || !aligned16(q))
+        return MOE_ERR_INVALID_ARG;
     if (batch >= 65536) return MOE_ERR_UNSUPPORTED;
     if (!device_ok()) return MOE_ERR_UNSUPPORTED;
     return cuda_status(launch_quant_weights_fp8_tensor(W, batch, rows, cols, q, scale, as_stream(stream)));
@@ -473,7 +484,7 @@ moe_status moe_quantize_act_fp8_static(const uint16_t* x, int64_t rows, int32_t 
     if (rows < 0 || cols <= 0 || !(scale > 0.0f) || !isfinite(scale)) return MOE_ERR_INVALID_ARG;
     if (cols % 8 != 0) return MOE_ERR_UNSUPPORTED;
     if (rows == 0) return MOE_OK;
-    if (x == nullptr || q == nullptr) return MOE_ERR_INVALID_ARG;
+    if (x == nullptr || q == nullptr || !aligned16(x) || !aligned16(q)) return MOE_ERR_INVALID_ARG;
     if (!device_ok()) return MOE_ERR_UNSUPPORTED;
     return cuda_status(launch_quant_act_fp8_static(x, nullptr, 0, 1, rows, cols, scale, q,
                                                    as_stream(stream)));
@@ -485,7 +496,8 @@ moe_status moe_quantize_act_fp8_static_permuted(const uint16_t* x, const int32_t
     if (T < 0 || k <= 0 || d <= 0 || !(scale > 0.0f) || !isfinite(scale)) return MOE_ERR_INVALID_ARG;
     if (d % 8 != 0 || (int64_t)T * k + T >= ((int64_t)1 << 31)) return MOE_ERR_UNSUPPORTED;
     if (T == 0) return MOE_OK;
-    if (x == nullptr || perm == nullptr || q == nullptr) return MOE_ERR_INVALID_ARG;
+    if (x == nullptr || perm == nullptr || q == nullptr || !aligned16(x) || !aligned16(q))
+        return MOE_ERR_INVALID_ARG;
     if (!device_ok()) return MOE_ERR_UNSUPPORTED;
     const int64_t R = (int64_t)T * k + (with_shared ? T : 0);
     return cuda_status(launch_quant_act_fp8_static(x, perm, T, k, R, d, scale, q, as_stream(stream)));
@@ -496,7 +508,8 @@ moe_status moe_quantize_weights_mxfp8(const uint16_t* W, int64_t batch, int32_t 
     if (batch < 0 || rows < 0 || cols < 0) return MOE_ERR_INVALID_ARG;
     if (cols % 128 != 0 || rows % 128 != 0) return MOE_ERR_UNSUPPORTED;
     if (batch * rows * (int64_t)cols == 0) return MOE_OK;
-    if (W == nullptr || q == nullptr || scale == nullptr) return MOE_ERR_INVALID_ARG;
+    if (W == nullptr || q == nullptr || scale == nullptr || !aligned16(W) || !aligned16(q))
+        return MOE_ERR_INVALID_ARG;
     if (!device_ok()) return MOE_ERR_UNSUPPORTED;
     return cuda_status(launch_quant_mx_weights(W, batch, rows, cols, q, scale, as_stream(stream)));
 }
@@ -506,7 +519,8 @@ moe_status moe_quantize_act_mxfp8(const uint16_t* x, int64_t rows, int32_t cols,
     if (rows < 0 || cols <= 0) return MOE_ERR_INVALID_ARG;
     if (cols % 128 != 0) return MOE_ERR_UNSUPPORTED;
     if (rows == 0) return MOE_OK;
-    if (x == nullptr || q == nullptr || scale == nullptr) return MOE_ERR_INVALID_ARG;
+    if (x == nullptr || q == nullptr || scale == nullptr || !aligned16(x) || !aligned16(q))
+        return MOE_ERR_INVALID_ARG;
     if (!device_ok()) return MOE_ERR_UNSUPPORTED;
     return cuda_status(launch_quant_mx_rows(x, rows, cols, q, scale, as_stream(stream)));
 }
@@ -517,7 +531,9 @@ moe_status moe_quantize_act_mxfp8_permuted(const uint16_t* x, const int32_t* per
     if (T < 0 || k <= 0 || d <= 0) return MOE_ERR_INVALID_ARG;
     if (d % 128 != 0 || (int64_t)T * k + T >= ((int64_t)1 << 31)) return MOE_ERR_UNSUPPORTED;
     if (T == 0) return MOE_OK;
-    if (x == nullptr || perm == nullptr || q == nullptr || scale == nullptr) return MOE_ERR_INVALID_ARG;
+    if (x == nullptr || perm == nullptr || q == nullptr || scale == nullptr || !aligned16(x) ||
+        !aligned16(q))
+        return MOE_ERR_INVALID_ARG;
     if (!device_ok()) return MOE_ERR_UNSUPPORTED;
     return cuda_status(launch_quant_mx_permuted(x, perm, T, k, with_shared ? 1 : 0, d, q, scale,
                                                 as_stream(stream)));
@@ -529,7 +545,9 @@ moe_status moe_quantize_act_fp8_permuted(const uint16_t* x, const int32_t* perm,
     if (T < 0 || k <= 0 || d <= 0) return MOE_ERR_INVALID_ARG;
     if (d % 128 != 0 || (int64_t)T * k + T >= ((int64_t)1 << 31)) return MOE_ERR_UNSUPPORTED;
     if (T == 0) return MOE_OK;
-    if (x == nullptr || perm == nullptr || q == nullptr || scale == nullptr) return MOE_ERR_INVALID_ARG;
+    if (x == nullptr || perm == nullptr || q == nullptr || scale == nullptr || !aligned16(x) ||
+        !aligned16(q))
+        return MOE_ERR_INVALID_ARG;
     if (!device_ok()) return MOE_ERR_UNSUPPORTED;
     return cuda_status(launch_quant_act_fp8_permuted(x, perm, T, k, with_shared ? 1 : 0, d, q, scale,
                                                      as_stream(stream)));
@@ -541,7 +559,9 @@ moe_status moe_router_logits(const uint16_t* x, const uint16_t* hi, const uint16
     if (T < 0 || d <= 0 || E <= 0) return MOE_ERR_INVALID_ARG;
     if (d % 128 != 0 || E > 256) return MOE_ERR_UNSUPPORTED;
     if (T == 0) return MOE_OK;
-    if (x == nullptr || hi == nullptr || lo == nullptr || logits == nullptr) return MOE_ERR_INVALID_ARG;
+    if (x == nullptr || hi == nullptr || lo == nullptr || logits == nullptr || !aligned16(x) ||
+        !aligned16(hi) || !aligned16(lo) || !aligned16(logits))
+        return MOE_ERR_INVALID_ARG;
     if (!device_ok()) return MOE_ERR_UNSUPPORTED;
     return cuda_status(launch_router_logits(x, hi, lo, bias, logits, T, d, E, nullptr,
                                             as_stream(stream)));
@@ -584,7 +604,7 @@ moe_status moe_gemm_gateup(const moe_shape* shape, const moe_weights* weights, c
     const bool fp8 = shape->wdtype != MOE_WDTYPE_BF16;  // permuted e4m3 rows
     const bool scaled = fp8 && shape->wdtype != MOE_WDTYPE_FP8_TENSOR;  // per-row scales
     if (x == nullptr || offsets == nullptr || h == nullptr || (!fp8 && perm == nullptr) ||
-        (scaled && (x_scale == nullptr || h_scale == nullptr)))
+        (scaled && (x_scale == nullptr || h_scale == nullptr)) || !aligned16(x) || !aligned16(h))
         return MOE_ERR_INVALID_ARG;
     if ((r = check_ws(ws, ws_bytes, kWsHeader)) != MOE_OK) return r;
     if (!device_ok()) return MOE_ERR_UNSUPPORTED;
@@ -602,7 +622,8 @@ moe_status moe_gemm_down(const moe_shape* shape, const moe_weights* weights, con
     if ((r = check_weights(shape, weights, false, true, false)) != MOE_OK) return r;
     if (shape->T == 0) return MOE_OK;
     const bool scaled = shape->wdtype == MOE_WDTYPE_FP8_BLOCK128 || shape->wdtype == MOE_WDTYPE_MXFP8;
-    if (h == nullptr || offsets == nullptr || o == nullptr || (scaled && h_scale == nullptr))
+    if (h == nullptr || offsets == nullptr || o == nullptr || (scaled && h_scale == nullptr) ||
+        !aligned16(h) || !aligned16(o))
         return MOE_ERR_INVALID_ARG;
     if ((r = check_ws(ws, ws_bytes, kWsHeader)) != MOE_OK) return r;
     if (!device_ok()) return MOE_ERR_UNSUPPORTED;
@@ -617,7 +638,9 @@ moe_status moe_combine(const moe_shape* shape, const void* o, const int32_t* inv
     moe_status r = check_shape(shape);
     if (r != MOE_OK) return r;
     if (shape->T == 0) return MOE_OK;
-    if (o == nullptr || inv == nullptr || w == nullptr || y == nullptr) return MOE_ERR_INVALID_ARG;
+    if (o == nullptr || inv == nullptr || w == nullptr || y == nullptr || !aligned16(o) ||
+        !aligned16(y))
+        return MOE_ERR_INVALID_ARG;
     if (!device_ok()) return MOE_ERR_UNSUPPORTED;
     return cuda_status(launch_combine(static_cast<const __half*>(o), inv, w, y, shape->T, shape->d,
                                       shape->k, shape->I_shared > 0 ? 1 : 0, as_stream(stream)));
@@ -629,7 +652,7 @@ moe_status moe_forward(const moe_shape* shape, const moe_weights* weights, const
     if (r != MOE_OK) return r;
     if ((r = check_weights(shape, weights, true, true, true)) != MOE_OK) return r;
     if (shape->T == 0) return MOE_OK;
-    if (x == nullptr || y == nullptr) return MOE_ERR_INVALID_ARG;
+    if (x == nullptr || y == nullptr || !aligned16(x) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
     if ((r = check_ws(ws, ws_bytes, ws_layout(*shape).total)) != MOE_OK) return r;
     if (!device_ok()) return MOE_ERR_UNSUPPORTED;
     return forward_device(shape, weights, x, y, ws, as_stream(stream));
@@ -645,7 +668,7 @@ moe_status moe_forward_profiled(const moe_shape* shape, const moe_weights* weigh
     if (r != MOE_OK) return r;
     if ((r = check_weights(shape, weights, true, true, true)) != MOE_OK) return r;
     if (shape->T == 0) return MOE_OK;
-    if (x == nullptr || y == nullptr) return MOE_ERR_INVALID_ARG;
+    if (x == nullptr || y == nullptr || !aligned16(x) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
     if ((r = check_ws(ws, ws_bytes, ws_layout(*shape).total)) != MOE_OK) return r;
     if (!device_ok()) return MOE_ERR_UNSUPPORTED;
     return forward_device(shape, weights, x, y, ws, as_stream(stream), events);
@@ -723,8 +746,7 @@ moe_status moe_calibrate_fp8_static(const moe_shape* shape, const moe_weights* w
     if (r != MOE_OK) return r;
     if (shape->wdtype != MOE_WDTYPE_BF16) return MOE_ERR_UNSUPPORTED;
     if ((r = check_weights(shape, weights, true, false, true)) != MOE_OK) return r;
-    if (shape->T == 0 || x == nullptr || scales == nullptr ||
-        (reinterpret_cast<uintptr_t>(x) & 15u) != 0)
+    if (shape->T == 0 || x == nullptr || scales == nullptr || !aligned16(x))
         return MOE_ERR_INVALID_ARG;
     const WsLayout L = ws_layout(*shape);
     if ((r = check_ws(ws, ws_bytes, L.total)) != MOE_OK) return r;
@@ -752,7 +774,7 @@ moe_status moe_route(const moe_shape* shape, const moe_weights* weights, const u
         return MOE_ERR_UNSUPPORTED;
     if ((r = check_weights(shape, weights, false, false, true)) != MOE_OK) return r;
     if (shape->T == 0) return MOE_OK;
-    if (x == nullptr) return MOE_ERR_INVALID_ARG;
+    if (x == nullptr || !aligned16(x)) return MOE_ERR_INVALID_ARG;
     const WsLayout L = ws_layout(*shape);
     if ((r = check_ws(ws, ws_bytes, L.total)) != MOE_OK) return r;
     if (!device_ok()) return MOE_ERR_UNSUPPORTED;
@@ -835,8 +857,6 @@ moe_status moe_peer_buffer_free(void* ptr) {
 }
 
 namespace {
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
 moe_status check_ar(int32_t G, int32_t T_max, int32_t T, int32_t d, const void* gamma) {
     if (G < 1 || T < 0 || T_max < 0 || d <= 0) return MOE_ERR_INVALID_ARG;
     if (G > kArMaxRanks || d % 8 != 0 || d > allreduce_norm_max_d() || T > T_max)

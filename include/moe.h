@@ -30,9 +30,14 @@
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *    stream).  Work is enqueued asynchronously in stream order; nothing
  *    reads back counts, so a forward can be captured in a CUDA graph.
+ *  - Row buffers (x, y, h, o, logits, FP8 codes q) and weight matrices
+ *    (w_gu, w_d, ws_gu, ws_d, router_hi, router_lo, and the W of the weight
+ *    quantisers) start on a 16-byte boundary: the kernels read them by TMA
+ *    or with 16-byte vector accesses.  The workspace starts on a 256-byte
+ *    boundary.
  *  - Arguments are validated on the host before any launch.  A failed check
- *    returns MOE_ERR_INVALID_ARG (null pointer, negative size, bad
- *    workspace alignment) or MOE_ERR_UNSUPPORTED (a shape outside the
+ *    returns MOE_ERR_INVALID_ARG (null pointer, negative size, a pointer
+ *    off the alignment above) or MOE_ERR_UNSUPPORTED (a shape outside the
  *    limits below, or no sm_100 device); nothing is launched then.  There is
  *    no fallback path.  T == 0 is a valid no-op.
  *  - Shape limits: d % 128 == 0, I % 128 == 0, I_shared in {0, I},

@@ -93,3 +93,41 @@ def test_workspace_map_regions(lib):
     assert regs["xq"] > 0 and regs["xs"] == 0
     nxt = min([off for off in regs.values() if off > regs["xq"]] + [m.total])
     assert nxt - regs["xq"] == T * k * d * 2
+
+
+def test_misaligned_pointers_are_rejected_on_the_host(lib):
+    # every case below is refused before any device work, so nothing is launched
+    # (row buffers and weight matrices must start on a 16-byte boundary)
+    from expert_layer_dual_b200 import moe as M
+    V = ctypes.c_void_p
+    s = M.moe_shape(16, 256, 8, 2, 128, 0, 0, 1)
+    good = [V(256)] * 10 + [None]
+    w = M.moe_weights(*good)
+    nb = M.workspace_bytes(s)
+    ws = V(1 << 20)
+    for bad_x, bad_y in ((V(1024 + 2), V(2048)), (V(1024), V(2048 + 8))):
+        assert lib.moe_forward(ctypes.byref(s), ctypes.byref(w), bad_x, bad_y, ws, nb, None) == M.INVALID_ARG
+    for i in range(10):
+        if i in (2, 3, 6, 7):   # scale arrays: no alignment rule
+            continue
+        fields = list(good)
+        fields[i] = V(256 + 4)
+        wb = M.moe_weights(*fields)
+        assert lib.moe_forward(ctypes.byref(s), ctypes.byref(wb), V(1024), V(2048), ws, nb, None) == \
+            M.INVALID_ARG, i
+    assert lib.moe_combine(ctypes.byref(s), V(1024 + 2), V(4096), V(8192), V(2048), None) == M.INVALID_ARG
+    assert lib.moe_combine(ctypes.byref(s), V(1024), V(4096), V(8192), V(2048 + 2), None) == M.INVALID_ARG
+    assert lib.moe_router_logits(V(1024 + 2), V(256), V(512), None, V(2048), 16, 256, 8, None) == M.INVALID_ARG
+    assert lib.moe_quantize_act_fp8(V(1024 + 2), ctypes.c_int64(16), 256, V(2048), V(4096), None) == \
+        M.INVALID_ARG
+    assert lib.moe_quantize_act_fp8(V(1024), ctypes.c_int64(16), 256, V(2048 + 1), V(4096), None) == \
+        M.INVALID_ARG
+    # the same calls with aligned pointers pass the host checks; without a GPU they
+    # stop at the device check (only run where no GPU could launch anything)
+    import torch
+    if not torch.cuda.is_available():
+        assert lib.moe_forward(ctypes.byref(s), ctypes.byref(w), V(1024), V(2048), ws, nb, None) == \
+            M.UNSUPPORTED
+        assert lib.moe_combine(ctypes.byref(s), V(1024), V(4096), V(8192), V(2048), None) == M.UNSUPPORTED
+        assert lib.moe_quantize_act_fp8(V(1024), ctypes.c_int64(16), 256, V(2048), V(4096), None) == \
+            M.UNSUPPORTED
