@@ -1051,7 +1051,8 @@ cudaError_t launch_quant_act_fp8_static_scatter(const uint16_t* x, const int32_t
 // x copied into the grouped GEMMs' permuted row order, token-major (bf16
 // rows; the CTA-pair gate-up then loads its A rows as TMA tiles): a warp per
 // 1024 columns of a token reads them once and stores them to each of the
-// token's k (+1) permuted rows.
+// token's k (+1) permuted rows.  The forward copies the routed rows only
+// (has_shared = 0): the pair gate-up reads the shared expert's rows from x.
 __global__ void __launch_bounds__(256)
     k_permute_rows_scatter(const uint16_t* __restrict__ x, const int32_t* __restrict__ inv, int T,
                            int k, int has_shared, int cols, uint16_t* __restrict__ xp) {
